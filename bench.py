@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of the SemKV mixed-precision KV-cache hot path on B200.
+
+One step = one pass of the whole hot path over one layer of synthetic input: precision
+assignment (semkv_assign_precision), affine quantization + radix packing of the prefill
+(semkv_quantize_pack) and one GQA decode step over the packed cache (semkv_decode_attention).
+Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32768 cached tokens, 8 KV heads,
+32 query heads, head_dim 128, group 64, L_hi 8 / L_lo 5, p 0.25.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl semkv|reference]
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload on its own data (independent
+units, no collective on the data path: weak scaling); the time is the max over ranks.
+Throughput unit: GB/s of algorithmic bytes (the bytes the method must move: fp16 K/V read once,
+packed codes + fp16 scale/zero written and read once, scores, queries, bitmap/rank).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn HBM GB/s & %roofline over packed mixed-precision KV; quantize GB/s"
+L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["semkv", "reference"], default="semkv")
+    ap.add_argument("--workload", default="llama8b_1L")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true", help="few steps, no clocks/e2e/cpu legs (for ncu)")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+
+
+def radix_words(L: int, n: int = 128) -> int:
+    k = 0
+    p = 1
+    while p * L <= 2 ** 32:
+        p *= L
+        k += 1
+    return -(-n // k)
+
+
+def alg_bytes(w, T: int, n_hi: int) -> dict:
+    """Algorithmic bytes of one layer, per hot-path step (measurement)."""
+    units = w.B * w.H
+    ng = w.D // w.G
+    rec = lambda L: 2 * (4 * radix_words(L, w.D) + 4 * ng)  # noqa: E731  K + V record of one token
+    cache = units * (n_hi * rec(w.L_hi) + (T - n_hi) * rec(w.L_lo))
+    bitmap_rank = units * 2 * 4 * ((T + 31) // 32)
+    q = w.B * w.Hq * w.D * 2
+    return {
+        "select": units * 4 * T + bitmap_rank,
+        "quantize": units * T * w.D * 2 * 2 + bitmap_rank + cache,
+        "decode": cache + q,
+        "cache": cache,
+    }
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+
+_SAMPLE_INPUTS = {}
+
+
+def oracle_sample(w, seconds_target: float = 15.0, max_units: int = 8):
+    """Time the oracle on a bounded sample of the workload: whole units (one (b, kv-head) of one
+    layer each: select + quantize/pack + fp64 attention), as many as fit the time target.
+    Input generation is not timed."""
+    import numpy as np
+
+    import oracle
+    from mixed_precision_kv_semkv_b200 import synth
+
+    if w.name not in _SAMPLE_INPUTS:
+        _SAMPLE_INPUTS[w.name] = synth.layer_cpu(w, 0, B=1)
+    d = _SAMPLE_INPUTS[w.name]
+    g = w.Hq // w.H
+    T = w.T
+    n_hi = oracle.n_hi(w.p, T)
+    tiles_hi, tiles_lo = max(1, -(-n_hi // 128)), max(1, -(-(T - n_hi) // 128))
+    done, t0 = 0, time.perf_counter()
+    while done < min(max_units, w.H):
+        h = done
+        bm, rk, nh, tau, _ = oracle.select(d["scores"][0, h], w.p)
+        hi, lo, _ = oracle.quantize_pack_unit(d["K"][0, h].view(np.uint16), d["V"][0, h].view(np.uint16), bm, w.G,
+                                              w.L_hi, w.L_lo, tiles_hi, tiles_lo)
+        Kh, Vh = oracle.dequantize_unit(T, w.D, w.G, w.L_hi, w.L_lo, bm, hi, lo)
+        oracle.attention_fp64(d["q"][0, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, synth.sm_scale())
+        done += 1
+        if time.perf_counter() - t0 > seconds_target:
+            break
+    el = time.perf_counter() - t0
+    per_unit = alg_bytes(w, T, n_hi)
+    units_layer = w.B * w.H
+    step_bytes = (per_unit["select"] + per_unit["quantize"] + per_unit["decode"]) / units_layer * done
+    return {"seconds": el, "units": done, "bytes": step_bytes, "gbs": step_bytes / el / 1e9,
+            "sample": f"{done} unit(s) (one batch row x kv head each, T={T}) of workload {w.name}: select + "
+                      f"quantize/pack + dequantize + fp64 attention, oracle as it stands, 1 thread"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from mixed_precision_kv_semkv_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    steps = max(1, min(args.steps, 3))
+    warm = max(0, min(args.warmup, 1))
+    for _ in range(warm):
+        oracle_sample(w, seconds_target=0.0, max_units=1)
+    secs, byts = 0.0, 0.0
+    for _ in range(steps):
+        r = oracle_sample(w, seconds_target=0.0, max_units=1)
+        secs += r["seconds"]
+        byts += r["bytes"]
+    gbs = byts / secs / 1e9
+    line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+            "ms_per_step": secs / steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Hq": w.Hq, "T": w.T, "G": w.G, "L_hi": w.L_hi,
+                       "L_lo": w.L_lo, "p": w.p, "sample": "1 unit per step"},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def run_semkv(args):
+    import torch
+
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_assign_precision, semkv_decode_attention,
+                                               semkv_quantize_pack, synth)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    build.build()
+    w = synth.WORKLOADS[args.workload]
+    T = w.T
+    d = synth.layer_gpu(w, seed=rank)
+    K, V, S, q = d["K"], d["V"], d["scores"], d["q"]
+    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p)
+    ws = cache.workspace()
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    scale = synth.sm_scale(w.D)
+    from mixed_precision_kv_semkv_b200.cache import n_hi_for
+
+    nb = alg_bytes(w, T, n_hi_for(w.p, T))
+    step_bytes = nb["select"] + nb["quantize"] + nb["decode"]
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        semkv_assign_precision(cache, S, T, w.p, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        semkv_quantize_pack(cache, K, V, T, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        semkv_decode_attention(cache, q, scale, out, ws, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    steps = 3 if args.profile else args.steps
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert cache.status() == 0, f"device status {cache.status()}"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    clocks = Clocks(local)
+    if not args.profile:
+        clocks.start()
+        time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()  # L2 flush between steps, outside the step's events
+        step(evs[i])
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ck = clocks.stop() if not args.profile else {}
+    t_sel = sum(e[0].elapsed_time(e[1]) for e in evs)
+    t_q = sum(e[1].elapsed_time(e[2]) for e in evs)
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in evs)
+    total_ms = t_sel + t_q + t_dec
+    if dist is not None:
+        tt = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    value = world * step_bytes * steps / (total_ms * 1e-3) / 1e9
+
+    # decode alone over an L2-cold cache (decode-attn HBM GB/s of the metric)
+    dec_ms = []
+    for _ in range(min(steps, 200)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        semkv_decode_attention(cache, q, scale, out, ws, stream=stream)
+        e1.record(stream)
+        dec_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    dec_cold = sum(a.elapsed_time(b) for a, b in dec_ms) / len(dec_ms)
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        pass
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_note = "measured" if "hbm_gbs" in peaks else "fallback"
+    per_kernel = {
+        "select": {"ms": t_sel / steps, "gbs": nb["select"] / (t_sel / steps * 1e-3) / 1e9},
+        "quantize": {"ms": t_q / steps, "gbs": nb["quantize"] / (t_q / steps * 1e-3) / 1e9},
+        "decode_in_step": {"ms": t_dec / steps, "gbs": nb["decode"] / (t_dec / steps * 1e-3) / 1e9},
+        "decode_l2_cold": {"ms": dec_cold, "gbs": nb["decode"] / (dec_cold * 1e-3) / 1e9},
+    }
+    dom = max(("select", "quantize", "decode_in_step"), key=lambda k: per_kernel[k]["ms"])
+    dom_name = {"select": "semkv_assign_precision (k_select)", "quantize": "semkv_quantize_pack (k_quantize)",
+                "decode_in_step": "semkv_decode_attention (k_decode_split + k_decode_merge)"}[dom]
+    ach = per_kernel[dom]["gbs"]
+    traffic = None
+    try:
+        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        traffic = prof.get(dom)
+    except (OSError, ValueError):
+        pass
+
+    e2e = None
+    if not args.no_e2e and not args.profile:
+        hK, hV, hS, hq = (t.cpu().pin_memory() for t in (K, V, S, q))
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        e2e_steps = min(steps, 20)
+        el = 0.0
+        for i in range(e2e_steps + 2):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            S.copy_(hS, non_blocking=True)
+            q.copy_(hq, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= 2:
+                el += e0.elapsed_time(e1)
+        h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hS, hq))
+        e2e = {"value": world * step_bytes * e2e_steps / (el * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * 4,
+               "ms_per_step": el / e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
+        r = oracle_sample(w)
+        cpu = {"value": r["gbs"], "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": r["sample"]}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warm,
+        "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u32-packed codes, fp32 math", "data": "synthetic",
+        "config": {"workload": f"{w.name}: Llama-3.1-8B-shaped layer, B{w.B} H{w.H} Hq{w.Hq} T{T} D{w.D}, "
+                               f"G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}",
+                   "l2": "flushed between steps (512 MB write)", "parallelism": f"dp{world} (independent units)",
+                   "step": "assign_precision + quantize_pack + decode_attention"},
+        "per_kernel": per_kernel,
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": ach / hbm_peak, "peak_kind": peak_note, "traffic": traffic,
+                     "frac_of_8000": ach / 8000.0},
+        "decode_roofline": {"achieved": per_kernel["decode_l2_cold"]["gbs"], "peak": hbm_peak,
+                            "frac": per_kernel["decode_l2_cold"]["gbs"] / hbm_peak,
+                            "frac_of_8000": per_kernel["decode_l2_cold"]["gbs"] / 8000.0},
+        "clocks": ck, "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 6 * steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_semkv(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * semkv.h -- C ABI of libsemkv: the hot path of SemKV-style semantic mixed-precision KV-cache
+ * quantization on NVIDIA B200 (sm_100a).
+ *
+ * The method is the one stated in the Abstract of the page "SemKV: Semantic Mixed-Precision KV
+ * Cache Quantization Guided by the Quality Cliff for Long-Context LLM Inference" (arXiv
+ * 2608.28911v1): every cached token is kept; tokens are ordered by an importance score taken from
+ * inside the model; a fraction p of them is stored on the finer of two neighbouring uniform grids
+ * (L_hi levels) and the rest on the coarser one (L_lo levels), both above the quality cliff; the
+ * level counts need not be powers of two (5 levels = 2.322 code bits per value), so the average
+ * precision interpolates between the two grids.  The Abstract also reports the cliff when tokens
+ * are quantized during generation, which is what semkv_append_token does.  Decode attention over
+ * the compressed cache is the consumer; the KVQuant blog page (section on the memory bottleneck)
+ * notes that for long sequences the KV cache is the dominant memory traffic of decoding.
+ *
+ * Conventions for every entry point
+ *   - All array pointers are DEVICE pointers (cudaMalloc'd or torch tensors), owned by the caller.
+ *     The library allocates nothing and never synchronizes; work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - fp16 data are IEEE binary16 bit patterns (uint16_t).  Scores are IEEE binary32.
+ *   - The return value is a host-side status (SEMKV_OK or SEMKV_ERR_*), known before any launch
+ *     except SEMKV_ERR_CUDA (launch failure).  Problems only the device can see (NaN score,
+ *     non-finite K/V, append past capacity) are OR-ed into the device word *status as
+ *     SEMKV_STATUS_* bits; the caller reads it when it chooses.  No kernel traps or asserts.
+ *   - A "unit" is one (batch row b, kv head h) pair, u = b*H + h.  Units are independent.
+ *
+ * Data layout of one layer's cache (all uint32 words; tile = 128 slots of one segment):
+ *   k_seg   [B*H][cap_seg/128][WK][128]   K codes of one token row, base-L radix words:
+ *                                          word j holds channels j*k .. j*k+k-1 of the slot,
+ *                                          value sum_i code_i * L^i  (k = max{k: L^k <= 2^32},
+ *                                          WK = ceil(D/k); channels past D are zero digits)
+ *   v_seg   [B*H][cap_seg/128][WV][D]     V codes of one channel, packed along the slots of a
+ *                                          tile: word w of channel d holds slots w*k .. w*k+k-1,
+ *                                          value sum_i code_i * L^i  (WV = ceil(128/k))
+ *   kz_seg, vz_seg [B*H][cap_seg/128][D/G][128]   per (slot, channel group): fp16 scale in the
+ *                                          low half, fp16 zero in the high half
+ *   bitmap  [B*H][T_cap/32]  bit t%32 of word t/32 = 1 iff token t is on the L_hi grid
+ *   rank    [B*H][T_cap/32]  rank[w] = number of L_hi tokens in words 0..w-1 (valid for words
+ *                            that hold at least one token)
+ *   n_hi, n_lo [B*H] int32   tokens in each segment (a token's slot is its rank in its class)
+ *   tau     [B*H] float      precision threshold of the unit (the n_hi-th largest score)
+ *   status  [1] int32        device status word (SEMKV_STATUS_* bits)
+ * Code c of value x on a group with scale s and zero z dequantizes to fmaf((float)c, s, z).
+ */
+#ifndef SEMKV_H
+#define SEMKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SEMKV_API __attribute__((visibility("default")))
+#else
+#define SEMKV_API
+#endif
+
+#define SEMKV_TILE 128
+
+/* host-side return codes */
+#define SEMKV_OK 0
+#define SEMKV_ERR_INVALID_ARG 1 /* null pointer, bad shape (Hq % H, D % G, T > T_cap, p outside [0,1]) */
+#define SEMKV_ERR_UNSUPPORTED 2 /* D != 128, L outside [2, 256], G not in {8,16,32,64,128}, Hq/H > 8 */
+#define SEMKV_ERR_CAPACITY 3    /* the host can already see that a segment or T_cap is too small */
+#define SEMKV_ERR_CUDA 4        /* a kernel launch failed (cudaGetLastError) */
+
+/* device status word bits */
+#define SEMKV_STATUS_NAN_SCORE 1       /* a score was NaN: its place in the order is unspecified */
+#define SEMKV_STATUS_NONFINITE_KV 2    /* a K or V value was inf/NaN: its codes are unspecified */
+#define SEMKV_STATUS_APPEND_OVERFLOW 4 /* an appended token found its segment (or T_cap) full and
+                                          was dropped; that unit's state is unchanged */
+#define SEMKV_STATUS_LENGTH_MISMATCH 8 /* semkv_dequantize: a unit's n_hi + n_lo != T */
+
+/* One layer's packed cache.  Shape fields are set by the caller; the pointers are device
+ * buffers of the sizes semkv_cache_bytes() reports, in the order of the SEMKV_BUF_* indices. */
+typedef struct semkv_cache {
+    int32_t B, H, Hq, D, G; /* batch, kv heads, query heads (GQA group g = Hq/H), head dim, group */
+    int32_t L_hi, L_lo;     /* level counts of the two grids (L_hi is used for the top fraction p) */
+    int32_t cap_hi, cap_lo; /* slot capacity of each segment per unit, multiples of 128 */
+    int32_t T_cap;          /* token capacity per unit (bitmap/rank length), multiple of 32 */
+    uint32_t *k_hi, *v_hi, *kz_hi, *vz_hi;
+    uint32_t *k_lo, *v_lo, *kz_lo, *vz_lo;
+    uint32_t *bitmap, *rank;
+    int32_t *n_hi, *n_lo;
+    float *tau;
+    int32_t *status;
+} semkv_cache_t;
+
+enum {
+    SEMKV_BUF_K_HI = 0, SEMKV_BUF_V_HI, SEMKV_BUF_KZ_HI, SEMKV_BUF_VZ_HI,
+    SEMKV_BUF_K_LO, SEMKV_BUF_V_LO, SEMKV_BUF_KZ_LO, SEMKV_BUF_VZ_LO,
+    SEMKV_BUF_BITMAP, SEMKV_BUF_RANK, SEMKV_BUF_N_HI, SEMKV_BUF_N_LO, SEMKV_BUF_TAU, SEMKV_BUF_STATUS,
+    SEMKV_NBUF
+};
+
+/* Byte size of each of the SEMKV_NBUF buffers of a cache with the shape fields of `shape`
+ * (pointers ignored).  Pure host function.  Returns SEMKV_OK or a validation error. */
+SEMKV_API int semkv_cache_bytes(const semkv_cache_t* shape, size_t sizes[SEMKV_NBUF]);
+
+/* Bytes of device workspace semkv_decode_attention needs for this shape on the current device
+ * (it depends on the device's SM count, which sets the split-K factor). */
+SEMKV_API int semkv_workspace_bytes(const semkv_cache_t* shape, size_t* bytes);
+
+/* Precision assignment (SemKV page, Abstract: tokens ranked by an internal score; the top fraction
+ * gets the finer of two neighbouring grids).  scores: device fp32 [B][H][T].  For every unit:
+ * n_hi = floor(p*T) (p in [0,1], computed in double); the n_hi tokens with the largest scores
+ * (equal scores: lower token index first; -0 == +0) get bit 1 in the bitmap; rank[] is filled;
+ * n_lo = T - n_hi; tau = the n_hi-th largest score (+inf if n_hi = 0).  Requires T <= T_cap,
+ * n_hi <= cap_hi and T - n_hi <= cap_lo (else SEMKV_ERR_CAPACITY).  NaN scores set
+ * SEMKV_STATUS_NAN_SCORE.  Bitmap words past the last token are cleared. */
+SEMKV_API int semkv_assign_precision(const semkv_cache_t* cache, const float* scores, int32_t T, float p,
+                           void* stream);
+
+/* Affine quantization and radix packing of a whole prefill (SemKV page, Abstract: uniform affine
+ * grids with a level count that need not be a power of two).  K, V: device fp16 [B][H][T][D];
+ * semkv_assign_precision must have run for this T.  Per token and group of G channels:
+ * mn, mx = min, max; s = fp16 rounded up of fp32 (mx - mn)/(L - 1) (saturated at 65504);
+ * z = mn; code = clamp(rint((x - z)/s), 0, L - 1) (fp32 subtract and divide, ties to even; 0 if
+ * s = 0).  Codes are packed and placed as described at the top of this file; slots past the
+ * segment's length inside its last tile get zero codes and zero scale/zero.  Non-finite inputs
+ * set SEMKV_STATUS_NONFINITE_KV. */
+SEMKV_API int semkv_quantize_pack(const semkv_cache_t* cache, const uint16_t* K, const uint16_t* V, int32_t T,
+                        void* stream);
+
+/* Quantization at generation time (SemKV page, Abstract): one new token per unit.  k, v: device
+ * fp16 [B][H][D]; score: device fp32 [B][H].  The token is on the L_hi grid iff score > tau of
+ * its unit (strict); it is quantized alone and written at slot n_seg of its segment; bitmap,
+ * rank and n_hi/n_lo advance.  A full segment (or n_hi + n_lo = T_cap) drops the token and sets
+ * SEMKV_STATUS_APPEND_OVERFLOW; a NaN score sets SEMKV_STATUS_NAN_SCORE (the token goes lo). */
+SEMKV_API int semkv_append_token(const semkv_cache_t* cache, const uint16_t* k, const uint16_t* v, const float* score,
+                       void* stream);
+
+/* GQA decode attention over the packed cache.  q: device fp16 [B][Hq][D]; out: device fp32
+ * [B][Hq][D].  Query head qh attends with kv head qh / (Hq/H) over all n_hi + n_lo tokens of its
+ * unit (no mask): out = sum_t softmax_t(softmax_scale * q.k^_t) v^_t with k^, v^ the dequantized
+ * codes (dequantized in registers; the packed words are read once from HBM).  Split-K over token
+ * tiles, then a log-sum-exp merge.  workspace: device buffer of at least
+ * semkv_workspace_bytes() bytes (partial softmax states), contents need not be initialized.
+ * A unit with no tokens gives zeros. */
+SEMKV_API int semkv_decode_attention(const semkv_cache_t* cache, const uint16_t* q, float softmax_scale, float* out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Dequantize every token back to original token order (test and inspection path, not tuned).
+ * K, V: device fp32 [B][H][T][D] outputs; T = n_hi + n_lo of every unit (else
+ * SEMKV_STATUS_LENGTH_MISMATCH and the unit's rows are left as they were). */
+SEMKV_API int semkv_dequantize(const semkv_cache_t* cache, float* K, float* V, int32_t T, void* stream);
+
+/* Name of a host return code (SEMKV_OK ... SEMKV_ERR_CUDA). */
+SEMKV_API const char* semkv_status_string(int code);
+
+/* Radix parameters for L levels: digits per 32-bit word k(L) and words per D-channel row.
+ * Pure host function; returns 0 for L outside [2, 256]. */
+SEMKV_API int32_t semkv_radix_digits(int32_t L);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEMKV_H */

@@ -1,0 +1,19 @@
+"""SemKV-style semantic mixed-precision KV-cache quantization: B200 (sm_100a) hot path.
+
+The compute lives in libsemkv.so (CUDA, C ABI in include/semkv.h); this package is its ctypes
+binding (`_lib`, same function names as the C entry points), a torch-allocated cache holder
+(`cache.SemkvCache`) and the seeded synthetic input generator (`synth`).
+"""
+from ._lib import (  # noqa: F401
+    SemkvError,
+    semkv_append_token,
+    semkv_assign_precision,
+    semkv_cache_bytes,
+    semkv_decode_attention,
+    semkv_dequantize,
+    semkv_quantize_pack,
+    semkv_radix_digits,
+    semkv_workspace_bytes,
+    status_string,
+)
+from .cache import SemkvCache, capacities, n_hi_for  # noqa: F401

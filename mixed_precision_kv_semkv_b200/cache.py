@@ -1,0 +1,79 @@
+"""Device buffers of one layer's packed cache, allocated with torch (plumbing only).
+
+SemkvCache sizes every buffer with semkv_cache_bytes, allocates it on the GPU and fills the
+semkv_cache_t descriptor that the C entry points take.
+"""
+from __future__ import annotations
+
+import math
+
+from . import _lib
+
+
+def n_hi_for(p: float, T: int) -> int:
+    """floor(p*T) with p as a 32-bit float, the count semkv_assign_precision uses."""
+    import numpy as np
+
+    return int(math.floor(float(np.float32(p)) * T))
+
+
+def round_up(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
+def capacities(T: int, p: float, extra: int = 0):
+    """(cap_hi, cap_lo, T_cap) for a prefill of T tokens at fraction p plus `extra` appends."""
+    nh = n_hi_for(p, T)
+    return round_up(nh + extra, 128), round_up(T - nh + extra, 128), round_up(T + extra, 32)
+
+
+class SemkvCache:
+    """One layer's cache: device buffers + the semkv_cache_t descriptor."""
+
+    def __init__(self, B: int, H: int, Hq: int, G: int, L_hi: int, L_lo: int, cap_hi: int, cap_lo: int,
+                 T_cap: int, D: int = 128, device="cuda"):
+        import torch
+
+        self.struct = _lib.CacheStruct(B=B, H=H, Hq=Hq, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=cap_hi,
+                                       cap_lo=cap_lo, T_cap=T_cap)
+        sizes = _lib.semkv_cache_bytes(self.struct)
+        self.sizes = dict(zip(_lib.BUF_NAMES, sizes))
+        self.bufs = {}
+        for name, nbytes in self.sizes.items():
+            dtype = torch.float32 if name == "tau" else torch.int32
+            t = torch.empty(max(nbytes // 4, 1), dtype=dtype, device=device)
+            self.bufs[name] = t
+            setattr(self.struct, name, int(t.data_ptr()))
+        self.bufs["status"].zero_()
+        self.shape = dict(B=B, H=H, Hq=Hq, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=cap_hi, cap_lo=cap_lo,
+                          T_cap=T_cap)
+
+    @classmethod
+    def for_prefill(cls, B, H, Hq, G, L_hi, L_lo, T, p, extra=0, device="cuda"):
+        ch, cl, tc = capacities(T, p, extra)
+        return cls(B, H, Hq, G, L_hi, L_lo, ch, cl, tc, device=device)
+
+    def __getattr__(self, name):
+        shape = self.__dict__.get("shape", {})
+        if name in shape:
+            return shape[name]
+        raise AttributeError(name)
+
+    @property
+    def packed_bytes(self) -> int:
+        """Bytes of the buffers that hold the compressed cache (codes, scales/zeros, bitmap)."""
+        names = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo", "bitmap")
+        return sum(self.sizes[n] for n in names)
+
+    def workspace(self):
+        import torch
+
+        nbytes = _lib.semkv_workspace_bytes(self.struct)
+        return torch.empty(max(nbytes, 4), dtype=torch.uint8, device=self.bufs["status"].device)
+
+    def status(self) -> int:
+        """Read the device status word (synchronizes)."""
+        return int(self.bufs["status"].item())
+
+    def clear_status(self):
+        self.bufs["status"].zero_()

@@ -1,0 +1,222 @@
+// C ABI of libsemkv: argument validation, buffer sizes, split-K choice and kernel launches.
+// Every entry point is documented in include/semkv.h.
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace semkv;
+
+namespace {
+
+constexpr int D_SUPPORTED = 128;
+
+bool level_ok(int L) { return L >= 2 && L <= 256; }
+
+int validate_shape(const semkv_cache_t* c)
+{
+    if (!c) return SEMKV_ERR_INVALID_ARG;
+    if (c->B < 1 || c->H < 1 || c->Hq < 1 || c->D < 1 || c->G < 1) return SEMKV_ERR_INVALID_ARG;
+    if (c->Hq % c->H != 0 || c->D % c->G != 0) return SEMKV_ERR_INVALID_ARG;
+    if (c->cap_hi < 0 || c->cap_lo < 0 || c->cap_hi % TILE || c->cap_lo % TILE) return SEMKV_ERR_INVALID_ARG;
+    if (c->T_cap < 0 || c->T_cap % 32) return SEMKV_ERR_INVALID_ARG;
+    if (c->D != D_SUPPORTED) return SEMKV_ERR_UNSUPPORTED;
+    if (!level_ok(c->L_hi) || !level_ok(c->L_lo)) return SEMKV_ERR_UNSUPPORTED;
+    if (c->G != 8 && c->G != 16 && c->G != 32 && c->G != 64 && c->G != 128) return SEMKV_ERR_UNSUPPORTED;
+    if (c->Hq / c->H > 8) return SEMKV_ERR_UNSUPPORTED;
+    return SEMKV_OK;
+}
+
+int validate_ptrs(const semkv_cache_t* c)
+{
+    const void* p[] = {c->k_hi, c->v_hi, c->kz_hi, c->vz_hi, c->k_lo, c->v_lo, c->kz_lo, c->vz_lo,
+                       c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau, c->status};
+    for (const void* x : p)
+        if (!x) return SEMKV_ERR_INVALID_ARG;
+    return SEMKV_OK;
+}
+
+int validate(const semkv_cache_t* c)
+{
+    int r = validate_shape(c);
+    return r != SEMKV_OK ? r : validate_ptrs(c);
+}
+
+int words_row(int L) { return ceil_div(D_SUPPORTED, radix_k(L)); }
+int words_col(int L) { return ceil_div(TILE, radix_k(L)); }
+
+int sm_count()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 148;
+    }
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+// Split-K factor per segment: about four CTAs per SM over the whole decode, shared between the
+// segments in proportion to their capacity in tiles, at most one split per tile.
+void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
+{
+    const int units = c->B * c->H;
+    const int th = c->cap_hi / TILE, tl = c->cap_lo / TILE, total = th + tl;
+    const long target = 4L * sm_count();
+    auto pick = [&](int tiles) -> int {
+        if (tiles == 0) return 0;
+        long s = (target * tiles + (long)units * total - 1) / ((long)units * total);
+        if (s < 1) s = 1;
+        if (s > tiles) s = tiles;
+        return (int)s;
+    };
+    *ns_hi = pick(th);
+    *ns_lo = pick(tl);
+}
+
+SegView seg_view(const semkv_cache_t* c, bool hi)
+{
+    SegView s;
+    s.k = hi ? c->k_hi : c->k_lo;
+    s.v = hi ? c->v_hi : c->v_lo;
+    s.kz = hi ? c->kz_hi : c->kz_lo;
+    s.vz = hi ? c->vz_hi : c->vz_lo;
+    s.n = hi ? c->n_hi : c->n_lo;
+    s.L = hi ? c->L_hi : c->L_lo;
+    s.tiles_cap = (hi ? c->cap_hi : c->cap_lo) / TILE;
+    s.is_hi = hi ? 1 : 0;
+    return s;
+}
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? SEMKV_OK : SEMKV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t semkv_radix_digits(int32_t L) { return level_ok(L) ? radix_k(L) : 0; }
+
+int semkv_cache_bytes(const semkv_cache_t* c, size_t sizes[SEMKV_NBUF])
+{
+    int r = validate_shape(c);
+    if (r != SEMKV_OK) return r;
+    if (!sizes) return SEMKV_ERR_INVALID_ARG;
+    const size_t units = (size_t)c->B * c->H, ng = (size_t)(c->D / c->G);
+    const size_t th = (size_t)c->cap_hi / TILE, tl = (size_t)c->cap_lo / TILE;
+    sizes[SEMKV_BUF_K_HI] = units * th * words_row(c->L_hi) * TILE * 4;
+    sizes[SEMKV_BUF_V_HI] = units * th * words_col(c->L_hi) * c->D * 4;
+    sizes[SEMKV_BUF_KZ_HI] = units * th * ng * TILE * 4;
+    sizes[SEMKV_BUF_VZ_HI] = sizes[SEMKV_BUF_KZ_HI];
+    sizes[SEMKV_BUF_K_LO] = units * tl * words_row(c->L_lo) * TILE * 4;
+    sizes[SEMKV_BUF_V_LO] = units * tl * words_col(c->L_lo) * c->D * 4;
+    sizes[SEMKV_BUF_KZ_LO] = units * tl * ng * TILE * 4;
+    sizes[SEMKV_BUF_VZ_LO] = sizes[SEMKV_BUF_KZ_LO];
+    sizes[SEMKV_BUF_BITMAP] = units * (size_t)(c->T_cap / 32) * 4;
+    sizes[SEMKV_BUF_RANK] = sizes[SEMKV_BUF_BITMAP];
+    sizes[SEMKV_BUF_N_HI] = units * 4;
+    sizes[SEMKV_BUF_N_LO] = units * 4;
+    sizes[SEMKV_BUF_TAU] = units * 4;
+    sizes[SEMKV_BUF_STATUS] = 4;
+    return SEMKV_OK;
+}
+
+int semkv_workspace_bytes(const semkv_cache_t* c, size_t* bytes)
+{
+    int r = validate_shape(c);
+    if (r != SEMKV_OK) return r;
+    if (!bytes) return SEMKV_ERR_INVALID_ARG;
+    int nh, nl;
+    decode_splits(c, &nh, &nl);
+    *bytes = (size_t)c->B * c->H * (size_t)(nh + nl) * (c->Hq / c->H) * (c->D + 2) * sizeof(float);
+    return SEMKV_OK;
+}
+
+int semkv_assign_precision(const semkv_cache_t* c, const float* scores, int32_t T, float p, void* stream)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (T < 0 || T > c->T_cap || !(p >= 0.0f && p <= 1.0f) || (!scores && T > 0)) return SEMKV_ERR_INVALID_ARG;
+    const int n_hi = (int)std::floor((double)p * (double)T);
+    if (n_hi > c->cap_hi || T - n_hi > c->cap_lo) return SEMKV_ERR_CAPACITY;
+    launch_select(scores, c->B * c->H, T, n_hi, c->T_cap / 32, c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau,
+                  c->status, (cudaStream_t)stream);
+    return launch_status();
+}
+
+int semkv_quantize_pack(const semkv_cache_t* c, const uint16_t* K, const uint16_t* V, int32_t T, void* stream)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (T < 0 || T > c->T_cap || ((!K || !V) && T > 0)) return SEMKV_ERR_INVALID_ARG;
+    if (T == 0) return SEMKV_OK;
+    const int units = c->B * c->H;
+    for (int hi = 1; hi >= 0; --hi)
+        launch_quantize(seg_view(c, hi != 0), K, V, c->bitmap, c->rank, units, T, c->D, c->G, c->T_cap / 32,
+                        c->status, (cudaStream_t)stream);
+    return launch_status();
+}
+
+int semkv_append_token(const semkv_cache_t* c, const uint16_t* k, const uint16_t* v, const float* score,
+                       void* stream)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
+    launch_append(*c, k, v, score, (cudaStream_t)stream);
+    return launch_status();
+}
+
+int semkv_decode_attention(const semkv_cache_t* c, const uint16_t* q, float softmax_scale, float* out,
+                           void* workspace, size_t workspace_bytes, void* stream)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (!q || !out || !std::isfinite(softmax_scale)) return SEMKV_ERR_INVALID_ARG;
+    size_t need = 0;
+    semkv_workspace_bytes(c, &need);
+    if (workspace_bytes < need || (need > 0 && !workspace)) return SEMKV_ERR_INVALID_ARG;
+    int nh, nl;
+    decode_splits(c, &nh, &nl);
+    const int units = c->B * c->H, g = c->Hq / c->H;
+    const float scale_log2 = softmax_scale * 1.4426950408889634f;
+    float* ws = static_cast<float*>(workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    launch_decode_split(seg_view(c, true), q, units, c->H, g, c->D, c->G, scale_log2, nh, 0, nh + nl, ws, st);
+    launch_decode_split(seg_view(c, false), q, units, c->H, g, c->D, c->G, scale_log2, nl, nh, nh + nl, ws, st);
+    launch_decode_merge(ws, units, c->H, g, c->D, nh + nl, out, st);
+    return launch_status();
+}
+
+int semkv_dequantize(const semkv_cache_t* c, float* K, float* V, int32_t T, void* stream)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (T < 0 || T > c->T_cap || ((!K || !V) && T > 0)) return SEMKV_ERR_INVALID_ARG;
+    if (T == 0) return SEMKV_OK;
+    launch_dequantize(*c, T, K, V, (cudaStream_t)stream);
+    return launch_status();
+}
+
+const char* semkv_status_string(int code)
+{
+    switch (code) {
+        case SEMKV_OK: return "SEMKV_OK";
+        case SEMKV_ERR_INVALID_ARG: return "SEMKV_ERR_INVALID_ARG";
+        case SEMKV_ERR_UNSUPPORTED: return "SEMKV_ERR_UNSUPPORTED";
+        case SEMKV_ERR_CAPACITY: return "SEMKV_ERR_CAPACITY";
+        case SEMKV_ERR_CUDA: return "SEMKV_ERR_CUDA";
+        default: return "SEMKV_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

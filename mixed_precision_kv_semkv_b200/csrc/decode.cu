@@ -1,0 +1,273 @@
+// GQA decode attention over the packed mixed-precision cache: split-K partials + LSE merge.
+//
+// The cache is read once: each CTA streams its share of one segment's 128-slot tiles of one
+// unit, unpacks the radix words in registers and folds the per-group scale and zero into the
+// dot products (the KVQuant blog page notes that decoding long sequences is bound by reading the
+// KV cache, so the packed words are the only large traffic).
+//
+// Per tile (4 warps, thread t = slot t for K, thread d = channel d for V):
+//   logit_h(t) = sum_grp [ s_grp * sum_{d in grp} q_hd (c_d - m) + (z_grp + m s_grp) * sum_{d in grp} q_hd ]
+// with m = (L - 1)/2: codes are centred so that the fp32 sums over channels and over tokens do
+// not grow a common offset that would later cancel.  Online softmax in the log2 domain; the
+// tile's probabilities p_h(t) times the V scale go to shared memory; thread d then accumulates
+// sum_t p_h(t) s_V(t) (c_td - m), and the zero terms sum_t p_h(t) (z_V + m s_V) are summed per
+// (group, head).  Each CTA writes (m_h, l_h, o_h[D]) to the workspace; a second kernel merges the
+// splits with log-sum-exp weights.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace semkv {
+
+constexpr int GMAX = 8;  // query heads per kv head supported by this kernel
+
+template <int LC>
+__device__ __forceinline__ void digits_of(uint32_t w, int L, int k, int (&out)[32])
+{
+    if constexpr (LC > 0) {
+        int tmp[Radix<LC>::k];
+        unpack_word<LC>(w, tmp);
+#pragma unroll
+        for (int i = 0; i < Radix<LC>::k; ++i) out[i] = tmp[i];
+    } else {
+        for (int i = 0; i < k; ++i) {
+            out[i] = (int)(w % (uint32_t)L);
+            w /= (uint32_t)L;
+        }
+    }
+}
+
+template <int LC>
+__global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_t* __restrict__ q, int H, int g, int G,
+                                                       float scale_log2, int nsplit, int split_off, int nsplit_total,
+                                                       float* __restrict__ ws)
+{
+    constexpr int D = 128;
+    const int L = LC ? LC : seg.L;
+    const int k = LC ? radix_k(LC) : radix_k(seg.L);
+    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
+    const int NG = D / G, NGg = NG * g;
+    const int split = blockIdx.x, u = blockIdx.y;
+    const int b = u / H, hk = u % H, Hq = H * g;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float mid = 0.5f * (float)(L - 1);
+
+    extern __shared__ __align__(16) float dsm[];
+    float* qs = dsm;                 // [D][GMAX]
+    float* qsum = qs + D * GMAX;     // [NG][GMAX]
+    float* red = qsum + 16 * GMAX;   // [4][GMAX]
+    float* zs = red + 4 * GMAX;      // [NG*g]
+    float* ls = zs + 16 * GMAX;      // [GMAX]
+    float* Pv = ls + GMAX;           // [TILE][NG*g]
+    float* part = Pv + TILE * NGg;   // [TILE][NG*g]
+    float* lpart = part + TILE * NGg;  // [TILE][GMAX]
+
+    for (int i = tid; i < g * D; i += blockDim.x) {
+        const int h = i / D, d = i % D;
+        qs[d * GMAX + h] = h2f(q[((size_t)b * Hq + hk * g + h) * D + d]);
+    }
+    __syncthreads();
+    for (int i = tid; i < NGg; i += blockDim.x) {
+        const int grp = i / g, h = i % g;
+        float s = 0.f;
+        for (int d = grp * G; d < (grp + 1) * G; ++d) s += qs[d * GMAX + h];
+        qsum[grp * GMAX + h] = s;
+    }
+    __syncthreads();
+
+    const int n = seg.n[u];
+    const int tiles = min(ceil_div(n, TILE), seg.tiles_cap);  // never past the segment's capacity
+    const int per = ceil_div(tiles, nsplit);
+    const int t0 = split * per, t1 = min(tiles, t0 + per);
+
+    float m[GMAX], acc[GMAX], zacc = 0.f, lacc = 0.f;
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+        m[h] = -__int_as_float(0x7f800000);
+        acc[h] = 0.f;
+    }
+    const int grp_d = tid / G;
+
+    for (int tile = t0; tile < t1; ++tile) {
+        const size_t tb = (size_t)u * seg.tiles_cap + tile;
+        const uint32_t* kw = seg.k + tb * WK * TILE;
+        const uint32_t* vw = seg.v + tb * WV * D;
+        const uint32_t* kz = seg.kz + tb * NG * TILE;
+        const uint32_t* vz = seg.vz + tb * NG * TILE;
+        const bool valid = tile * TILE + tid < n;
+
+        // ---- K side: thread = slot
+        float logit[GMAX], a[GMAX];
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) logit[h] = a[h] = 0.f;
+        int cur = 0;
+        auto flush = [&](int grp) {
+            const uint32_t zz = kz[grp * TILE + tid];
+            const float s = h2f((uint16_t)(zz & 0xffffu));
+            const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(zz >> 16)));
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h)
+                if (h < g) logit[h] += s * a[h] + zc * qsum[grp * GMAX + h];
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) a[h] = 0.f;
+        };
+        for (int j = 0; j < WK; ++j) {
+            int dg[32];
+            digits_of<LC>(kw[j * TILE + tid], L, k, dg);
+#pragma unroll
+            for (int i = 0; i < (LC ? Radix<(LC ? LC : 2)>::k : 32); ++i) {
+                if (i >= k) break;
+                const int d = j * k + i;
+                if (d >= D) break;
+                const int grp = d / G;
+                if (grp != cur) {
+                    flush(cur);
+                    cur = grp;
+                }
+                const float cf = (float)dg[i] - mid;
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h)
+                    if (h < g) a[h] += qs[d * GMAX + h] * cf;
+            }
+        }
+        flush(cur);
+
+        // ---- online softmax (log2 domain)
+        float alpha[GMAX], p[GMAX];
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            if (h < g) {
+                logit[h] = valid ? logit[h] * scale_log2 : -__int_as_float(0x7f800000);
+                const float mx = warp_max(logit[h]);
+                if (lane == 0) red[warp * GMAX + h] = mx;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            if (h < g) {
+                const float mt = fmaxf(fmaxf(red[h], red[GMAX + h]), fmaxf(red[2 * GMAX + h], red[3 * GMAX + h]));
+                const float mn = fmaxf(m[h], mt);
+                alpha[h] = exp2f(m[h] - mn);
+                m[h] = mn;
+                p[h] = valid ? exp2f(logit[h] - mn) : 0.f;
+            } else {
+                alpha[h] = p[h] = 0.f;
+            }
+        }
+        for (int grp = 0; grp < NG; ++grp) {
+            const uint32_t zz = vz[grp * TILE + tid];
+            const float s = h2f((uint16_t)(zz & 0xffffu));
+            const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(zz >> 16)));
+            for (int h = 0; h < g; ++h) {
+                Pv[tid * NGg + grp * g + h] = p[h] * s;
+                part[tid * NGg + grp * g + h] = p[h] * zc;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) lpart[tid * GMAX + h] = p[h];
+        __syncthreads();
+
+        // ---- V side: thread = channel
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) acc[h] *= alpha[h];
+        for (int w = 0; w < WV; ++w) {
+            int dg[32];
+            digits_of<LC>(vw[w * D + tid], L, k, dg);
+#pragma unroll
+            for (int i = 0; i < (LC ? Radix<(LC ? LC : 2)>::k : 32); ++i) {
+                if (i >= k) break;
+                const int t = w * k + i;
+                if (t >= TILE) break;
+                const float cf = (float)dg[i] - mid;
+                const float* pv = Pv + t * NGg + grp_d * g;
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h)
+                    if (h < g) acc[h] += pv[h] * cf;
+            }
+        }
+        if (tid < NGg) {
+            float s = 0.f;
+            for (int t = 0; t < TILE; ++t) s += part[t * NGg + tid];
+            zacc = zacc * alpha[tid % g] + s;
+        }
+        if (tid < g) {
+            float s = 0.f;
+            for (int t = 0; t < TILE; ++t) s += lpart[t * GMAX + tid];
+            lacc = lacc * alpha[tid] + s;
+        }
+        __syncthreads();
+    }
+
+    if (tid < NGg) zs[tid] = zacc;
+    if (tid < g) ls[tid] = lacc;
+    __syncthreads();
+    float* out = ws + ((size_t)u * nsplit_total + split_off + split) * g * (D + 2);
+    for (int h = 0; h < g; ++h) {
+        out[h * (D + 2) + tid] = acc[h] + zs[grp_d * g + h];
+        if (tid == 0) {
+            out[h * (D + 2) + D] = m[h];
+            out[h * (D + 2) + D + 1] = ls[h];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128) k_decode_merge(const float* __restrict__ ws, int g, int nsplit_total,
+                                                       float* __restrict__ out)
+{
+    constexpr int D = 128;
+    const int u = blockIdx.x / g, h = blockIdx.x % g, d = threadIdx.x;
+    const float* base = ws + (size_t)u * nsplit_total * g * (D + 2) + h * (D + 2);
+    const size_t stride = (size_t)g * (D + 2);
+    float M = -__int_as_float(0x7f800000);
+    for (int s = 0; s < nsplit_total; ++s) M = fmaxf(M, base[s * stride + D]);
+    float O = 0.f, Ls = 0.f;
+    if (M != -__int_as_float(0x7f800000)) {
+        for (int s = 0; s < nsplit_total; ++s) {
+            const float wgt = exp2f(base[s * stride + D] - M);
+            Ls += base[s * stride + D + 1] * wgt;
+            O += base[s * stride + d] * wgt;
+        }
+    }
+    out[((size_t)u * g + h) * D + d] = Ls > 0.f ? O / Ls : 0.f;
+}
+
+static size_t decode_smem(int NGg)
+{
+    return sizeof(float) * ((size_t)128 * GMAX + 16 * GMAX + 4 * GMAX + 16 * GMAX + GMAX + (size_t)2 * TILE * NGg +
+                            (size_t)TILE * GMAX);
+}
+
+template <int LC>
+static void launch_ds(const SegView& seg, const uint16_t* q, int units, int H, int g, int G, float scale_log2,
+                      int nsplit, int split_off, int nsplit_total, float* ws, cudaStream_t st)
+{
+    const size_t sm = decode_smem((128 / G) * g);
+    cudaFuncSetAttribute(k_decode_split<LC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    dim3 grid(nsplit, units);
+    k_decode_split<LC><<<grid, 128, sm, st>>>(seg, q, H, g, G, scale_log2, nsplit, split_off, nsplit_total, ws);
+}
+
+void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H, int g, int D, int G,
+                         float scale_log2, int nsplit, int split_off, int nsplit_total, float* ws, cudaStream_t st)
+{
+    (void)D;
+    if (nsplit == 0 || units == 0) return;
+    switch (seg.L) {
+#define SEMKV_D(LL) \
+    case LL: launch_ds<LL>(seg, q, units, H, g, G, scale_log2, nsplit, split_off, nsplit_total, ws, st); break;
+        SEMKV_D(2) SEMKV_D(3) SEMKV_D(4) SEMKV_D(5) SEMKV_D(6) SEMKV_D(7) SEMKV_D(8) SEMKV_D(9)
+        SEMKV_D(10) SEMKV_D(11) SEMKV_D(12) SEMKV_D(13) SEMKV_D(14) SEMKV_D(15) SEMKV_D(16)
+#undef SEMKV_D
+        default: launch_ds<0>(seg, q, units, H, g, G, scale_log2, nsplit, split_off, nsplit_total, ws, st); break;
+    }
+}
+
+void launch_decode_merge(const float* ws, int units, int H, int g, int D, int nsplit_total, float* out,
+                         cudaStream_t st)
+{
+    (void)H;
+    (void)D;
+    k_decode_merge<<<units * g, 128, 0, st>>>(ws, g, nsplit_total, out);
+}
+
+}  // namespace semkv

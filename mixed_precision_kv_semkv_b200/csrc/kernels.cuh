@@ -1,0 +1,40 @@
+// Host-side launchers of the libsemkv kernels (defined in the .cu files of this directory).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/semkv.h"
+
+namespace semkv {
+
+// One segment (hi or lo) of one layer's cache, as the kernels see it.
+struct SegView {
+    uint32_t* k;    // [units][tiles_cap][WK][128]
+    uint32_t* v;    // [units][tiles_cap][WV][D]
+    uint32_t* kz;   // [units][tiles_cap][NG][128]
+    uint32_t* vz;   // [units][tiles_cap][NG][128]
+    int32_t* n;     // [units] tokens in the segment
+    int L;          // levels
+    int tiles_cap;  // capacity in tiles of 128 slots
+    int is_hi;      // 1: L_hi segment (bitmap bit 1), 0: L_lo segment
+};
+
+void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
+                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st);
+
+void launch_quantize(const SegView& seg, const uint16_t* K, const uint16_t* V, const uint32_t* bitmap,
+                     const uint32_t* rank, int units, int T, int D, int G, int words_cap, int32_t* status,
+                     cudaStream_t st);
+
+void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, cudaStream_t st);
+
+// decode: split partials of one segment go to splits [split_off, split_off + nsplit) of each unit
+void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H, int g, int D, int G,
+                         float scale_log2, int nsplit, int split_off, int nsplit_total, float* ws, cudaStream_t st);
+void launch_decode_merge(const float* ws, int units, int H, int g, int D, int nsplit_total, float* out,
+                         cudaStream_t st);
+
+void launch_dequantize(const semkv_cache_t& c, int T, float* K, float* V, cudaStream_t st);
+
+}  // namespace semkv

@@ -1,0 +1,142 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI and the oracle on
+the same inputs, and compare (bit-exact for bitmaps, ranks, counts, thresholds, packed words,
+scale/zero and dequantized values; attention within max-abs 2e-3 and relative L2 1e-3 of fp64)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle
+from mixed_precision_kv_semkv_b200 import (SemkvCache, semkv_append_token, semkv_assign_precision,
+                                           semkv_decode_attention, semkv_dequantize, semkv_quantize_pack)
+
+ATOL = 2e-3
+RTOL_L2 = 1e-3
+
+
+def to_dev(a):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def unit_views(cache: SemkvCache, bufs: dict, u: int):
+    """Per-unit numpy views of the fetched device buffers, in the oracle's array shapes."""
+    B, H, G, D = cache.B, cache.H, cache.G, cache.D
+    units = B * H
+    out = {}
+    for seg, L, cap in (("hi", cache.L_hi, cache.cap_hi), ("lo", cache.L_lo, cache.cap_lo)):
+        tiles = cap // 128
+        sh = oracle.segment_shapes(D, G, L, tiles)
+        d = {}
+        for name in ("k", "v", "kz", "vz"):
+            arr = bufs[f"{name}_{seg}"].view(np.uint32)
+            per = int(np.prod(sh[name]))
+            d[name] = arr[: units * per].reshape(units, *sh[name])[u]
+        out[seg] = d
+    wc = cache.T_cap // 32
+    out["bitmap"] = bufs["bitmap"].view(np.uint32)[: units * wc].reshape(units, wc)[u]
+    out["rank"] = bufs["rank"].view(np.uint32)[: units * wc].reshape(units, wc)[u]
+    out["n_hi"] = int(bufs["n_hi"][u])
+    out["n_lo"] = int(bufs["n_lo"][u])
+    out["tau"] = np.float32(bufs["tau"].view(np.float32)[u])
+    return out
+
+
+def fetch(cache: SemkvCache) -> dict:
+    import torch
+
+    torch.cuda.synchronize()
+    return {n: t.cpu().numpy() for n, t in cache.bufs.items()}
+
+
+def gpu_prefill(K, V, S, p, G, L_hi, L_lo, extra=0):
+    """select + quantize_pack on the GPU. K, V numpy fp16 [B][H][T][D], S fp32 [B][H][T]."""
+    B, H, T, D = K.shape
+    cache = SemkvCache.for_prefill(B, H, H, G, L_hi, L_lo, T, p, extra=extra)
+    return cache
+
+
+def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0):
+    import torch
+
+    B, H, T, D = K.shape
+    Hq = q.shape[1]
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra)
+    dK, dV, dS, dq = to_dev(K), to_dev(V), to_dev(S), to_dev(q)
+    semkv_assign_precision(cache, dS, T, p)
+    semkv_quantize_pack(cache, dK, dV, T)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device="cuda")
+    ws = cache.workspace()
+    semkv_decode_attention(cache, dq, scale, out, ws)
+    Kh = torch.empty((B, H, T, D), dtype=torch.float32, device="cuda")
+    Vh = torch.empty_like(Kh)
+    semkv_dequantize(cache, Kh, Vh, T)
+    res = {"cache": cache, "bufs": fetch(cache), "out": out.cpu().numpy(), "Kh": Kh.cpu().numpy(),
+           "Vh": Vh.cpu().numpy(), "status": cache.status()}
+    return res
+
+
+def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo):
+    """Oracle results of one unit. K, V [T][D] fp16; S [T]; q [g][D] fp16."""
+    bm, rk, nh, tau, st = oracle.select(S, p)
+    hi, lo, st2 = oracle.quantize_pack_unit(K.view(np.uint16), V.view(np.uint16), bm, G, L_hi, L_lo, tiles_hi,
+                                            tiles_lo)
+    T = K.shape[0]
+    Kh, Vh = oracle.dequantize_unit(T, K.shape[1], G, L_hi, L_lo, bm, hi, lo)
+    o = oracle.attention_fp64(q.view(np.uint16), Kh, Vh, scale)
+    return {"bitmap": bm, "rank": rk, "n_hi": nh, "tau": tau, "hi": hi, "lo": lo, "Kh": Kh, "Vh": Vh, "out": o,
+            "status": st | st2}
+
+
+def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = ""):
+    nw = (T + 31) // 32
+    assert np.array_equal(g["bitmap"][:nw], o["bitmap"][:nw]), f"bitmap {where}"
+    assert np.array_equal(g["rank"][:nw], o["rank"][:nw]), f"rank {where}"
+    assert g["n_hi"] == o["n_hi"] and g["n_lo"] == T - o["n_hi"], f"counts {where}"
+    assert np.float32(g["tau"]).view(np.uint32) == np.float32(o["tau"]).view(np.uint32), f"tau {where}"
+    for seg, n in (("hi", o["n_hi"]), ("lo", T - o["n_hi"])):
+        nt = -(-n // 128)
+        for name in ("k", "v", "kz", "vz"):
+            a, b = g[seg][name][:nt], o[seg][name][:nt]
+            if not np.array_equal(a, b):
+                bad = np.argwhere(a != b)
+                raise AssertionError(f"{seg}.{name} {where}: {len(bad)} words differ, first at {bad[0].tolist()} "
+                                     f"gpu={a[tuple(bad[0])]:#x} oracle={b[tuple(bad[0])]:#x}")
+
+
+def attention_errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    max_abs = float(np.abs(got - ref).max()) if got.size else 0.0
+    den = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got - ref))
+    return max_abs, rel
+
+
+def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None):
+    """Run the GPU path on a whole case and compare the chosen units (default: all) with the oracle."""
+    B, H, T, D = K.shape
+    g = q.shape[1] // H
+    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale)
+    cache = res["cache"]
+    assert res["status"] == 0, f"status {res['status']}"
+    units = range(B * H) if units is None else units
+    worst = (0.0, 0.0)
+    for u in units:
+        b, h = divmod(u, H)
+        o = oracle_unit(K[b, h], V[b, h], S[b, h], q[b, h * g:(h + 1) * g], p, G, L_hi, L_lo, scale,
+                        cache.cap_hi // 128, cache.cap_lo // 128)
+        gu = unit_views(cache, res["bufs"], u)
+        compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}")
+        assert np.array_equal(res["Kh"][b, h].view(np.uint32), o["Kh"].view(np.uint32)), f"Khat unit {u}"
+        assert np.array_equal(res["Vh"][b, h].view(np.uint32), o["Vh"].view(np.uint32)), f"Vhat unit {u}"
+        ma, rl = attention_errors(res["out"][b, h * g:(h + 1) * g], o["out"])
+        worst = (max(worst[0], ma), max(worst[1], rl))
+        assert ma <= ATOL and rl <= RTOL_L2, f"attention unit {u}: max_abs {ma:.3g} rel_l2 {rl:.3g}"
+    return worst
+
+
+def sm_scale(D=128):
+    return 1.0 / math.sqrt(D)
