@@ -19,8 +19,9 @@
  *
  *   select      order the tokens of one (batch, kv-head) unit by score; the n_hi = floor(p*T) with
  *               the largest scores get L_hi levels, the rest L_lo.  [reading: floor; equal scores
- *               are ordered by lower token index first; tau = the n_hi-th largest score, +inf if
- *               n_hi = 0.]  Done here with a full sort -- no selection algorithm.
+ *               are ordered by lower token index first (-0 and +0 are equal); tau = the n_hi-th
+ *               largest score (a zero stored as +0), +inf if n_hi = 0.]  Done here with a full
+ *               sort -- no selection algorithm.
  *   quantize    per token, per group of G channels: mn = min x, mx = max x;
  *               s = (mx - mn)/(L - 1) in fp32, then rounded UP to fp16 [reading: rounding up keeps
  *               the grid z + c*s, c = 0..L-1, over [mn, mx]; saturates at 65504];  z = mn (exact
@@ -185,7 +186,8 @@ int oracle_select(const float* score, int32_t T, float p, uint32_t* bitmap, uint
         }
     }
     *n_hi_out = n_hi;
-    *tau_out = n_hi > 0 ? v[n_hi - 1].s : INFINITY;
+    /* -0 and +0 are the same score; the threshold is stored as +0 */
+    *tau_out = n_hi > 0 ? v[n_hi - 1].s + 0.0f : INFINITY;
     free(v);
     return status;
 }

@@ -153,6 +153,7 @@ def test_select_matches_brute_force_on_tiny_units(orc, seed):
     assert n_hi == len(want)
     if n_hi:
         assert tau == np.sort(scores)[::-1][n_hi - 1]
+        assert not (tau == 0 and np.signbit(tau))  # a zero threshold is stored as +0
     else:
         assert tau == np.inf
 
