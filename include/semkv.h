@@ -38,6 +38,9 @@
  *   rank    [B*H][T_cap/32]  rank[w] = number of L_hi tokens in words 0..w-1 (valid for words
  *                            that hold at least one token)
  *   n_hi, n_lo [B*H] int32   tokens in each segment (a token's slot is its rank in its class)
+ *                            Slots past n of a segment hold unspecified words, except that after
+ *                            semkv_quantize_pack the rest of the last tile is zero, and a V word
+ *                            that holds a live slot always has zero digits at the slots past n.
  *   tau     [B*H] float      precision threshold of the unit (the n_hi-th largest score)
  *   status  [1] int32        device status word (SEMKV_STATUS_* bits)
  * Code c of value x on a group with scale s and zero z dequantizes to fmaf((float)c, s, z).

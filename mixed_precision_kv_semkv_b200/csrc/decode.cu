@@ -158,9 +158,9 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
             const uint32_t zz = vz[grp * TILE + tid];
             const float s = h2f((uint16_t)(zz & 0xffffu));
             const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(zz >> 16)));
-            for (int h = 0; h < g; ++h) {
-                Pv[tid * NGg + grp * g + h] = p[h] * s;
-                part[tid * NGg + grp * g + h] = p[h] * zc;
+            for (int h = 0; h < g; ++h) {  // slots past n may hold stale scale/zero bits: write zeros
+                Pv[tid * NGg + grp * g + h] = valid ? p[h] * s : 0.f;
+                part[tid * NGg + grp * g + h] = valid ? p[h] * zc : 0.f;
             }
         }
 #pragma unroll

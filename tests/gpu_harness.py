@@ -51,13 +51,6 @@ def fetch(cache: SemkvCache) -> dict:
     return {n: t.cpu().numpy() for n, t in cache.bufs.items()}
 
 
-def gpu_prefill(K, V, S, p, G, L_hi, L_lo, extra=0):
-    """select + quantize_pack on the GPU. K, V numpy fp16 [B][H][T][D], S fp32 [B][H][T]."""
-    B, H, T, D = K.shape
-    cache = SemkvCache.for_prefill(B, H, H, G, L_hi, L_lo, T, p, extra=extra)
-    return cache
-
-
 def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0):
     import torch
 
@@ -90,20 +83,37 @@ def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo):
             "status": st | st2}
 
 
-def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = ""):
+def _words_equal(a, b, what):
+    if not np.array_equal(a, b):
+        bad = np.argwhere(a != b)
+        raise AssertionError(f"{what}: {len(bad)} words differ, first at {bad[0].tolist()} "
+                             f"gpu={a[tuple(bad[0])]:#x} oracle={b[tuple(bad[0])]:#x}")
+
+
+def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = "", strict_tail: bool = True):
+    """Bit-exact comparison of one unit's state.  strict_tail: the last tile's slots past n must be
+    zero as well (true after a prefill; after appends into a new tile they are unspecified, except
+    that V words holding a live slot have zero digits past n)."""
     nw = (T + 31) // 32
     assert np.array_equal(g["bitmap"][:nw], o["bitmap"][:nw]), f"bitmap {where}"
     assert np.array_equal(g["rank"][:nw], o["rank"][:nw]), f"rank {where}"
     assert g["n_hi"] == o["n_hi"] and g["n_lo"] == T - o["n_hi"], f"counts {where}"
     assert np.float32(g["tau"]).view(np.uint32) == np.float32(o["tau"]).view(np.uint32), f"tau {where}"
-    for seg, n in (("hi", o["n_hi"]), ("lo", T - o["n_hi"])):
-        nt = -(-n // 128)
+    for seg, n, L in (("hi", o["n_hi"], L_hi), ("lo", T - o["n_hi"], L_lo)):
+        if strict_tail:
+            nt = -(-n // 128)
+            for name in ("k", "v", "kz", "vz"):
+                _words_equal(g[seg][name][:nt], o[seg][name][:nt], f"{seg}.{name} {where}")
+            continue
+        full, rem = divmod(n, 128)
+        k = oracle.radix_digits(L)
         for name in ("k", "v", "kz", "vz"):
-            a, b = g[seg][name][:nt], o[seg][name][:nt]
-            if not np.array_equal(a, b):
-                bad = np.argwhere(a != b)
-                raise AssertionError(f"{seg}.{name} {where}: {len(bad)} words differ, first at {bad[0].tolist()} "
-                                     f"gpu={a[tuple(bad[0])]:#x} oracle={b[tuple(bad[0])]:#x}")
+            _words_equal(g[seg][name][:full], o[seg][name][:full], f"{seg}.{name} {where}")
+        if rem:
+            for name in ("k", "kz", "vz"):
+                _words_equal(g[seg][name][full][:, :rem], o[seg][name][full][:, :rem], f"{seg}.{name} tail {where}")
+            nwv = -(-rem // k)
+            _words_equal(g[seg]["v"][full][:nwv], o[seg]["v"][full][:nwv], f"{seg}.v tail {where}")
 
 
 def attention_errors(got, ref):

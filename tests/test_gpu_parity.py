@@ -163,7 +163,7 @@ def test_append_matches_oracle_in_lockstep(p, L_hi, L_lo, G):
         assert ost == 0
         gu = unit_views(cache, bufs, u)
         o = {"bitmap": st.bitmap, "rank": st.rank, "n_hi": st.n_hi, "tau": st.tau, "hi": st.hi, "lo": st.lo}
-        compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}")
+        compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}", strict_tail=False)
         b, h = divmod(u, H)
         Kh, Vh = oracle.dequantize_unit(T, 128, G, L_hi, L_lo, st.bitmap, st.hi, st.lo)
         ref = oracle.attention_fp64(q[b, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, sm_scale())
@@ -180,7 +180,7 @@ def test_append_overflow_sets_status_and_keeps_state():
     st, ost = states[0]
     assert ost & 4 and st.n_lo == 128
     compare_state(gu, {"bitmap": st.bitmap, "rank": st.rank, "n_hi": 0, "tau": st.tau, "hi": st.hi, "lo": st.lo},
-                  128, 8, 5)
+                  128, 8, 5, strict_tail=False)
 
 
 def test_empty_unit_decodes_to_zero():
