@@ -190,7 +190,8 @@ def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi:
     T, D = K16.shape
     hi, lo = _alloc_unit(D, G, L_hi, L_lo, tiles_hi, tiles_lo)
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
-    bm[: len(bitmap)] = bitmap
+    n = min(len(bitmap), len(bm))
+    bm[:n] = bitmap[:n]
     st = lib().oracle_quantize_pack_unit(K16.ravel(), V16.ravel(), T, D, G, L_hi, L_lo, bm, tiles_hi, tiles_lo,
                                          *_seg_args(hi, lo))
     return hi, lo, st
@@ -201,7 +202,8 @@ def dequantize_unit(T: int, D: int, G: int, L_hi: int, L_lo: int, bitmap, hi, lo
     Kh = np.zeros((max(T, 1), D), np.float32)
     Vh = np.zeros((max(T, 1), D), np.float32)
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
-    bm[: len(bitmap)] = bitmap
+    n = min(len(bitmap), len(bm))
+    bm[:n] = bitmap[:n]
     lib().oracle_dequantize_unit(T, D, G, L_hi, L_lo, bm, *_seg_args(hi, lo), Kh.ravel(), Vh.ravel())
     return Kh[:T], Vh[:T]
 
