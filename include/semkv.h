@@ -76,6 +76,8 @@ extern "C" {
 #define SEMKV_STATUS_APPEND_OVERFLOW 4 /* an appended token found its segment (or T_cap) full and
                                           was dropped; that unit's state is unchanged */
 #define SEMKV_STATUS_LENGTH_MISMATCH 8 /* semkv_dequantize: a unit's n_hi + n_lo != T */
+#define SEMKV_STATUS_TIMEOUT 16        /* a kernel gave up a bounded wait (asynchronous copy or tensor-core
+                                          result); that call's outputs are incomplete */
 
 /* One layer's packed cache.  Shape fields are set by the caller; the pointers are device
  * buffers of the sizes semkv_cache_bytes() reports, in the order of the SEMKV_BUF_* indices. */
@@ -122,7 +124,7 @@ SEMKV_API int semkv_assign_precision(const semkv_cache_t* cache, const float* sc
  * semkv_assign_precision must have run for this T.  Per token and group of G channels:
  * mn, mx = min, max; s = fp16 rounded up of fp32 (mx - mn)/(L - 1) (saturated at 65504);
  * z = mn; code = clamp(rint((x - z)/s), 0, L - 1) (fp32 subtract and divide, ties to even; 0 if
- * s = 0).  Codes are packed and placed as described at the top of this file; slots past the
+ * s = 0).  K and V must be 16-byte aligned (rows are fetched with bulk copies).  Codes are packed and placed as described at the top of this file; slots past the
  * segment's length inside its last tile get zero codes and zero scale/zero.  Non-finite inputs
  * set SEMKV_STATUS_NONFINITE_KV. */
 SEMKV_API int semkv_quantize_pack(const semkv_cache_t* cache, const uint16_t* K, const uint16_t* V, int32_t T,

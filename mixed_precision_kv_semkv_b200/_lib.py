@@ -23,6 +23,7 @@ STATUS_NAN_SCORE = 1
 STATUS_NONFINITE_KV = 2
 STATUS_APPEND_OVERFLOW = 4
 STATUS_LENGTH_MISMATCH = 8
+STATUS_TIMEOUT = 16
 
 SHAPE_FIELDS = ("B", "H", "Hq", "D", "G", "L_hi", "L_lo", "cap_hi", "cap_lo", "T_cap")
 BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",

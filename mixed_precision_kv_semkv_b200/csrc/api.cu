@@ -63,13 +63,13 @@ int sm_count()
     return n;
 }
 
-// Split-K factor per segment: about four CTAs per SM over the whole decode, shared between the
-// segments in proportion to their capacity in tiles, at most one split per tile.
+// Split-K factor per segment: one wave of two CTAs per SM over the whole decode, shared between
+// the segments in proportion to their capacity in tiles, at most one split per tile.
 void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
 {
     const int units = c->B * c->H;
     const int th = c->cap_hi / TILE, tl = c->cap_lo / TILE, total = th + tl;
-    const long target = 4L * sm_count();
+    const long target = 2L * sm_count();
     auto pick = [&](int tiles) -> int {
         if (tiles == 0) return 0;
         long s = (target * tiles + (long)units * total - 1) / ((long)units * total);
@@ -159,10 +159,9 @@ int semkv_quantize_pack(const semkv_cache_t* c, const uint16_t* K, const uint16_
     if (r != SEMKV_OK) return r;
     if (T < 0 || T > c->T_cap || ((!K || !V) && T > 0)) return SEMKV_ERR_INVALID_ARG;
     if (T == 0) return SEMKV_OK;
-    const int units = c->B * c->H;
-    for (int hi = 1; hi >= 0; --hi)
-        launch_quantize(seg_view(c, hi != 0), K, V, c->bitmap, c->rank, units, T, c->D, c->G, c->T_cap / 32,
-                        c->status, (cudaStream_t)stream);
+    if ((((uintptr_t)K) | ((uintptr_t)V)) & 15u) return SEMKV_ERR_INVALID_ARG;  // rows are fetched by bulk copies
+    launch_quantize(seg_view(c, true), seg_view(c, false), K, V, c->bitmap, c->rank, c->B * c->H, T, c->D, c->G,
+                    c->T_cap / 32, c->status, (cudaStream_t)stream);
     return launch_status();
 }
 
@@ -191,8 +190,18 @@ int semkv_decode_attention(const semkv_cache_t* c, const uint16_t* q, float soft
     const float scale_log2 = softmax_scale * 1.4426950408889634f;
     float* ws = static_cast<float*>(workspace);
     cudaStream_t st = (cudaStream_t)stream;
-    launch_decode_split(seg_view(c, true), q, units, c->H, g, c->D, c->G, scale_log2, nh, 0, nh + nl, ws, st);
-    launch_decode_split(seg_view(c, false), q, units, c->H, g, c->D, c->G, scale_log2, nl, nh, nh + nl, ws, st);
+    bool dependent = false;
+    for (int hi = 1; hi >= 0; --hi) {
+        const SegView sv = seg_view(c, hi != 0);
+        const int ns = hi ? nh : nl, off = hi ? 0 : nh;
+        if (ns == 0) continue;
+        if (decode_tc_supported(sv.L, c->G, g)) {
+            launch_decode_tc(sv, q, units, c->H, g, c->G, scale_log2, ns, off, nh + nl, ws, c->status, dependent, st);
+        } else {
+            launch_decode_split(sv, q, units, c->H, g, c->D, c->G, scale_log2, ns, off, nh + nl, ws, st);
+        }
+        dependent = true;
+    }
     launch_decode_merge(ws, units, c->H, g, c->D, nh + nl, out, st);
     return launch_status();
 }

@@ -211,23 +211,39 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
     }
 }
 
+// Log-sum-exp merge of the split partials of one (unit, query head): all splits' maxima are read
+// in parallel, the weights 2^(m_s - M) go to shared memory, then thread d sums o_s[d] with
+// independent loads.
 __global__ void __launch_bounds__(128) k_decode_merge(const float* __restrict__ ws, int g, int nsplit_total,
                                                        float* __restrict__ out)
 {
     constexpr int D = 128;
-    const int u = blockIdx.x / g, h = blockIdx.x % g, d = threadIdx.x;
+    const int u = blockIdx.x / g, h = blockIdx.x % g, d = threadIdx.x, lane = d & 31, warp = d >> 5;
     const float* base = ws + (size_t)u * nsplit_total * g * (D + 2) + h * (D + 2);
     const size_t stride = (size_t)g * (D + 2);
-    float M = -__int_as_float(0x7f800000);
-    for (int s = 0; s < nsplit_total; ++s) M = fmaxf(M, base[s * stride + D]);
-    float O = 0.f, Ls = 0.f;
-    if (M != -__int_as_float(0x7f800000)) {
-        for (int s = 0; s < nsplit_total; ++s) {
-            const float wgt = exp2f(base[s * stride + D] - M);
-            Ls += base[s * stride + D + 1] * wgt;
-            O += base[s * stride + d] * wgt;
-        }
+    extern __shared__ float wts[];  // [nsplit_total]
+    __shared__ float red[4], redl[4];
+    const float NEG = -__int_as_float(0x7f800000);
+    float M = NEG;
+    for (int s = d; s < nsplit_total; s += 128) M = fmaxf(M, base[s * stride + D]);
+    M = warp_max(M);
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    float l = 0.f;
+    for (int s = d; s < nsplit_total; s += 128) {
+        const float w = M == NEG ? 0.f : exp2f(base[s * stride + D] - M);
+        wts[s] = w;
+        l += w * base[s * stride + D + 1];
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) redl[warp] = l;
+    __syncthreads();
+    const float Ls = redl[0] + redl[1] + redl[2] + redl[3];
+    float O = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < nsplit_total; ++s) O += wts[s] * base[s * stride + d];
     out[((size_t)u * g + h) * D + d] = Ls > 0.f ? O / Ls : 0.f;
 }
 
@@ -267,7 +283,8 @@ void launch_decode_merge(const float* ws, int units, int H, int g, int D, int ns
 {
     (void)H;
     (void)D;
-    k_decode_merge<<<units * g, 128, 0, st>>>(ws, g, nsplit_total, out);
+    k_decode_merge<<<units * g, 128, (size_t)(nsplit_total > 0 ? nsplit_total : 1) * sizeof(float), st>>>(
+        ws, g, nsplit_total, out);
 }
 
 }  // namespace semkv

@@ -23,9 +23,9 @@ struct SegView {
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st);
 
-void launch_quantize(const SegView& seg, const uint16_t* K, const uint16_t* V, const uint32_t* bitmap,
-                     const uint32_t* rank, int units, int T, int D, int G, int words_cap, int32_t* status,
-                     cudaStream_t st);
+void launch_quantize(const SegView& hi, const SegView& lo, const uint16_t* K, const uint16_t* V,
+                     const uint32_t* bitmap, const uint32_t* rank, int units, int T, int D, int G, int words_cap,
+                     int32_t* status, cudaStream_t st);
 
 void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, cudaStream_t st);
 
@@ -34,6 +34,14 @@ void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H
                          float scale_log2, int nsplit, int split_off, int nsplit_total, float* ws, cudaStream_t st);
 void launch_decode_merge(const float* ws, int units, int H, int g, int D, int nsplit_total, float* out,
                          cudaStream_t st);
+
+// tcgen05 decode (decode_tc.cu): supported for L in {2, 4..8, 10..16}, G >= 32, g <= 8.
+bool decode_tc_supported(int L, int G, int g);
+// `dependent`: launched as a programmatic dependent of the previous kernel in the stream (it may
+// start while that kernel drains, and waits for it to complete before it exits).
+void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, int g, int G, float scale_log2,
+                      int nsplit, int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
+                      cudaStream_t st);
 
 void launch_dequantize(const semkv_cache_t& c, int T, float* K, float* V, cudaStream_t st);
 

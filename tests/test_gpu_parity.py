@@ -88,6 +88,36 @@ def test_constant_and_extreme_groups():
     check_case(K, V, S, q, 0.5, 64, 8, 5, sm_scale())
 
 
+@pytest.mark.parametrize("L", [3, 4, 5, 6, 8, 16])
+def test_quotients_at_and_near_half_steps(L):
+    """Values at, and one fp16 step around, the half-way points between grid levels: the codes
+    depend on the exact IEEE quotient and on ties-to-even, so any other division rule shows up."""
+    import oracle
+
+    r = np.random.default_rng(100 + L)
+    T, G = 384, 64
+    K = np.empty((1, 1, T, 128), np.float16)
+    for t in range(T):
+        for grp in range(2):
+            mn = np.float16(r.standard_normal() * 2)
+            mx = np.float16(float(mn) + abs(r.standard_normal()) * 4 + 0.01)
+            probe = np.array([mn, mx] * (G // 2), np.float16)
+            _, s16, _, _ = oracle.quantize_group(probe.view(np.uint16), L)
+            s = float(np.uint16(s16).view(np.float16))
+            c = r.integers(0, L - 1, size=G)
+            x = (float(mn) + (c + 0.5) * s).astype(np.float16)
+            nudge = r.integers(-1, 2, size=G)  # -1, 0, +1 fp16 step
+            x = np.where(nudge < 0, np.nextafter(x, np.float16(-np.inf)),
+                         np.where(nudge > 0, np.nextafter(x, np.float16(np.inf)), x))
+            x = np.clip(x, mn, mx)
+            x[0], x[1] = mn, mx
+            K[0, 0, t, grp * G:(grp + 1) * G] = x
+    V = K[:, :, ::-1].copy()
+    S = r.standard_normal((1, 1, T)).astype(np.float32)
+    q = r.standard_normal((1, 4, 128)).astype(np.float16)
+    check_case(K, V, S, q, 0.5, G, L, max(2, L - 1), sm_scale())
+
+
 def test_device_status_flags():
     import torch
 
