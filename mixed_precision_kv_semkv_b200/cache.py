@@ -71,6 +71,14 @@ class SemkvCache:
         nbytes = _lib.semkv_workspace_bytes(self.struct)
         return torch.empty(max(nbytes, 4), dtype=torch.uint8, device=self.bufs["status"].device)
 
+    def poison(self):
+        """Fill every buffer except the status word with 0xFF bytes (NaN as fp16/fp32), so that a
+        read of bytes the library never wrote shows up in tests."""
+        for name, t in self.bufs.items():
+            if name != "status":
+                t.view(__import__("torch").int32).fill_(-1)
+        return self
+
     def status(self) -> int:
         """Read the device status word (synchronizes)."""
         return int(self.bufs["status"].item())

@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(128, 1) k_decode_tc(SegView seg, const uint16_
             const float mx = warp_max(lg[h]);
             if (lane == 0) red[warp * 48 + h] = mx;
         }
-        // slots past n may hold stale words: their probabilities are exactly zero below
+        // slots past n may hold stale words (after appends): their p, P' and zero terms are exact zeros
         __syncthreads();
         float alpha[TC_GMAX], p[TC_GMAX];
 #pragma unroll
@@ -289,7 +289,8 @@ __global__ void __launch_bounds__(128, 1) k_decode_tc(SegView seg, const uint16_
             p[h] = (valid && h < g) ? exp2f(lg[h] - mn) : 0.f;
             lacc[h] = lacc[h] * alpha[h] + p[h];
 #pragma unroll
-            for (int gg = 0; gg < TC_NGMAX; ++gg) zacc[gg][h] = zacc[gg][h] * alpha[h] + p[h] * zv[gg];
+            for (int gg = 0; gg < TC_NGMAX; ++gg)  // a stale slot's scale/zero may be NaN: never multiply it
+                zacc[gg][h] = zacc[gg][h] * alpha[h] + (valid ? p[h] * zv[gg] : 0.f);
         }
         // ---- P' = p s_V as two fp16 limbs, into my slot's row of B_P
 #pragma unroll
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(128, 1) k_decode_tc(SegView seg, const uint16_
 #pragma unroll
                 for (int h = 0; h < TC_GMAX; ++h) {
                     if (h < g) {
-                        const float pv = p[h] * sv[gg];
+                        const float pv = valid ? p[h] * sv[gg] : 0.f;
                         const __half hi = __float2half_rn(pv);
                         const __half lo = __float2half_rn(pv - __half2float(hi));
                         const int n0 = gg * GSTR + h, n1 = gg * GSTR + g + h;

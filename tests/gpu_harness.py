@@ -56,7 +56,7 @@ def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0):
 
     B, H, T, D = K.shape
     Hq = q.shape[1]
-    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra)
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra).poison()
     dK, dV, dS, dq = to_dev(K), to_dev(V), to_dev(S), to_dev(q)
     semkv_assign_precision(cache, dS, T, p)
     semkv_quantize_pack(cache, dK, dV, T)

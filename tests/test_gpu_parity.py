@@ -155,7 +155,7 @@ def _append_lockstep(B, H, Hq, T0, steps, G, L_hi, L_lo, p, seed, extra):
     S = r.standard_normal((B, H, T0 + steps)).astype(np.float32)
     q = r.standard_normal((B, Hq, 128)).astype(np.float16)
     g = Hq // H
-    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T0, p, extra=extra)
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T0, p, extra=extra).poison()
     semkv_assign_precision(cache, to_dev(S[:, :, :T0].copy()), T0, p)
     semkv_quantize_pack(cache, to_dev(K[:, :, :T0].copy()), to_dev(V[:, :, :T0].copy()), T0)
     for t in range(T0, T0 + steps):
