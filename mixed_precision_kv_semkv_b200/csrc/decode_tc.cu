@@ -130,24 +130,34 @@ __global__ void __launch_bounds__(128, 1) k_decode_tc(SegView seg, const uint16_
         const __half2 pr = __floats2half2_rn((float)(P / L) - MID, (float)(P % L) - MID);  // exact: |x| <= 7.5
         lut[i] = *reinterpret_cast<const uint32_t*>(&pr);
     }
-    const uint16_t* qu = q + ((size_t)b * Hq + (size_t)hk * g) * D;
-    for (int i = tid; i < NK * KSLOTS; i += 128) {
-        const int nrow = i / KSLOTS, ks = i % KSLOTS;
-        uint16_t v = 0;
+    // the g query rows (g x 128 fp16) staged once in shared memory (reuses the B_P area, zeroed after)
+    uint16_t* qs = reinterpret_cast<uint16_t*>(bp);
+    {
+        const uint16_t* qu = q + ((size_t)b * Hq + (size_t)hk * g) * D;
+        for (int i = tid; i < g * D / 8; i += 128)
+            reinterpret_cast<uint4*>(qs)[i] = __ldg(reinterpret_cast<const uint4*>(qu) + i);
+    }
+    __syncthreads();
+    // B_Q: row n = (group, head) holds q_head at the K index of each channel of that group
+    for (int ks = tid; ks < KSLOTS; ks += 128) {
         const int col = ks >> 1, h2 = ks & 1, j = col / NPAIR, pp = col % NPAIR;
         const int pos = pair_digit(k, pp, h2);
-        const int dim = j * k + pos;
-        if (nrow < NG * g && col < KC && pos >= 0 && dim < D && dim / G == nrow / g) v = qu[(nrow % g) * D + dim];
-        *reinterpret_cast<uint16_t*>(bq + bq_off(nrow, ks, M::LBO_Q, M::SBO_Q)) = v;
+        const int dim = (col < KC && pos >= 0) ? j * k + pos : D;
+        const int dgrp = dim < D ? dim / G : -1;
+        for (int nrow = 0; nrow < NK; ++nrow) {
+            const uint16_t v = (nrow < NG * g && nrow / g == dgrp) ? qs[(nrow % g) * D + dim] : (uint16_t)0;
+            *reinterpret_cast<uint16_t*>(bq + bq_off(nrow, ks, M::LBO_Q, M::SBO_Q)) = v;
+        }
     }
-    for (int i = tid; i < (int)(M::BP_BYTES / 16); i += 128) reinterpret_cast<uint4*>(bp)[i] = make_uint4(0, 0, 0, 0);
     if (tid < NG * TC_GMAX) {
         const int grp = tid / TC_GMAX, h = tid % TC_GMAX;
         float s = 0.f;
         if (h < g)
-            for (int d = grp * G; d < (grp + 1) * G; ++d) s += h2f(qu[h * D + d]);
+            for (int d = grp * G; d < (grp + 1) * G; ++d) s += h2f(qs[h * D + d]);
         qsum[grp * TC_GMAX + h] = s;
     }
+    __syncthreads();
+    for (int i = tid; i < (int)(M::BP_BYTES / 16); i += 128) reinterpret_cast<uint4*>(bp)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
