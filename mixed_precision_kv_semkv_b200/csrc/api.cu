@@ -63,13 +63,13 @@ int sm_count()
     return n;
 }
 
-// Split-K factor per segment: one wave of two CTAs per SM over the whole decode, shared between
+// Split-K factor per segment: one wave of four CTAs per SM over the whole decode, shared between
 // the segments in proportion to their capacity in tiles, at most one split per tile.
 void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
 {
     const int units = c->B * c->H;
     const int th = c->cap_hi / TILE, tl = c->cap_lo / TILE, total = th + tl;
-    const long target = 2L * sm_count();
+    const long target = 4L * sm_count();
     auto pick = [&](int tiles) -> int {
         if (tiles == 0) return 0;
         long s = (target * tiles + (long)units * total - 1) / ((long)units * total);

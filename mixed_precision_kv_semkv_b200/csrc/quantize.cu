@@ -10,9 +10,9 @@
 //      first bitmap word, then a ballot scan), and fetches each token's K and V row (256 B each)
 //      with one cp.async.bulk per row into shared memory, completing on an mbarrier; the other
 //      warps zero the rows of slots past the segment's end meanwhile;
-//   2. thread t quantizes K row t and packs it along the channels (Horner, top digit first);
-//   3. thread t writes the scale/zero of V row t; after a barrier thread d quantizes channel d of
-//      every slot and packs it along the tile's slots.
+//   2. thread t quantizes K row t and packs it along the channels;
+//   3. thread t writes the scale/zero of V row t; after a barrier thread d packs channel d of
+//      every slot along the tile's slots.
 // The quotient (x - z)/s is the IEEE round-to-nearest quotient, computed by Markstein's method
 // (P. Markstein, IBM J. Res. Dev. 34(1), 1990): with r = RN(1/s) (one __frcp_rn per group),
 // q0 = RN(d r), e = d - s q0 (exact with one FMA), q = RN(q0 + e r) is the correctly rounded d/s
@@ -73,37 +73,20 @@ __device__ __forceinline__ uint32_t code_of(float x, const Grid& g, float top)
     return __float_as_uint(__fadd_rn(q, 12582912.0f)) - 0x4B400000u;
 }
 
-__global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
-                                                   const uint16_t* __restrict__ V,
-                                                   const uint32_t* __restrict__ bitmap,
-                                                   const uint32_t* __restrict__ rank, int T, int G, int words_cap,
-                                                   int32_t* __restrict__ status)
+// Slots [s0, s0 + nv) of a segment of unit u -> token indices (tok), and each token's K and V row
+// (256 B each) into shared memory: warp 0 searches the rank directory (32-ary) for the first
+// bitmap word, scans the following words with ballots, and issues one cp.async.bulk per row on
+// `bar`; rows of slots past nv are zeroed.  Returns false (status set) if the copies timed out.
+__device__ __forceinline__ bool gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok, uint64_t* bar, bool is_hi, int u,
+                                            int s0, int nv, const uint16_t* __restrict__ K,
+                                            const uint16_t* __restrict__ V, const uint32_t* __restrict__ bitmap,
+                                            const uint32_t* __restrict__ rank, int T, int words_cap,
+                                            int32_t* __restrict__ status)
 {
     constexpr int D = 128;
-    const int per_unit = hi.tiles_cap + lo.tiles_cap;
-    const int u = blockIdx.x / per_unit;
-    int tile = blockIdx.x % per_unit;
-    const bool is_hi = tile < hi.tiles_cap;
-    const QuantSeg& seg = is_hi ? hi : lo;
-    if (!is_hi) tile -= hi.tiles_cap;
-    const int L = seg.L, k = seg.k_digits;
-    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
-    const int NG = D / G;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = seg.n[u];
-    const int s0 = tile * TILE;
-    if (s0 >= n) return;
-    const int nv = min(TILE, n - s0);
-
-    extern __shared__ __align__(128) unsigned char smem[];
-    uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
-    uint16_t* Vs = Ks + TILE * QROW;
-    int* tok = reinterpret_cast<int*>(Vs + TILE * QROW);
-    float4* vgrid = reinterpret_cast<float4*>(tok + TILE);  // [TILE][NG] (s, r, z, -)
-    __shared__ __align__(8) uint64_t bar;
-
     if (tid == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(bar, 1);
         fence_mbar_init();
     }
     tok[tid] = -1;
@@ -153,14 +136,14 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
         for (int r = lane; r < nv; r += 32) valid_rows += (tok[r] >= 0 && tok[r] < T);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) valid_rows += __shfl_xor_sync(0xffffffffu, valid_rows, o);
-        if (lane == 0) mbar_arrive_expect_tx(&bar, (uint32_t)valid_rows * 2u * D * 2u);
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)valid_rows * 2u * D * 2u);
         __syncwarp();
         for (int r = lane; r < nv; r += 32) {
             const int t = tok[r];
             if (t >= 0 && t < T) {
                 const size_t off = ((size_t)u * T + t) * D;
-                bulk_g2s(Ks + r * QROW, K + off, D * 2, &bar);
-                bulk_g2s(Vs + r * QROW, V + off, D * 2, &bar);
+                bulk_g2s(Ks + r * QROW, K + off, D * 2, bar);
+                bulk_g2s(Vs + r * QROW, V + off, D * 2, bar);
             } else {
                 for (int i = 0; i < D; i += 8) {
                     *reinterpret_cast<uint4*>(Ks + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
@@ -176,13 +159,46 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
             }
         }
     }
-    const bool arrived = mbar_wait(&bar, 0);
+    const bool arrived = mbar_wait(bar, 0);
     __syncthreads();
     if (!arrived) {  // copies did not land in time: report, wait once more for them, and stop
         if (tid == 0) atomicOr(status, SEMKV_STATUS_TIMEOUT);
-        mbar_wait(&bar, 0);
-        return;
+        mbar_wait(bar, 0);
+        return false;
     }
+    return true;
+}
+
+__global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
+                                                   const uint16_t* __restrict__ V,
+                                                   const uint32_t* __restrict__ bitmap,
+                                                   const uint32_t* __restrict__ rank, int T, int G, int words_cap,
+                                                   int32_t* __restrict__ status)
+{
+    constexpr int D = 128;
+    const int per_unit = hi.tiles_cap + lo.tiles_cap;
+    const int u = blockIdx.x / per_unit;
+    int tile = blockIdx.x % per_unit;
+    const bool is_hi = tile < hi.tiles_cap;
+    const QuantSeg& seg = is_hi ? hi : lo;
+    if (!is_hi) tile -= hi.tiles_cap;
+    const int L = seg.L, k = seg.k_digits;
+    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
+    const int NG = D / G;
+    const int tid = threadIdx.x;
+    const int n = seg.n[u];
+    const int s0 = tile * TILE;
+    if (s0 >= n) return;
+    const int nv = min(TILE, n - s0);
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
+    uint16_t* Vs = Ks + TILE * QROW;
+    int* tok = reinterpret_cast<int*>(Vs + TILE * QROW);
+    float4* vgrid = reinterpret_cast<float4*>(tok + TILE);  // [TILE][NG] (s, r, z, -)
+    __shared__ __align__(8) uint64_t bar;
+
+    if (!gather_rows(Ks, Vs, tok, &bar, is_hi, u, s0, nv, K, V, bitmap, rank, T, words_cap, status)) return;
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     uint32_t* kw = seg.k + tile_base * WK * TILE;
@@ -276,6 +292,221 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     }
 }
 
+// ------------------------------------------------------------------ compile-time fast path
+//
+// Same tile work with L and G known at compile time: words are accumulated as sum_i code_i L^i with
+// constant powers (no serial Horner chain), codes are the low byte of the round-to-nearest-even
+// magic sum 1.5 * 2^23 + q (the offset is removed once per word), group minima and maxima use
+// packed fp16 (NaN-propagating, so a non-finite value shows up in the group's range), and the
+// quotient runs two lanes at a time in packed fp32.  For L >= 3 no clamp is needed: q <= L - 1
+// up to one rounding when the scale did not saturate, and q <= 131008/65504 = 2 when it did.
+
+__host__ __device__ constexpr uint32_t upow(int L, int i)
+{
+    uint32_t p = 1u;
+    for (int j = 0; j < i; ++j) p *= (uint32_t)L;
+    return p;
+}
+
+// magic offset carried by a word of `cnt` digits: 0x4B400000 * sum_{i < cnt} L^i (mod 2^32)
+__host__ __device__ constexpr uint32_t magic_sum(int L, int cnt)
+{
+    uint32_t s = 0u;
+    for (int i = 0; i < cnt; ++i) s += 0x4B400000u * upow(L, i);
+    return s;
+}
+
+__device__ __forceinline__ uint64_t f2_pack(float a, float b)
+{
+    return ((uint64_t)__float_as_uint(b) << 32) | __float_as_uint(a);
+}
+
+// rint(RN((x - z)/s)) + 1.5 * 2^23 as fp32 bits, two lanes at once (Markstein: q0 = d r,
+// e = d - s q0, q = q0 + e r)
+__device__ __forceinline__ uint64_t code2_bits(uint64_t x2, uint64_t z2, uint64_t r2, uint64_t ns2, uint64_t m2)
+{
+    uint64_t d, q0, e, q, y;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x2), "l"(z2));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(d), "l"(r2));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e) : "l"(ns2), "l"(q0), "l"(d));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(e), "l"(r2), "l"(q0));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(q), "l"(m2));
+    return y;
+}
+
+struct GroupGrid {
+    uint64_t z2, r2, ns2;
+    uint32_t packed;
+    bool finite;
+};
+
+template <int L, int G>
+__device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2])
+{
+    __half2 mn2 = *reinterpret_cast<const __half2*>(&h[0]), mx2 = mn2;
+#pragma unroll
+    for (int i = 1; i < G / 2; ++i) {
+        const __half2 v = *reinterpret_cast<const __half2*>(&h[i]);
+        mn2 = __hmin2_nan(mn2, v);
+        mx2 = __hmax2_nan(mx2, v);
+    }
+    const float mn = __half2float(__hmin_nan(__low2half(mn2), __high2half(mn2)));
+    const float mx = __half2float(__hmax_nan(__low2half(mx2), __high2half(mx2)));
+    GroupGrid g;
+    g.finite = fabsf(mn) <= 65504.0f && fabsf(mx) <= 65504.0f;
+    const uint16_t s16 = scale_half_ru(__fdiv_rn(__fsub_rn(mx, mn), (float)(L - 1)));
+    const uint16_t z16 = zero_half(mn);
+    const float s = h2f(s16), z = h2f(z16);
+    const float r = s != 0.0f ? __frcp_rn(s) : 0.0f;
+    g.z2 = f2_pack(z, z);
+    g.r2 = f2_pack(r, r);
+    g.ns2 = f2_pack(-s, -s);
+    g.packed = (uint32_t)s16 | ((uint32_t)z16 << 16);
+    return g;
+}
+
+// codes (as magic-offset fp32 bits) of one group's G values, two at a time, handed to `sink(i, bits)`
+template <int L, int G, typename Sink>
+__device__ __forceinline__ void group_codes(const uint32_t (&h)[G / 2], const GroupGrid& g, Sink&& sink)
+{
+    const uint64_t m2 = f2_pack(12582912.0f, 12582912.0f);
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) {
+        const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+        uint64_t y = code2_bits(f2_pack(xf.x, xf.y), g.z2, g.r2, g.ns2, m2);
+        uint32_t b0 = (uint32_t)y, b1 = (uint32_t)(y >> 32);
+        if constexpr (L == 2) {  // the only level count whose codes can exceed L - 1 (saturated scale)
+            b0 = min(b0, 0x4B400001u);
+            b1 = min(b1, 0x4B400001u);
+        }
+        sink(2 * i, b0);
+        sink(2 * i + 1, b1);
+    }
+}
+
+template <int L, int G>
+__device__ __forceinline__ void quantize_tile_fast(uint16_t* Ks, uint16_t* Vs, uint32_t* kw, uint32_t* vw,
+                                                   uint32_t* kz, uint32_t* vz, int tid, bool& bad)
+{
+    constexpr int D = 128, k = radix_k(L), WK = ceil_div(D, k), WV = ceil_div(TILE, k), NG = D / G;
+    // ---- K row `tid`
+    {
+        uint32_t w[WK];
+#pragma unroll
+        for (int j = 0; j < WK; ++j) w[j] = 0u;
+        const uint16_t* row = Ks + tid * QROW;
+#pragma unroll
+        for (int grp = 0; grp < NG; ++grp) {
+            uint32_t h[G / 2];
+#pragma unroll
+            for (int i = 0; i < G / 8; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(row + grp * G + 8 * i);
+                h[4 * i] = v.x;
+                h[4 * i + 1] = v.y;
+                h[4 * i + 2] = v.z;
+                h[4 * i + 3] = v.w;
+            }
+            const GroupGrid g = group_grid<L, G>(h);
+            bad |= !g.finite;
+            kz[grp * TILE + tid] = g.packed;
+            group_codes<L, G>(h, g, [&](int i, uint32_t bits) {
+                const int d = grp * G + i;
+                w[d / k] += bits * upow(L, d % k);
+            });
+        }
+#pragma unroll
+        for (int j = 0; j < WK; ++j) {
+            const int cnt = (j + 1) * k <= D ? k : D - j * k;
+            kw[j * TILE + tid] = w[j] - magic_sum(L, cnt);
+        }
+    }
+    // ---- V row `tid`: grids, and its codes as bytes over the first half of its own row
+    {
+        uint16_t* row = Vs + tid * QROW;
+        uint32_t packed[NG];
+        uint32_t bytes[D / 4];
+#pragma unroll
+        for (int grp = 0; grp < NG; ++grp) {
+            uint32_t h[G / 2];
+#pragma unroll
+            for (int i = 0; i < G / 8; ++i) {
+                const uint4 v = *reinterpret_cast<const uint4*>(row + grp * G + 8 * i);
+                h[4 * i] = v.x;
+                h[4 * i + 1] = v.y;
+                h[4 * i + 2] = v.z;
+                h[4 * i + 3] = v.w;
+            }
+            const GroupGrid g = group_grid<L, G>(h);
+            bad |= !g.finite;
+            packed[grp] = g.packed;
+            // the low byte of each magic sum is the code: byte i%4 of word i/4
+            group_codes<L, G>(h, g, [&](int i, uint32_t b) {
+                const int c = grp * G + i;
+                constexpr uint32_t sel[4] = {0x3214u, 0x3240u, 0x3410u, 0x4210u};
+                bytes[c / 4] = (c % 4 == 0) ? (b & 0xffu) : __byte_perm(bytes[c / 4], b, sel[c % 4]);
+            });
+        }
+#pragma unroll
+        for (int grp = 0; grp < NG; ++grp) vz[grp * TILE + tid] = packed[grp];
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i)
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(row) + 16 * i) =
+                make_uint4(bytes[4 * i], bytes[4 * i + 1], bytes[4 * i + 2], bytes[4 * i + 3]);
+    }
+    __syncthreads();
+    // ---- V channel `tid` across the tile's slots
+    {
+        uint32_t w[WV];
+#pragma unroll
+        for (int j = 0; j < WV; ++j) w[j] = 0u;
+        const unsigned char* cb = reinterpret_cast<const unsigned char*>(Vs) + tid;
+#pragma unroll
+        for (int t = 0; t < TILE; ++t) w[t / k] += (uint32_t)cb[t * QROW * 2] * upow(L, t % k);
+#pragma unroll
+        for (int j = 0; j < WV; ++j) vw[j * D + tid] = w[j];
+    }
+}
+
+template <int LH, int LL, int G>
+__global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
+                                                        const uint16_t* __restrict__ V,
+                                                        const uint32_t* __restrict__ bitmap,
+                                                        const uint32_t* __restrict__ rank, int T, int words_cap,
+                                                        int32_t* __restrict__ status)
+{
+    constexpr int D = 128, NG = D / G;
+    const int per_unit = hi.tiles_cap + lo.tiles_cap;
+    const int u = blockIdx.x / per_unit;
+    int tile = blockIdx.x % per_unit;
+    const bool is_hi = tile < hi.tiles_cap;
+    const QuantSeg& seg = is_hi ? hi : lo;
+    if (!is_hi) tile -= hi.tiles_cap;
+    const int tid = threadIdx.x;
+    const int n = seg.n[u];
+    const int s0 = tile * TILE;
+    if (s0 >= n) return;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
+    uint16_t* Vs = Ks + TILE * QROW;
+    int* tok = reinterpret_cast<int*>(Vs + TILE * QROW);
+    __shared__ __align__(8) uint64_t bar;
+    if (!gather_rows(Ks, Vs, tok, &bar, is_hi, u, s0, min(TILE, n - s0), K, V, bitmap, rank, T, words_cap, status))
+        return;
+
+    const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
+    const int W_hi = ceil_div(D, radix_k(LH)), W_lo = ceil_div(D, radix_k(LL));
+    const int Wd = is_hi ? W_hi : W_lo;
+    uint32_t* kw = seg.k + tile_base * Wd * TILE;
+    uint32_t* vw = seg.v + tile_base * Wd * D;
+    uint32_t* kz = seg.kz + tile_base * NG * TILE;
+    uint32_t* vz = seg.vz + tile_base * NG * TILE;
+    bool bad = false;
+    if (is_hi) quantize_tile_fast<LH, G>(Ks, Vs, kw, vw, kz, vz, tid, bad);
+    else quantize_tile_fast<LL, G>(Ks, Vs, kw, vw, kz, vz, tid, bad);
+    if (bad && tid < n - s0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
+}
+
 static size_t quantize_smem(int G)
 {
     return (size_t)2 * TILE * QROW * 2 + TILE * 4 + (size_t)TILE * (128 / G) * 16;
@@ -301,10 +532,23 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
         q.is_hi = s.is_hi;
         return q;
     };
+    const unsigned grid = (unsigned)units * per_unit;
+    const QuantSeg qh = conv(shi), ql = conv(slo);
+    // compile-time level pairs and group sizes of the common configurations
+#define SEMKV_QF(LH, LL, GG)                                                                                  \
+    if (shi.L == LH && slo.L == LL && G == GG) {                                                              \
+        const size_t sm = (size_t)2 * TILE * QROW * 2 + TILE * 4;                                             \
+        cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+        k_quantize_fast<LH, LL, GG><<<grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, words_cap, status);   \
+        return;                                                                                               \
+    }
+#define SEMKV_QF_G(LH, LL) SEMKV_QF(LH, LL, 32) SEMKV_QF(LH, LL, 64) SEMKV_QF(LH, LL, 128)
+    SEMKV_QF_G(8, 5) SEMKV_QF_G(6, 5) SEMKV_QF_G(8, 6) SEMKV_QF_G(16, 8) SEMKV_QF_G(5, 4)
+#undef SEMKV_QF_G
+#undef SEMKV_QF
     const size_t sm = quantize_smem(G);
     cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_quantize<<<(unsigned)units * per_unit, 128, sm, st>>>(conv(shi), conv(slo), K, V, bitmap, rank, T, G, words_cap,
-                                                             status);
+    k_quantize<<<grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, G, words_cap, status);
 }
 
 }  // namespace semkv
