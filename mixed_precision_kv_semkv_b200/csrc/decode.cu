@@ -219,6 +219,8 @@ __global__ void __launch_bounds__(128) k_decode_merge(const float* __restrict__ 
 {
     constexpr int D = 128;
     const int u = blockIdx.x / g, h = blockIdx.x % g, d = threadIdx.x, lane = d & 31, warp = d >> 5;
+    // launched as a programmatic dependent of the split kernels: wait for them (and their writes)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const float* base = ws + (size_t)u * nsplit_total * g * (D + 2) + h * (D + 2);
     const size_t stride = (size_t)g * (D + 2);
     extern __shared__ float wts[];  // [nsplit_total]
@@ -241,9 +243,17 @@ __global__ void __launch_bounds__(128) k_decode_merge(const float* __restrict__ 
     if (lane == 0) redl[warp] = l;
     __syncthreads();
     const float Ls = redl[0] + redl[1] + redl[2] + redl[3];
-    float O = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < nsplit_total; ++s) O += wts[s] * base[s * stride + d];
+    float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+    int s = 0;
+#pragma unroll 4
+    for (; s + 4 <= nsplit_total; s += 4) {  // independent loads, four accumulators
+        O0 += wts[s] * base[s * stride + d];
+        O1 += wts[s + 1] * base[(s + 1) * stride + d];
+        O2 += wts[s + 2] * base[(s + 2) * stride + d];
+        O3 += wts[s + 3] * base[(s + 3) * stride + d];
+    }
+    for (; s < nsplit_total; ++s) O0 += wts[s] * base[s * stride + d];
+    const float O = (O0 + O1) + (O2 + O3);
     out[((size_t)u * g + h) * D + d] = Ls > 0.f ? O / Ls : 0.f;
 }
 
@@ -283,8 +293,17 @@ void launch_decode_merge(const float* ws, int units, int H, int g, int D, int ns
 {
     (void)H;
     (void)D;
-    k_decode_merge<<<units * g, 128, (size_t)(nsplit_total > 0 ? nsplit_total : 1) * sizeof(float), st>>>(
-        ws, g, nsplit_total, out);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * g));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = (size_t)(nsplit_total > 0 ? nsplit_total : 1) * sizeof(float);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, k_decode_merge, ws, g, nsplit_total, out);
 }
 
 }  // namespace semkv

@@ -27,26 +27,27 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase)
+// One potentially blocking test of the phase parity: the thread may sleep until the phase
+// completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase, uint32_t hint_ns)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
 
-// Poll the barrier's phase parity; false after `limit` unsuccessful polls (~ms scale).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = 1u << 22)
+// Wait for the barrier's phase parity; false after `limit` tests (each sleeps at most ~hint_ns, so
+// the wait is bounded by about a second).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = 1u << 16)
 {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_test(bar, phase)) return true;
-        if (i > 64) __nanosleep(64);
-    }
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_test(bar, phase, 20000u)) return true;
     return false;
 }
 

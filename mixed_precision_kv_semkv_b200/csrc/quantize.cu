@@ -5,7 +5,8 @@
 // (max - min)/(L - 1) (saturated at 65504), z = min, code = clamp(rint((x - z)/s), 0, L - 1),
 // with IEEE fp32 subtract and divide and ties to even.
 //
-// One launch covers both segments; one CTA (4 warps) per 128-slot output tile:
+// One launch covers both segments; one CTA (4 warps) per 128-slot output tile (the compile-time
+// path uses two CTAs per tile, one for its K rows and one for its V rows):
 //   1. warp 0 maps the tile's slots to token indices (32-ary search of the rank directory for the
 //      first bitmap word, then a ballot scan), and fetches each token's K and V row (256 B each)
 //      with one cp.async.bulk per row into shared memory, completing on an mbarrier; the other
@@ -73,10 +74,11 @@ __device__ __forceinline__ uint32_t code_of(float x, const Grid& g, float top)
     return __float_as_uint(__fadd_rn(q, 12582912.0f)) - 0x4B400000u;
 }
 
-// Slots [s0, s0 + nv) of a segment of unit u -> token indices (tok), and each token's K and V row
-// (256 B each) into shared memory: warp 0 searches the rank directory (32-ary) for the first
-// bitmap word, scans the following words with ballots, and issues one cp.async.bulk per row on
-// `bar`; rows of slots past nv are zeroed.  Returns false (status set) if the copies timed out.
+// Slots [s0, s0 + nv) of a segment of unit u -> token indices (tok), and each token's K row and V
+// row (256 B each; V/Vs may be null) into shared memory: warp 0 searches the rank directory
+// (32-ary) for the first bitmap word, scans the following words with ballots, and issues one
+// cp.async.bulk per row on `bar`; rows of slots past nv are zeroed.  Returns false (status set)
+// if the copies timed out.
 __device__ __forceinline__ bool gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok, uint64_t* bar, bool is_hi, int u,
                                             int s0, int nv, const uint16_t* __restrict__ K,
                                             const uint16_t* __restrict__ V, const uint32_t* __restrict__ bitmap,
@@ -136,18 +138,19 @@ __device__ __forceinline__ bool gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok
         for (int r = lane; r < nv; r += 32) valid_rows += (tok[r] >= 0 && tok[r] < T);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) valid_rows += __shfl_xor_sync(0xffffffffu, valid_rows, o);
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)valid_rows * 2u * D * 2u);
+        const uint32_t mats = V ? 2u : 1u;
+        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)valid_rows * mats * D * 2u);
         __syncwarp();
         for (int r = lane; r < nv; r += 32) {
             const int t = tok[r];
             if (t >= 0 && t < T) {
                 const size_t off = ((size_t)u * T + t) * D;
                 bulk_g2s(Ks + r * QROW, K + off, D * 2, bar);
-                bulk_g2s(Vs + r * QROW, V + off, D * 2, bar);
+                if (V) bulk_g2s(Vs + r * QROW, V + off, D * 2, bar);
             } else {
                 for (int i = 0; i < D; i += 8) {
                     *reinterpret_cast<uint4*>(Ks + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4*>(Vs + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
+                    if (V) *reinterpret_cast<uint4*>(Vs + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
         }
@@ -155,7 +158,7 @@ __device__ __forceinline__ bool gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok
         for (int r = nv + (tid - 32); r < TILE; r += 96) {
             for (int i = 0; i < D; i += 8) {
                 *reinterpret_cast<uint4*>(Ks + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(Vs + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
+                if (V) *reinterpret_cast<uint4*>(Vs + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
     }
@@ -384,12 +387,11 @@ __device__ __forceinline__ void group_codes(const uint32_t (&h)[G / 2], const Gr
     }
 }
 
+// K rows of a tile: thread `tid` quantizes row tid and packs it along the channels
 template <int L, int G>
-__device__ __forceinline__ void quantize_tile_fast(uint16_t* Ks, uint16_t* Vs, uint32_t* kw, uint32_t* vw,
-                                                   uint32_t* kz, uint32_t* vz, int tid, bool& bad)
+__device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw, uint32_t* kz, int tid, bool& bad)
 {
-    constexpr int D = 128, k = radix_k(L), WK = ceil_div(D, k), WV = ceil_div(TILE, k), NG = D / G;
-    // ---- K row `tid`
+    constexpr int D = 128, k = radix_k(L), WK = ceil_div(D, k), NG = D / G;
     {
         uint32_t w[WK];
 #pragma unroll
@@ -420,7 +422,14 @@ __device__ __forceinline__ void quantize_tile_fast(uint16_t* Ks, uint16_t* Vs, u
             kw[j * TILE + tid] = w[j] - magic_sum(L, cnt);
         }
     }
-    // ---- V row `tid`: grids, and its codes as bytes over the first half of its own row
+}
+
+// V rows of a tile: thread `tid` writes the grids of row tid and its codes as bytes over the first
+// half of its own row; after a barrier thread `tid` packs channel tid along the tile's slots
+template <int L, int G>
+__device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint32_t* vz, int tid, bool& bad)
+{
+    constexpr int D = 128, k = radix_k(L), WV = ceil_div(TILE, k), NG = D / G;
     {
         uint16_t* row = Vs + tid * QROW;
         uint32_t packed[NG];
@@ -476,8 +485,9 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
 {
     constexpr int D = 128, NG = D / G;
     const int per_unit = hi.tiles_cap + lo.tiles_cap;
-    const int u = blockIdx.x / per_unit;
-    int tile = blockIdx.x % per_unit;
+    const int part = blockIdx.x & 1;  // 0: K rows, 1: V rows of the tile
+    const int u = (blockIdx.x >> 1) / per_unit;
+    int tile = (blockIdx.x >> 1) % per_unit;
     const bool is_hi = tile < hi.tiles_cap;
     const QuantSeg& seg = is_hi ? hi : lo;
     if (!is_hi) tile -= hi.tiles_cap;
@@ -487,23 +497,28 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
     if (s0 >= n) return;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
-    uint16_t* Vs = Ks + TILE * QROW;
-    int* tok = reinterpret_cast<int*>(Vs + TILE * QROW);
+    uint16_t* Xs = reinterpret_cast<uint16_t*>(smem);  // this CTA's rows: K rows or V rows
+    int* tok = reinterpret_cast<int*>(Xs + TILE * QROW);
     __shared__ __align__(8) uint64_t bar;
-    if (!gather_rows(Ks, Vs, tok, &bar, is_hi, u, s0, min(TILE, n - s0), K, V, bitmap, rank, T, words_cap, status))
+    if (!gather_rows(Xs, nullptr, tok, &bar, is_hi, u, s0, min(TILE, n - s0), part ? V : K, nullptr, bitmap, rank, T,
+                     words_cap, status))
         return;
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     const int W_hi = ceil_div(D, radix_k(LH)), W_lo = ceil_div(D, radix_k(LL));
     const int Wd = is_hi ? W_hi : W_lo;
-    uint32_t* kw = seg.k + tile_base * Wd * TILE;
-    uint32_t* vw = seg.v + tile_base * Wd * D;
-    uint32_t* kz = seg.kz + tile_base * NG * TILE;
-    uint32_t* vz = seg.vz + tile_base * NG * TILE;
     bool bad = false;
-    if (is_hi) quantize_tile_fast<LH, G>(Ks, Vs, kw, vw, kz, vz, tid, bad);
-    else quantize_tile_fast<LL, G>(Ks, Vs, kw, vw, kz, vz, tid, bad);
+    if (part == 0) {
+        uint32_t* kw = seg.k + tile_base * Wd * TILE;
+        uint32_t* kz = seg.kz + tile_base * NG * TILE;
+        if (is_hi) quantize_k_rows<LH, G>(Xs, kw, kz, tid, bad);
+        else quantize_k_rows<LL, G>(Xs, kw, kz, tid, bad);
+    } else {
+        uint32_t* vw = seg.v + tile_base * Wd * D;
+        uint32_t* vz = seg.vz + tile_base * NG * TILE;
+        if (is_hi) quantize_v_rows<LH, G>(Xs, vw, vz, tid, bad);
+        else quantize_v_rows<LL, G>(Xs, vw, vz, tid, bad);
+    }
     if (bad && tid < n - s0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
 }
 
@@ -537,9 +552,9 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     // compile-time level pairs and group sizes of the common configurations
 #define SEMKV_QF(LH, LL, GG)                                                                                  \
     if (shi.L == LH && slo.L == LL && G == GG) {                                                              \
-        const size_t sm = (size_t)2 * TILE * QROW * 2 + TILE * 4;                                             \
+        const size_t sm = (size_t)TILE * QROW * 2 + TILE * 4;                                                 \
         cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        k_quantize_fast<LH, LL, GG><<<grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, words_cap, status);   \
+        k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, words_cap, status); \
         return;                                                                                               \
     }
 #define SEMKV_QF_G(LH, LL) SEMKV_QF(LH, LL, 32) SEMKV_QF(LH, LL, 64) SEMKV_QF(LH, LL, 128)

@@ -4,11 +4,13 @@
 // top fraction is stored at the finer of two neighbouring precisions.  Ties: equal scores are
 // taken in increasing token order (-0 and +0 are equal).
 //
-// One CTA of 1024 threads per unit.  The n_hi-th largest key K* is found by a most-significant-
+// The n_hi-th largest key K* is found by a most-significant-
 // digit radix select over the order-preserving uint32 image of the scores (4 passes of 8 bits,
-// shared-memory histograms; the scores stay in L2 between passes).  A final pass forms each
+// shared-memory histograms).  A final pass forms each
 // bitmap word from warp ballots (key > K*, key == K*), takes the first (n_hi - #greater) ties in
 // token order with a block-wide exclusive scan, and writes the rank directory with a second scan.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -146,9 +148,184 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
     }
 }
 
+// ------------------------------------------------------------------ cluster version
+//
+// The same selection spread over a cluster of SEL_CS CTAs (512 threads each) per unit.  CTA c owns
+// a contiguous range of bitmap words; each thread keeps its KPT keys in registers.  Every radix
+// pass builds per-CTA histograms; each CTA then sums all SEL_CS histograms through distributed
+// shared memory and finds the same bin, so no broadcast is needed.  The bitmap pass takes the tie
+// and one counts of the earlier CTAs from distributed shared memory for its prefix sums.
+
+constexpr int SEL_CS = 8, SEL_THREADS = 512, SEL_WARPS = SEL_THREADS / 32;
+
+template <int KPT>
+__global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
+    k_select_cluster(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
+                     uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
+                     float* __restrict__ tau_out, int32_t* __restrict__ status)
+{
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int c = (int)cluster.block_rank();
+    const int u = blockIdx.x / SEL_CS;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const float* s = scores + (size_t)u * T;
+    const int nwords = (T + 31) / 32;
+    const int wpc = (nwords + SEL_CS - 1) / SEL_CS;  // words per CTA
+    const int w0 = min(nwords, c * wpc), w1 = min(nwords, w0 + wpc);
+    const int tok0 = 32 * w0;
+
+    __shared__ uint32_t hist[256];
+    __shared__ uint32_t gtm[KPT * SEL_WARPS], eqm[KPT * SEL_WARPS];
+    __shared__ uint32_t scan_tmp[33];
+    __shared__ uint32_t totals[2];  // this CTA's ties and strictly-greater counts
+    __shared__ uint32_t sh_prefix, sh_remaining;
+
+    // my keys: tokens tok0 + j*512 + tid (j < KPT) that fall in my CTA's range and below T
+    uint32_t key[KPT];
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int t = tok0 + j * SEL_THREADS + tid;
+        const bool in = t < 32 * w1 && t < T;
+        const float f = in ? s[t] : 0.f;
+        bad |= in && isnan(f);
+        key[j] = in ? score_key(f) : 0u;
+    }
+    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, SEMKV_STATUS_NAN_SCORE);
+
+    uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)n_hi;
+    if (n_hi > 0) {
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            if (tid < 256) hist[tid] = 0u;
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < KPT; ++j) {
+                const int t = tok0 + j * SEL_THREADS + tid;
+                if (t < 32 * w1 && t < T && (key[j] & mask) == prefix) atomicAdd(&hist[(key[j] >> shift) & 255u], 1u);
+            }
+            cluster.sync();  // every CTA's histogram of this pass is complete
+            if (wid == 0) {
+                uint32_t cnt[8], sum = 0u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) cnt[j] = 0u;
+                for (int r = 0; r < SEL_CS; ++r) {
+                    const uint32_t* rh = cluster.map_shared_rank(hist, r);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) cnt[j] += rh[255 - 8 * lane - j];
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sum += cnt[j];
+                const uint32_t inc = warp_incl_scan(sum);
+                const uint32_t exc = inc - sum;
+                if (exc < remaining && remaining <= inc) {
+                    uint32_t cum = exc;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (cum + cnt[j] >= remaining) {
+                            sh_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+                            sh_remaining = remaining - cum;
+                            break;
+                        }
+                        cum += cnt[j];
+                    }
+                }
+            }
+            cluster.sync();  // all remote reads of this pass are done before the histograms are reset
+            prefix = sh_prefix;
+            remaining = sh_remaining;
+            mask |= 255u << shift;
+        }
+    } else {
+        prefix = 0xffffffffu;
+        remaining = 0u;
+    }
+    const uint32_t kstar = prefix, take = remaining;
+
+    // ---- word masks of my range (word w0 + j*SEL_WARPS + wid is formed by warp wid at step j)
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int t = tok0 + j * SEL_THREADS + tid;
+        const bool in = t < 32 * w1 && t < T;
+        const uint32_t gt = __ballot_sync(0xffffffffu, in && key[j] > kstar);
+        const uint32_t eq = __ballot_sync(0xffffffffu, in && key[j] == kstar);
+        if (lane == 0) {
+            gtm[j * SEL_WARPS + wid] = gt;
+            eqm[j * SEL_WARPS + wid] = eq;
+        }
+    }
+    __syncthreads();
+    const int nw = w1 - w0;  // <= KPT * SEL_WARPS
+    uint32_t my_gt = 0u, my_eq = 0u;
+    if (tid < nw) {
+        my_gt = gtm[tid];
+        my_eq = eqm[tid];
+    }
+    uint32_t tot_ties, tot_gt;
+    uint32_t ties_before = block_excl_scan((uint32_t)__popc(my_eq), scan_tmp, &tot_ties);
+    block_excl_scan((uint32_t)__popc(my_gt), scan_tmp, &tot_gt);
+    if (tid == 0) {
+        totals[0] = tot_ties;
+        totals[1] = tot_gt;
+    }
+    cluster.sync();
+    // ties and ones of the earlier CTAs
+    uint32_t cta_ties_before = 0u, cta_ones_before = 0u;
+    for (int r = 0; r < c; ++r) {
+        const uint32_t* rt = cluster.map_shared_rank(totals, r);
+        const uint32_t rties = rt[0], rgt = rt[1];
+        const uint32_t taken = cta_ties_before >= take ? 0u : min(rties, take - cta_ties_before);
+        cta_ones_before += rgt + taken;
+        cta_ties_before += rties;
+    }
+    ties_before += cta_ties_before;
+    uint32_t take_mask = 0u;
+    if (ties_before < take) {
+        const uint32_t need = take - ties_before;
+        if (need >= (uint32_t)__popc(my_eq)) {
+            take_mask = my_eq;
+        } else {
+            const uint32_t pos = __fns(my_eq, 0u, (int)need);
+            take_mask = my_eq & (0xffffffffu >> (31u - pos));
+        }
+    }
+    const uint32_t word = my_gt | take_mask;
+    uint32_t tot_ones;
+    const uint32_t ones_before = cta_ones_before + block_excl_scan((uint32_t)__popc(word), scan_tmp, &tot_ones);
+    uint32_t* bm = bitmap + (size_t)u * words_cap;
+    uint32_t* rk = rank + (size_t)u * words_cap;
+    if (tid < nw) {
+        bm[w0 + tid] = word;
+        rk[w0 + tid] = ones_before;
+    }
+    for (int w = nwords + c * SEL_THREADS + tid; w < words_cap; w += SEL_CS * SEL_THREADS) {
+        bm[w] = 0u;
+        rk[w] = (uint32_t)n_hi;
+    }
+    if (c == 0 && tid == 0) {
+        n_hi_out[u] = n_hi;
+        n_lo_out[u] = T - n_hi;
+        tau_out[u] = n_hi > 0 ? key_score(kstar) : __int_as_float(0x7f800000);
+    }
+    cluster.sync();  // no CTA leaves while another may still read its shared memory
+}
+
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st)
 {
+    const int nwords = (T + 31) / 32;
+    const int wpc = (nwords + SEL_CS - 1) / SEL_CS;
+    const int kpt = (wpc * 32 + SEL_THREADS - 1) / SEL_THREADS;  // keys per thread
+    const dim3 grid((unsigned)(units * SEL_CS));
+#define SEMKV_SEL(K)                                                                                           \
+    if (kpt <= K) {                                                                                            \
+        k_select_cluster<K><<<grid, SEL_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, \
+                                                          n_lo_out, tau, status);                             \
+        return;                                                                                                \
+    }
+    SEMKV_SEL(1) SEMKV_SEL(2) SEMKV_SEL(4) SEMKV_SEL(8) SEMKV_SEL(16) SEMKV_SEL(32)
+#undef SEMKV_SEL
+    // more than 32 keys per thread: the one-CTA-per-unit kernel streams the scores from L2
     k_select<<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau, status);
 }
 
