@@ -212,28 +212,33 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
 }
 
 // Log-sum-exp merge of the split partials of one (unit, query head): all splits' maxima are read
-// in parallel, the weights 2^(m_s - M) go to shared memory, then thread d sums o_s[d] with
-// independent loads.
-__global__ void __launch_bounds__(128) k_decode_merge(const float* __restrict__ ws, int g, int nsplit_total,
-                                                       float* __restrict__ out)
+// in parallel, the weights 2^(m_s - M) go to shared memory, then four slices of 128 threads each
+// sum a quarter of the splits of o_s[d] with independent loads, and the slices are added.
+constexpr int MERGE_SLICES = 4;
+
+__global__ void __launch_bounds__(128 * MERGE_SLICES) k_decode_merge(const float* __restrict__ ws, int g,
+                                                                      int nsplit_total, float* __restrict__ out)
 {
-    constexpr int D = 128;
-    const int u = blockIdx.x / g, h = blockIdx.x % g, d = threadIdx.x, lane = d & 31, warp = d >> 5;
+    constexpr int D = 128, NT = 128 * MERGE_SLICES;
     // launched as a programmatic dependent of the split kernels: wait for them (and their writes)
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int u = blockIdx.x / g, h = blockIdx.x % g;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, d = tid & (D - 1), slice = tid / D;
     const float* base = ws + (size_t)u * nsplit_total * g * (D + 2) + h * (D + 2);
     const size_t stride = (size_t)g * (D + 2);
     extern __shared__ float wts[];  // [nsplit_total]
-    __shared__ float red[4], redl[4];
+    __shared__ float red[NT / 32], redl[NT / 32], part[MERGE_SLICES][D];
     const float NEG = -__int_as_float(0x7f800000);
     float M = NEG;
-    for (int s = d; s < nsplit_total; s += 128) M = fmaxf(M, base[s * stride + D]);
+    for (int s = tid; s < nsplit_total; s += NT) M = fmaxf(M, base[s * stride + D]);
     M = warp_max(M);
     if (lane == 0) red[warp] = M;
     __syncthreads();
-    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    M = NEG;
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) M = fmaxf(M, red[i]);
     float l = 0.f;
-    for (int s = d; s < nsplit_total; s += 128) {
+    for (int s = tid; s < nsplit_total; s += NT) {
         const float w = M == NEG ? 0.f : exp2f(base[s * stride + D] - M);
         wts[s] = w;
         l += w * base[s * stride + D + 1];
@@ -242,19 +247,25 @@ __global__ void __launch_bounds__(128) k_decode_merge(const float* __restrict__ 
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     if (lane == 0) redl[warp] = l;
     __syncthreads();
-    const float Ls = redl[0] + redl[1] + redl[2] + redl[3];
-    float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-    int s = 0;
+    float Ls = 0.f;
+#pragma unroll
+    for (int i = 0; i < NT / 32; ++i) Ls += redl[i];
+    float O0 = 0.f, O1 = 0.f;
+    int s = slice;
 #pragma unroll 4
-    for (; s + 4 <= nsplit_total; s += 4) {  // independent loads, four accumulators
+    for (; s + MERGE_SLICES < nsplit_total; s += 2 * MERGE_SLICES) {  // two independent loads per step
         O0 += wts[s] * base[s * stride + d];
-        O1 += wts[s + 1] * base[(s + 1) * stride + d];
-        O2 += wts[s + 2] * base[(s + 2) * stride + d];
-        O3 += wts[s + 3] * base[(s + 3) * stride + d];
+        O1 += wts[s + MERGE_SLICES] * base[(s + MERGE_SLICES) * stride + d];
     }
-    for (; s < nsplit_total; ++s) O0 += wts[s] * base[s * stride + d];
-    const float O = (O0 + O1) + (O2 + O3);
-    out[((size_t)u * g + h) * D + d] = Ls > 0.f ? O / Ls : 0.f;
+    for (; s < nsplit_total; s += MERGE_SLICES) O0 += wts[s] * base[s * stride + d];
+    part[slice][d] = O0 + O1;
+    __syncthreads();
+    if (slice == 0) {
+        float O = 0.f;
+#pragma unroll
+        for (int i = 0; i < MERGE_SLICES; ++i) O += part[i][d];
+        out[((size_t)u * g + h) * D + d] = Ls > 0.f ? O / Ls : 0.f;
+    }
 }
 
 static size_t decode_smem(int NGg)
@@ -295,7 +306,7 @@ void launch_decode_merge(const float* ws, int units, int H, int g, int D, int ns
     (void)D;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * g));
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(128 * MERGE_SLICES);
     cfg.dynamicSmemBytes = (size_t)(nsplit_total > 0 ? nsplit_total : 1) * sizeof(float);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

@@ -201,8 +201,12 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
             __syncthreads();
 #pragma unroll
             for (int j = 0; j < KPT; ++j) {
+                // scores share few leading bytes: lanes with the same bin add once (warp-aggregated)
                 const int t = tok0 + j * SEL_THREADS + tid;
-                if (t < 32 * w1 && t < T && (key[j] & mask) == prefix) atomicAdd(&hist[(key[j] >> shift) & 255u], 1u);
+                const bool in = t < 32 * w1 && t < T && (key[j] & mask) == prefix;
+                const uint32_t bin = in ? (key[j] >> shift) & 255u : 256u;
+                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
             }
             cluster.sync();  // every CTA's histogram of this pass is complete
             if (wid == 0) {
