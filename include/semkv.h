@@ -148,6 +148,28 @@ SEMKV_API int semkv_append_token(const semkv_cache_t* cache, const uint16_t* k, 
 SEMKV_API int semkv_decode_attention(const semkv_cache_t* cache, const uint16_t* q, float softmax_scale, float* out,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of the fixed device scratch that semkv_decode_attention_noalloc uses (per GPU). */
+#define SEMKV_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* semkv_decode_attention without a workspace argument, for callers that cannot allocate device
+ * memory when they decode (for example a plugin in a server whose process has already given all
+ * device memory to its own pool allocator, or a service that forbids allocator calls after
+ * start-up).  There is no counterpart on the SemKV page: this is a deployment convenience.
+ * The split-K partials live in a fixed array of SEMKV_NOALLOC_SCRATCH_BYTES in device memory that
+ * is part of the library image; every GPU that loads the library holds one until the process
+ * exits.  Same arguments and results as semkv_decode_attention otherwise.
+ *   - Allocates nothing: no cudaMalloc/cudaFree and no allocating library routine is called.
+ *   - The first call on a device looks up the array's device address for that device
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any stream
+ *     capture on the device.
+ *   - Shapes whose workspace (semkv_workspace_bytes) exceeds SEMKV_NOALLOC_SCRATCH_BYTES are
+ *     rejected with SEMKV_ERR_CAPACITY before any launch.
+ *   - All calls on a device share the one array and it keeps the last call's contents; nothing in
+ *     it needs clearing (every partial is written before it is read), but two calls whose work
+ *     overlaps on the GPU (different streams, no ordering between them) race on it. */
+SEMKV_API int semkv_decode_attention_noalloc(const semkv_cache_t* cache, const uint16_t* q, float softmax_scale,
+                                             float* out, void* stream);
+
 /* Dequantize every token back to original token order (test and inspection path, not tuned).
  * K, V: device fp32 [B][H][T][D] outputs; T = n_hi + n_lo of every unit (else
  * SEMKV_STATUS_LENGTH_MISMATCH and the unit's rows are left as they were). */

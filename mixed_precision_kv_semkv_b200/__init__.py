@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     semkv_assign_precision,
     semkv_cache_bytes,
     semkv_decode_attention,
+    semkv_decode_attention_noalloc,
     semkv_dequantize,
     semkv_quantize_pack,
     semkv_radix_digits,

@@ -29,8 +29,9 @@ SHAPE_FIELDS = ("B", "H", "Hq", "D", "G", "L_hi", "L_lo", "cap_hi", "cap_lo", "T
 BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
              "bitmap", "rank", "n_hi", "n_lo", "tau", "status")
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
-            "semkv_append_token", "semkv_decode_attention", "semkv_dequantize", "semkv_status_string",
-            "semkv_radix_digits")
+            "semkv_append_token", "semkv_decode_attention", "semkv_decode_attention_noalloc", "semkv_dequantize",
+            "semkv_status_string", "semkv_radix_digits")
+NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
 class CacheStruct(ctypes.Structure):
@@ -62,6 +63,7 @@ def lib() -> ctypes.CDLL:
         L.semkv_quantize_pack.argtypes = [cp, vp, vp, i32, vp]
         L.semkv_append_token.argtypes = [cp, vp, vp, vp, vp]
         L.semkv_decode_attention.argtypes = [cp, vp, f32, vp, vp, sz, vp]
+        L.semkv_decode_attention_noalloc.argtypes = [cp, vp, f32, vp, vp]
         L.semkv_dequantize.argtypes = [cp, vp, vp, i32, vp]
         L.semkv_status_string.argtypes = [ctypes.c_int]
         L.semkv_status_string.restype = ctypes.c_char_p
@@ -139,6 +141,14 @@ def semkv_decode_attention(cache, q, softmax_scale: float, out, workspace, works
     return _check("semkv_decode_attention",
                   lib().semkv_decode_attention(ctypes.byref(_struct(cache)), _ptr(q), float(softmax_scale), _ptr(out),
                                                _ptr(workspace), nbytes, _stream(stream)))
+
+
+def semkv_decode_attention_noalloc(cache, q, softmax_scale: float, out, stream=None) -> int:
+    """Decode attention using the library's fixed device scratch instead of a workspace (for
+    callers that cannot allocate device memory when they decode)."""
+    return _check("semkv_decode_attention_noalloc",
+                  lib().semkv_decode_attention_noalloc(ctypes.byref(_struct(cache)), _ptr(q), float(softmax_scale),
+                                                       _ptr(out), _stream(stream)))
 
 
 def semkv_dequantize(cache, K, V, T: int, stream=None) -> int:
