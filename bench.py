@@ -73,6 +73,36 @@ def alg_bytes(w, T: int, n_hi: int) -> dict:
     }
 
 
+# ---------------------------------------------------------------- ranks (one process per GPU)
+
+
+def rank_env() -> tuple[int, int, int]:
+    """(world size, rank, local rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own independent units (weak scaling: the per-GPU work is fixed)."""
+    return 1000003 * rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's value (used for the timed region); no data-path collective."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, step_bytes: float, steps: int, total_ms: float) -> float:
+    """Whole-job GB/s: every rank moves step_bytes per step; time = the max over ranks."""
+    return world * step_bytes * steps / (total_ms * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------- clocks
 
 
@@ -197,9 +227,7 @@ def run_semkv(args):
     from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_assign_precision, semkv_decode_attention,
                                                semkv_quantize_pack, synth)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -212,7 +240,7 @@ def run_semkv(args):
     build.build()
     w = synth.WORKLOADS[args.workload]
     T = w.T
-    d = synth.layer_gpu(w, seed=rank)
+    d = synth.layer_gpu(w, seed=rank_seed(rank))
     K, V, S, q = d["K"], d["V"], d["scores"], d["q"]
     cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p)
     ws = cache.workspace()
@@ -274,12 +302,8 @@ def run_semkv(args):
     t_sel = sum(e[0].elapsed_time(e[1]) for e in evs)
     t_q = sum(e[1].elapsed_time(e[2]) for e in evs)
     t_dec = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms = t_sel + t_q + t_dec
-    if dist is not None:
-        tt = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    value = world * step_bytes * steps / (total_ms * 1e-3) / 1e9
+    total_ms = max_over_ranks(t_sel + t_q + t_dec, dist, "cuda")
+    value = weak_scaling_value(world, step_bytes, steps, total_ms)
 
     # decode alone over an L2-cold cache (decode-attn HBM GB/s of the metric)
     dec_ms = []

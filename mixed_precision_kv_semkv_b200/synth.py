@@ -242,3 +242,29 @@ def layer_gpu(w: Workload, seed: int, layer: int = 0, device: str = "cuda", T: i
             lg = torch.einsum("hqd,htd->hqt", qs[b], K[b].float()) * sm_scale(w.D)
             S[b] = torch.softmax(lg, dim=-1).sum(dim=1)
     return {"K": K, "V": V, "scores": S, "q": q}
+
+
+def gen_steps_gpu(w: Workload, K16, seed: int, layer: int, steps: int, device: str = "cuda"):
+    """Generated tokens on the GPU: new k, v fp16 [steps][B][H][D] with the prefill's per-channel
+    scales, their scores fp32 [steps][B][H] (softmax mass against 64 scoring queries, normalised by
+    those queries' prefill max and sum), and decode queries fp16 [steps][B][Hq][D]."""
+    import torch
+
+    B, H, T, D = K16.shape
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 1000 + layer + 500000)
+    sk = torch.empty((1, 1, H, D), device=device).log_normal_(0.0, w.sigma_c, generator=g)
+    sv = torch.empty((1, 1, H, D), device=device).log_normal_(0.0, w.sigma_c, generator=g)
+    kn = (torch.randn((steps, B, H, D), device=device, generator=g) * sk).to(torch.float16)
+    vn = (torch.randn((steps, B, H, D), device=device, generator=g) * sv).to(torch.float16)
+    qs = torch.randn((steps, B, w.Hq, D), device=device, generator=g).to(torch.float16)
+    qsc = torch.randn((B, H, 64, D), device=device, generator=g)
+    sc = torch.empty((steps, B, H), device=device, dtype=torch.float32)
+    scale = sm_scale(D)
+    for b in range(B):
+        lg = torch.einsum("hqd,htd->hqt", qsc[b], K16[b].float()) * scale  # [H][64][T]
+        m = lg.amax(dim=-1)                                                 # [H][64]
+        z = torch.exp(lg - m[..., None]).sum(dim=-1)                        # [H][64]
+        ln = torch.einsum("shd,hqd->shq", kn[:, b].float(), qsc[b]) * scale  # [steps][H][64]
+        sc[:, b] = (torch.exp(ln - m[None]) / z[None]).sum(dim=-1)
+    return {"k": kn, "v": vn, "scores": sc, "q": qs}
