@@ -336,7 +336,7 @@ def run_semkv(args):
     ach = per_kernel[dom]["gbs"]
     traffic = None
     try:
-        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic_llama8b_1L.json")))
         traffic = prof.get(dom)
     except (OSError, ValueError):
         pass
