@@ -334,11 +334,17 @@ def run_semkv(args):
     dom_name = {"select": "semkv_assign_precision (k_select)", "quantize": "semkv_quantize_pack (k_quantize)",
                 "decode_in_step": "semkv_decode_attention (k_decode_split + k_decode_merge)"}[dom]
     ach = per_kernel[dom]["gbs"]
-    traffic = None
+    traffic = None  # DRAM bytes per launch from the committed ncu capture, if the kernel is unchanged since
     try:
-        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic_llama8b_1L.json")))
-        traffic = prof.get(dom)
-    except (OSError, ValueError):
+        import hashlib
+
+        prof = json.load(open(os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")))
+        m = hashlib.sha256()
+        for f in prof["sources"][dom]:
+            m.update(open(os.path.join(ROOT, f), "rb").read())
+        if m.hexdigest() == prof["source_sha256"][dom]:
+            traffic = prof[dom]
+    except (OSError, ValueError, KeyError):
         pass
 
     e2e = None
