@@ -29,6 +29,9 @@ __device__ __forceinline__ float key_score(uint32_t k)
     return __uint_as_float(u);
 }
 
+// One CTA of 1024 threads per unit.  CACHED: the keys are first copied into shared memory (T up to
+// 48K tokens), otherwise every pass streams them from global memory (L2).
+template <bool CACHED>
 __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ scores, int T, int n_hi, int words_cap,
                                                   uint32_t* __restrict__ bitmap, uint32_t* __restrict__ rank,
                                                   int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
@@ -43,22 +46,34 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
     __shared__ uint32_t hist[256];
     __shared__ uint32_t scan_tmp[33];
     __shared__ uint32_t sh_prefix, sh_remaining;
+    extern __shared__ uint32_t kcache[];  // [T] when CACHED
 
     // NaN scores: flag; their keys sort above +inf (order unspecified, as documented)
     {
         bool bad = false;
-        for (int t = tid; t < T; t += blockDim.x) bad |= isnan(s[t]);
+#pragma unroll 8
+        for (int t = tid; t < T; t += blockDim.x) {
+            const float f = s[t];
+            bad |= isnan(f);
+            if (CACHED) kcache[t] = score_key(f);
+        }
         if (__syncthreads_or(bad) && tid == 0) atomicOr(status, SEMKV_STATUS_NAN_SCORE);
     }
+    auto key_at = [&](int t) -> uint32_t { return CACHED ? kcache[t] : score_key(s[t]); };
 
     uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)n_hi;
     if (n_hi > 0) {
         for (int shift = 24; shift >= 0; shift -= 8) {
             if (tid < 256) hist[tid] = 0u;
             __syncthreads();
-            for (int t = tid; t < T; t += blockDim.x) {
-                uint32_t key = score_key(s[t]);
-                if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+#pragma unroll 4
+            for (int t0 = 0; t0 < T; t0 += blockDim.x) {  // warp-uniform trip count: match_any needs full warps
+                const int t = t0 + tid;
+                const uint32_t key = t < T ? key_at(t) : 0u;
+                const bool in = t < T && (key & mask) == prefix;
+                const uint32_t bin = in ? (key >> shift) & 255u : 256u;
+                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
             }
             __syncthreads();
             if (wid == 0) {
@@ -106,7 +121,7 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
             int w = c + 32 * wid + j;
             if (w >= nwords) break;  // uniform across the warp
             int t = 32 * w + lane;
-            uint32_t key = t < T ? score_key(s[t]) : 0u;
+            uint32_t key = t < T ? key_at(t) : 0u;
             bool valid = t < T;
             uint32_t gt = __ballot_sync(0xffffffffu, valid && key > kstar);
             uint32_t eq = __ballot_sync(0xffffffffu, valid && key == kstar);
@@ -314,9 +329,147 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     cluster.sync();  // no CTA leaves while another may still read its shared memory
 }
 
+// ------------------------------------------------------------------ one CTA, keys in registers
+//
+// For T <= 32768 one CTA of 1024 threads per unit holds every key in registers (KPT per thread):
+// the radix passes re-read nothing and need no cross-CTA exchange.  Thread tid holds tokens
+// j*1024 + tid; warp w at step j forms bitmap word j*32 + w.
+
+constexpr int SELR_THREADS = 1024, SELR_WARPS = SELR_THREADS / 32;
+
+template <int KPT>
+__global__ void __launch_bounds__(SELR_THREADS)
+    k_select_reg(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
+                 uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
+                 float* __restrict__ tau_out, int32_t* __restrict__ status)
+{
+    const int u = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const float* s = scores + (size_t)u * T;
+    const int nwords = (T + 31) / 32;
+    __shared__ uint32_t hist[256];
+    __shared__ uint32_t gtm[KPT * SELR_WARPS], eqm[KPT * SELR_WARPS];
+    __shared__ uint32_t scan_tmp[33];
+    __shared__ uint32_t sh_prefix, sh_remaining;
+
+    uint32_t key[KPT];
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int t = j * SELR_THREADS + tid;
+        const float f = t < T ? s[t] : 0.f;
+        bad |= t < T && isnan(f);
+        key[j] = score_key(f);
+    }
+    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, SEMKV_STATUS_NAN_SCORE);
+
+    uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)n_hi;
+    if (n_hi > 0) {
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            if (tid < 256) hist[tid] = 0u;
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < KPT; ++j) {
+                const bool in = j * SELR_THREADS + tid < T && (key[j] & mask) == prefix;
+                const uint32_t bin = in ? (key[j] >> shift) & 255u : 256u;
+                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+            }
+            __syncthreads();
+            if (wid == 0) {
+                uint32_t cnt[8], sum = 0u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    cnt[j] = hist[255 - 8 * lane - j];
+                    sum += cnt[j];
+                }
+                const uint32_t inc = warp_incl_scan(sum);
+                const uint32_t exc = inc - sum;
+                if (exc < remaining && remaining <= inc) {
+                    uint32_t cum = exc;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (cum + cnt[j] >= remaining) {
+                            sh_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+                            sh_remaining = remaining - cum;
+                            break;
+                        }
+                        cum += cnt[j];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix = sh_prefix;
+            remaining = sh_remaining;
+            mask |= 255u << shift;
+        }
+    } else {
+        prefix = 0xffffffffu;
+        remaining = 0u;
+    }
+    const uint32_t kstar = prefix, take = remaining;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const bool in = j * SELR_THREADS + tid < T;
+        const uint32_t gt = __ballot_sync(0xffffffffu, in && key[j] > kstar);
+        const uint32_t eq = __ballot_sync(0xffffffffu, in && key[j] == kstar);
+        if (lane == 0) {
+            gtm[j * SELR_WARPS + wid] = gt;
+            eqm[j * SELR_WARPS + wid] = eq;
+        }
+    }
+    __syncthreads();
+    const uint32_t my_gt = tid < nwords ? gtm[tid] : 0u, my_eq = tid < nwords ? eqm[tid] : 0u;
+    uint32_t tot;
+    const uint32_t ties_before = block_excl_scan((uint32_t)__popc(my_eq), scan_tmp, &tot);
+    uint32_t take_mask = 0u;
+    if (ties_before < take) {
+        const uint32_t need = take - ties_before;
+        if (need >= (uint32_t)__popc(my_eq)) {
+            take_mask = my_eq;
+        } else {
+            const uint32_t pos = __fns(my_eq, 0u, (int)need);
+            take_mask = my_eq & (0xffffffffu >> (31u - pos));
+        }
+    }
+    const uint32_t word = my_gt | take_mask;
+    const uint32_t ones_before = block_excl_scan((uint32_t)__popc(word), scan_tmp, &tot);
+    uint32_t* bm = bitmap + (size_t)u * words_cap;
+    uint32_t* rk = rank + (size_t)u * words_cap;
+    if (tid < nwords) {
+        bm[tid] = word;
+        rk[tid] = ones_before;
+    }
+    for (int w = nwords + tid; w < words_cap; w += SELR_THREADS) {
+        bm[w] = 0u;
+        rk[w] = (uint32_t)n_hi;
+    }
+    if (tid == 0) {
+        n_hi_out[u] = n_hi;
+        n_lo_out[u] = T - n_hi;
+        tau_out[u] = n_hi > 0 ? key_score(kstar) : __int_as_float(0x7f800000);
+    }
+}
+
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st)
 {
+    const int kpt_reg = (T + SELR_THREADS - 1) / SELR_THREADS;
+#define SEMKV_SELR(K)                                                                                           \
+    if (kpt_reg <= K) {                                                                                         \
+        k_select_reg<K><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out,     \
+                                                        n_lo_out, tau, status);                                 \
+        return;                                                                                                 \
+    }
+    SEMKV_SELR(1) SEMKV_SELR(2) SEMKV_SELR(4) SEMKV_SELR(8) SEMKV_SELR(16)
+#undef SEMKV_SELR
+    if (T <= 48 * 1024) {  // keys cached in shared memory by one CTA
+        const size_t sm = (size_t)T * 4;
+        cudaFuncSetAttribute(k_select<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        k_select<true><<<units, 1024, sm, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
+                                                status);
+        return;
+    }
     const int nwords = (T + 31) / 32;
     const int wpc = (nwords + SEL_CS - 1) / SEL_CS;
     const int kpt = (wpc * 32 + SEL_THREADS - 1) / SEL_THREADS;  // keys per thread
@@ -330,7 +483,8 @@ void launch_select(const float* scores, int units, int T, int n_hi, int words_ca
     SEMKV_SEL(1) SEMKV_SEL(2) SEMKV_SEL(4) SEMKV_SEL(8) SEMKV_SEL(16) SEMKV_SEL(32)
 #undef SEMKV_SEL
     // more than 32 keys per thread: the one-CTA-per-unit kernel streams the scores from L2
-    k_select<<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau, status);
+    k_select<false><<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
+                                            status);
 }
 
 }  // namespace semkv

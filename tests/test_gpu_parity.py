@@ -53,6 +53,8 @@ def test_tiny_workload_all_outputs():
     (1, 1, 4, 700, 64, 256, 17, 0.5),
     (1, 1, 4, 500, 32, 100, 31, 0.4),
     (3, 1, 2, 4095, 64, 8, 5, 0.25),
+    (1, 1, 4, 20000, 64, 8, 5, 0.25),     # selection: keys cached in shared memory
+    (1, 1, 4, 140000, 128, 6, 5, 0.5),    # selection: scores streamed (more than a cluster holds)
 ])
 def test_ragged_shapes_and_levels(B, H, Hq, T, G, L_hi, L_lo, p):
     K, V, S, q = _rand_case(B, H, Hq, T, seed=T + L_hi)
