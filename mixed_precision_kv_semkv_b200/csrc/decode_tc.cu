@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     uint32_t ph_k = 0, ph_v = 0;
     bool timeout = false;
 
+    const uint32_t* lut_lane = lut + lane;  // this lane's copy: entry P at lut_lane[32 * P]
     // W words (from shared memory) -> KCP TMEM columns of this thread's lane
     auto unpack_to_tmem = [&](const uint32_t* words) {
         uint32_t chunk[8];
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
             for (int pp = 0; pp < NPAIR; ++pp) {
                 const unsigned long long t = (unsigned long long)f * (unsigned long long)(L * L);
                 f = (uint32_t)t;
-                chunk[ci++] = lut[((uint32_t)(t >> 32) << 5) + lane];
+                chunk[ci++] = lut_lane[(uint32_t)(t >> 32) << 5];
                 if (ci == 8) {
                     tmem_st8(lane_base + cbase, chunk);
                     cbase += 8;

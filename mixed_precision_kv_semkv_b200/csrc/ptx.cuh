@@ -27,6 +27,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// named barrier `id` over `count` threads (a multiple of 32)
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // One potentially blocking test of the phase parity: the thread may sleep until the phase
 // completes or about `hint_ns` nanoseconds pass.
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase, uint32_t hint_ns)

@@ -166,10 +166,15 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
 // ------------------------------------------------------------------ cluster version
 //
 // The same selection spread over a cluster of SEL_CS CTAs (512 threads each) per unit.  CTA c owns
-// a contiguous range of bitmap words; each thread keeps its KPT keys in registers.  Every radix
-// pass builds per-CTA histograms; each CTA then sums all SEL_CS histograms through distributed
-// shared memory and finds the same bin, so no broadcast is needed.  The bitmap pass takes the tie
-// and one counts of the earlier CTAs from distributed shared memory for its prefix sums.
+// a contiguous range of bitmap words; each thread keeps its KPT keys in registers.
+//   * the bits every key shares (cluster-wide AND / OR of the keys) are taken as known: the radix
+//     passes start at the highest bit where keys differ, so their digits are spread and plain
+//     shared-memory atomics see little contention;
+//   * every pass builds per-CTA histograms (two buffers, alternating); after one cluster barrier
+//     each CTA sums all SEL_CS histograms through distributed shared memory and finds the same bin,
+//     so nothing is broadcast;
+//   * the bitmap pass takes the tie and one counts of the earlier CTAs from distributed shared
+//     memory for its prefix sums.
 
 constexpr int SEL_CS = 8, SEL_THREADS = 512, SEL_WARPS = SEL_THREADS / 32;
 
@@ -190,15 +195,17 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     const int w0 = min(nwords, c * wpc), w1 = min(nwords, w0 + wpc);
     const int tok0 = 32 * w0;
 
-    __shared__ uint32_t hist[256];
+    __shared__ uint32_t hist[2][256];
     __shared__ uint32_t gtm[KPT * SEL_WARPS], eqm[KPT * SEL_WARPS];
     __shared__ uint32_t scan_tmp[33];
+    __shared__ uint32_t andor[2];   // this CTA's AND and OR of its keys
     __shared__ uint32_t totals[2];  // this CTA's ties and strictly-greater counts
-    __shared__ uint32_t sh_prefix, sh_remaining;
+    __shared__ uint32_t sh_prefix, sh_remaining, red_and[SEL_WARPS], red_or[SEL_WARPS];
 
     // my keys: tokens tok0 + j*512 + tid (j < KPT) that fall in my CTA's range and below T
     uint32_t key[KPT];
     bool bad = false;
+    uint32_t kand = 0xffffffffu, kor = 0u;
 #pragma unroll
     for (int j = 0; j < KPT; ++j) {
         const int t = tok0 + j * SEL_THREADS + tid;
@@ -206,30 +213,67 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
         const float f = in ? s[t] : 0.f;
         bad |= in && isnan(f);
         key[j] = in ? score_key(f) : 0u;
+        if (in) {
+            kand &= key[j];
+            kor |= key[j];
+        }
     }
     if (__syncthreads_or(bad) && tid == 0) atomicOr(status, SEMKV_STATUS_NAN_SCORE);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+        kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+    }
+    if (lane == 0) {
+        red_and[wid] = kand;
+        red_or[wid] = kor;
+    }
+    if (tid < 256) {
+        hist[0][tid] = 0u;
+        hist[1][tid] = 0u;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t a = 0xffffffffu, o = 0u;
+        for (int i = 0; i < SEL_WARPS; ++i) {
+            a &= red_and[i];
+            o |= red_or[i];
+        }
+        andor[0] = a;
+        andor[1] = o;
+    }
+    cluster.sync();
+    uint32_t gand = 0xffffffffu, gor = 0u;
+    for (int r = 0; r < SEL_CS; ++r) {
+        const uint32_t* ro = cluster.map_shared_rank(andor, r);
+        gand &= ro[0];
+        gor |= ro[1];
+    }
+    const uint32_t diff = gand ^ gor;  // bits where some keys differ (gand > gor only if T == 0)
+    const int top = diff ? 31 - __clz(diff) : -1;
 
-    uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)n_hi;
+    uint32_t prefix, mask, remaining = (uint32_t)n_hi;
     if (n_hi > 0) {
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            if (tid < 256) hist[tid] = 0u;
-            __syncthreads();
+        mask = top >= 31 ? 0u : (0xffffffffu << (top + 1));
+        prefix = gand & mask;  // the shared leading bits
+        int pass = 0;
+        for (int hi = top; hi >= 0; hi -= 8, ++pass) {
+            const int lo = hi >= 7 ? hi - 7 : 0;
+            const uint32_t dmask = (2u << (hi - lo)) - 1u;
+            uint32_t* hcur = hist[pass & 1];
 #pragma unroll
             for (int j = 0; j < KPT; ++j) {
-                // scores share few leading bytes: lanes with the same bin add once (warp-aggregated)
                 const int t = tok0 + j * SEL_THREADS + tid;
-                const bool in = t < 32 * w1 && t < T && (key[j] & mask) == prefix;
-                const uint32_t bin = in ? (key[j] >> shift) & 255u : 256u;
-                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+                if (t < 32 * w1 && t < T && (key[j] & mask) == prefix) atomicAdd(&hcur[(key[j] >> lo) & dmask], 1u);
             }
-            cluster.sync();  // every CTA's histogram of this pass is complete
+            cluster.sync();  // this pass's histograms are complete everywhere, and last pass's reads are done
+            if (tid < 256) hist[(pass + 1) & 1][tid] = 0u;  // free now: nobody reads it any more
             if (wid == 0) {
                 uint32_t cnt[8], sum = 0u;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) cnt[j] = 0u;
                 for (int r = 0; r < SEL_CS; ++r) {
-                    const uint32_t* rh = cluster.map_shared_rank(hist, r);
+                    const uint32_t* rh = cluster.map_shared_rank(hcur, r);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) cnt[j] += rh[255 - 8 * lane - j];
                 }
@@ -242,7 +286,7 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         if (cum + cnt[j] >= remaining) {
-                            sh_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+                            sh_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << lo);
                             sh_remaining = remaining - cum;
                             break;
                         }
@@ -250,10 +294,10 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
                     }
                 }
             }
-            cluster.sync();  // all remote reads of this pass are done before the histograms are reset
+            __syncthreads();
             prefix = sh_prefix;
             remaining = sh_remaining;
-            mask |= 255u << shift;
+            mask |= dmask << lo;
         }
     } else {
         prefix = 0xffffffffu;
@@ -454,25 +498,14 @@ __global__ void __launch_bounds__(SELR_THREADS)
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st)
 {
-    const int kpt_reg = (T + SELR_THREADS - 1) / SELR_THREADS;
-#define SEMKV_SELR(K)                                                                                           \
-    if (kpt_reg <= K) {                                                                                         \
-        k_select_reg<K><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out,     \
-                                                        n_lo_out, tau, status);                                 \
-        return;                                                                                                 \
-    }
-    SEMKV_SELR(1) SEMKV_SELR(2) SEMKV_SELR(4) SEMKV_SELR(8) SEMKV_SELR(16)
-#undef SEMKV_SELR
-    if (T <= 48 * 1024) {  // keys cached in shared memory by one CTA
-        const size_t sm = (size_t)T * 4;
-        cudaFuncSetAttribute(k_select<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        k_select<true><<<units, 1024, sm, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
-                                                status);
+    if (T <= SELR_THREADS) {  // one key per thread: a single CTA
+        k_select_reg<1><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out,
+                                                        n_lo_out, tau, status);
         return;
     }
     const int nwords = (T + 31) / 32;
     const int wpc = (nwords + SEL_CS - 1) / SEL_CS;
-    const int kpt = (wpc * 32 + SEL_THREADS - 1) / SEL_THREADS;  // keys per thread
+    const int kpt = (wpc * 32 + SEL_THREADS - 1) / SEL_THREADS;  // keys per thread in the cluster kernel
     const dim3 grid((unsigned)(units * SEL_CS));
 #define SEMKV_SEL(K)                                                                                           \
     if (kpt <= K) {                                                                                            \
@@ -482,7 +515,7 @@ void launch_select(const float* scores, int units, int T, int n_hi, int words_ca
     }
     SEMKV_SEL(1) SEMKV_SEL(2) SEMKV_SEL(4) SEMKV_SEL(8) SEMKV_SEL(16) SEMKV_SEL(32)
 #undef SEMKV_SEL
-    // more than 32 keys per thread: the one-CTA-per-unit kernel streams the scores from L2
+    // more keys than a cluster holds in registers: one CTA per unit streams the scores from L2
     k_select<false><<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
                                             status);
 }
