@@ -11,7 +11,7 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libsemkv.so")
+LIB_PATH = os.environ.get("SEMKV_LIB") or os.path.join(_PKG, "libsemkv.so")  # SEMKV_LIB: another build
 
 SEMKV_OK = 0
 SEMKV_ERR_INVALID_ARG = 1

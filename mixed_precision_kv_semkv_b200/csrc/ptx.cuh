@@ -53,11 +53,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase, uint32_
     return ok != 0;
 }
 
-// Wait for the barrier's phase parity; false after `limit` tests (each sleeps at most ~hint_ns, so
+// Wait for the barrier's phase parity; false after 2^16 tests (each sleeps at most ~20 us, so
 // the wait is bounded by about a second).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit = 1u << 16)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase)
 {
-    for (uint32_t i = 0; i < limit; ++i)
+    for (uint32_t i = 0; i < (1u << 16); ++i)
         if (mbar_test(bar, phase, 20000u)) return true;
     return false;
 }

@@ -5,9 +5,8 @@
 // (max - min)/(L - 1) (saturated at 65504), z = min, code = clamp(rint((x - z)/s), 0, L - 1),
 // with IEEE fp32 subtract and divide and ties to even.
 //
-// One launch covers both segments.  The compile-time path (k_quantize_pipe, below) is a persistent
-// producer/consumer kernel over (tile, K-or-V) items; the generic kernel uses one CTA per 128-slot
-// output tile:
+// One launch covers both segments; one CTA (4 warps) per 128-slot output tile (the compile-time
+// path uses two CTAs per tile, one for its K rows and one for its V rows):
 //   1. warp 0 maps the tile's slots to token indices (32-ary search of the rank directory for the
 //      first bitmap word, then a ballot scan), and fetches each token's K and V row (256 B each)
 //      with one cp.async.bulk per row into shared memory, completing on an mbarrier; the other
@@ -484,123 +483,50 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
     }
 }
 
-// Persistent pipelined version: each CTA walks a strided list of (unit, segment, tile, K-or-V)
-// items.  Warp 4 is the producer: for the next item it maps the tile's slots to tokens, zeroes
-// the rows of slots past the segment's end and fetches the others with one cp.async.bulk per
-// row into one of two stages; warps 0-3 quantize the item in the other stage meanwhile.  Stage
-// hand-over uses a "full" mbarrier (copies landed) and an "empty" mbarrier (rows consumed).
-constexpr uint32_t PIPE_ROWS_BYTES = TILE * QROW * 2;
-constexpr uint32_t PIPE_STAGE_BYTES = PIPE_ROWS_BYTES + TILE * 4;  // rows + slot->token map
-
 template <int LH, int LL, int G>
-__global__ void __launch_bounds__(160) k_quantize_pipe(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
+__global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
                                                         const uint16_t* __restrict__ V,
                                                         const uint32_t* __restrict__ bitmap,
                                                         const uint32_t* __restrict__ rank, int T, int words_cap,
-                                                        int units, int32_t* __restrict__ status)
+                                                        int32_t* __restrict__ status)
 {
     constexpr int D = 128, NG = D / G;
     const int per_unit = hi.tiles_cap + lo.tiles_cap;
-    const int total = 2 * units * per_unit;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int part = blockIdx.x & 1;  // 0: K rows, 1: V rows of the tile
+    const int u = (blockIdx.x >> 1) / per_unit;
+    int tile = (blockIdx.x >> 1) % per_unit;
+    const bool is_hi = tile < hi.tiles_cap;
+    const QuantSeg& seg = is_hi ? hi : lo;
+    if (!is_hi) tile -= hi.tiles_cap;
+    const int tid = threadIdx.x;
+    const int n = seg.n[u];
+    const int s0 = tile * TILE;
+    if (s0 >= n) return;
+
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t full[2], empty[2];
-    if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(&empty[0], 1);
-        mbar_init(&empty[1], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
+    uint16_t* Xs = reinterpret_cast<uint16_t*>(smem);  // this CTA's rows: K rows or V rows
+    int* tok = reinterpret_cast<int*>(Xs + TILE * QROW);
+    __shared__ __align__(8) uint64_t bar;
+    if (!gather_rows(Xs, nullptr, tok, &bar, is_hi, u, s0, min(TILE, n - s0), part ? V : K, nullptr, bitmap, rank, T,
+                     words_cap, status))
+        return;
 
-    struct Item {
-        int u, tile, part, s0, nv;
-        bool is_hi;
-    };
-    auto decode_item = [&](int idx, Item& it) -> bool {
-        it.part = idx & 1;
-        const int r = idx >> 1;
-        it.u = r / per_unit;
-        const int tl = r % per_unit;
-        it.is_hi = tl < hi.tiles_cap;
-        it.tile = it.is_hi ? tl : tl - hi.tiles_cap;
-        const int n = (it.is_hi ? hi : lo).n[it.u];
-        it.s0 = it.tile * TILE;
-        if (it.s0 >= n) return false;  // a tile past the segment's end: nothing to do (both roles skip it)
-        it.nv = min(TILE, n - it.s0);
-        return true;
-    };
-    bool timeout = false;
-
-    if (warp == 4) {  // ---------------- producer
-        int it = 0;
-        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            Item itm;
-            if (!decode_item(idx, itm)) continue;
-            const int stg = it & 1;
-            const uint32_t use = (uint32_t)it >> 1;
-            uint16_t* rows = reinterpret_cast<uint16_t*>(smem + stg * PIPE_STAGE_BYTES);
-            int* tok = reinterpret_cast<int*>(smem + stg * PIPE_STAGE_BYTES + PIPE_ROWS_BYTES);
-            if (it >= 2 && !mbar_wait(&empty[stg], (use - 1u) & 1u)) timeout = true;
-            for (int r = lane; r < TILE; r += 32) tok[r] = -1;
-            __syncwarp();
-            map_slots_warp(tok, itm.is_hi, itm.s0, itm.nv, bitmap + (size_t)itm.u * words_cap,
-                           rank + (size_t)itm.u * words_cap, T);
-            int valid_rows = 0;
-            for (int r = lane; r < TILE; r += 32) {
-                const int t = r < itm.nv ? tok[r] : -1;
-                if (t >= 0 && t < T) {
-                    ++valid_rows;
-                } else {
-#pragma unroll
-                    for (int i = 0; i < D; i += 8) *reinterpret_cast<uint4*>(rows + r * QROW + i) = make_uint4(0, 0, 0, 0);
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) valid_rows += __shfl_xor_sync(0xffffffffu, valid_rows, o);
-            __syncwarp();  // zeroed rows are ordered before the arrive below (release)
-            if (lane == 0) mbar_arrive_expect_tx(&full[stg], (uint32_t)valid_rows * D * 2u);
-            __syncwarp();
-            const uint16_t* src = itm.part ? V : K;
-            for (int r = lane; r < itm.nv; r += 32) {
-                const int t = tok[r];
-                if (t >= 0 && t < T) bulk_g2s(rows + r * QROW, src + ((size_t)itm.u * T + t) * D, D * 2, &full[stg]);
-            }
-            ++it;
-        }
-    } else {  // ---------------- consumers: thread tid owns row tid (K) or channel tid (V)
-        int it = 0;
-        for (int idx = blockIdx.x; idx < total; idx += gridDim.x) {
-            Item itm;
-            if (!decode_item(idx, itm)) continue;
-            const int stg = it & 1;
-            const uint32_t use = (uint32_t)it >> 1;
-            uint16_t* rows = reinterpret_cast<uint16_t*>(smem + stg * PIPE_STAGE_BYTES);
-            if (!mbar_wait(&full[stg], use & 1u)) timeout = true;
-            const QuantSeg& seg = itm.is_hi ? hi : lo;
-            const size_t tile_base = (size_t)itm.u * seg.tiles_cap + itm.tile;
-            const int Wd = itm.is_hi ? ceil_div(D, radix_k(LH)) : ceil_div(D, radix_k(LL));
-            bool bad = false;
-            if (itm.part == 0) {
-                uint32_t* kw = seg.k + tile_base * Wd * TILE;
-                uint32_t* kz = seg.kz + tile_base * NG * TILE;
-                if (itm.is_hi) quantize_k_rows<LH, G>(rows, kw, kz, tid, bad);
-                else quantize_k_rows<LL, G>(rows, kw, kz, tid, bad);
-            } else {
-                uint32_t* vw = seg.v + tile_base * Wd * D;
-                uint32_t* vz = seg.vz + tile_base * NG * TILE;
-                if (itm.is_hi) quantize_v_rows<LH, G>(rows, vw, vz, tid, bad);
-                else quantize_v_rows<LL, G>(rows, vw, vz, tid, bad);
-            }
-            if (bad && tid < itm.nv) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
-            fence_async_smem();  // the V path wrote codes into the stage: order before its refill
-            named_sync(1, 128);
-            if (tid == 0) mbar_arrive(&empty[stg]);
-            ++it;
-        }
+    const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
+    const int W_hi = ceil_div(D, radix_k(LH)), W_lo = ceil_div(D, radix_k(LL));
+    const int Wd = is_hi ? W_hi : W_lo;
+    bool bad = false;
+    if (part == 0) {
+        uint32_t* kw = seg.k + tile_base * Wd * TILE;
+        uint32_t* kz = seg.kz + tile_base * NG * TILE;
+        if (is_hi) quantize_k_rows<LH, G>(Xs, kw, kz, tid, bad);
+        else quantize_k_rows<LL, G>(Xs, kw, kz, tid, bad);
+    } else {
+        uint32_t* vw = seg.v + tile_base * Wd * D;
+        uint32_t* vz = seg.vz + tile_base * NG * TILE;
+        if (is_hi) quantize_v_rows<LH, G>(Xs, vw, vz, tid, bad);
+        else quantize_v_rows<LL, G>(Xs, vw, vz, tid, bad);
     }
-    if (timeout) atomicOr(status, SEMKV_STATUS_TIMEOUT);
+    if (bad && tid < n - s0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
 }
 
 static size_t quantize_smem(int G)
@@ -629,17 +555,13 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
         return q;
     };
     const unsigned grid = (unsigned)units * per_unit;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        cudaGetLastError();
     const QuantSeg qh = conv(shi), ql = conv(slo);
     // compile-time level pairs and group sizes of the common configurations
 #define SEMKV_QF(LH, LL, GG)                                                                                  \
     if (shi.L == LH && slo.L == LL && G == GG) {                                                              \
-        const size_t sm = 2 * (size_t)PIPE_STAGE_BYTES;                                                       \
-        cudaFuncSetAttribute(k_quantize_pipe<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        const unsigned nct = 2 * grid < 3u * (unsigned)sms ? 2 * grid : 3u * (unsigned)sms;                     \
-        k_quantize_pipe<LH, LL, GG><<<nct, 160, sm, st>>>(qh, ql, K, V, bitmap, rank, T, words_cap, units, status); \
+        const size_t sm = (size_t)TILE * QROW * 2 + TILE * 4;                                                 \
+        cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+        k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, words_cap, status); \
         return;                                                                                               \
     }
 #define SEMKV_QF_G(LH, LL) SEMKV_QF(LH, LL, 32) SEMKV_QF(LH, LL, 64) SEMKV_QF(LH, LL, 128)

@@ -195,7 +195,7 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     const int w0 = min(nwords, c * wpc), w1 = min(nwords, w0 + wpc);
     const int tok0 = 32 * w0;
 
-    __shared__ uint32_t hist[2][256];
+    __shared__ uint32_t hist[2][256], merged[256];
     __shared__ uint32_t gtm[KPT * SEL_WARPS], eqm[KPT * SEL_WARPS];
     __shared__ uint32_t scan_tmp[33];
     __shared__ uint32_t andor[2];   // this CTA's AND and OR of its keys
@@ -267,16 +267,18 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
                 if (t < 32 * w1 && t < T && (key[j] & mask) == prefix) atomicAdd(&hcur[(key[j] >> lo) & dmask], 1u);
             }
             cluster.sync();  // this pass's histograms are complete everywhere, and last pass's reads are done
-            if (tid < 256) hist[(pass + 1) & 1][tid] = 0u;  // free now: nobody reads it any more
+            if (tid < 256) {
+                hist[(pass + 1) & 1][tid] = 0u;  // free now: nobody reads it any more
+                uint32_t v = 0u;                 // bin tid summed over the cluster (independent remote loads)
+#pragma unroll
+                for (int r = 0; r < SEL_CS; ++r) v += cluster.map_shared_rank(hcur, r)[tid];
+                merged[tid] = v;
+            }
+            __syncthreads();
             if (wid == 0) {
                 uint32_t cnt[8], sum = 0u;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) cnt[j] = 0u;
-                for (int r = 0; r < SEL_CS; ++r) {
-                    const uint32_t* rh = cluster.map_shared_rank(hcur, r);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) cnt[j] += rh[255 - 8 * lane - j];
-                }
+                for (int j = 0; j < 8; ++j) cnt[j] = merged[255 - 8 * lane - j];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) sum += cnt[j];
                 const uint32_t inc = warp_incl_scan(sum);
