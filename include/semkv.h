@@ -142,8 +142,9 @@ SEMKV_API int semkv_append_token(const semkv_cache_t* cache, const uint16_t* k, 
  * [B][Hq][D].  Query head qh attends with kv head qh / (Hq/H) over all n_hi + n_lo tokens of its
  * unit (no mask): out = sum_t softmax_t(softmax_scale * q.k^_t) v^_t with k^, v^ the dequantized
  * codes (dequantized in registers; the packed words are read once from HBM).  Split-K over token
- * tiles, then a log-sum-exp merge.  workspace: device buffer of at least
- * semkv_workspace_bytes() bytes (partial softmax states), contents need not be initialized.
+ * tiles, then a log-sum-exp merge.  q must be 16-byte aligned (its rows are read 16 bytes at a
+ * time).  workspace: device buffer of at least semkv_workspace_bytes() bytes (partial softmax
+ * states), contents need not be initialized.
  * A unit with no tokens gives zeros. */
 SEMKV_API int semkv_decode_attention(const semkv_cache_t* cache, const uint16_t* q, float softmax_scale, float* out,
                            void* workspace, size_t workspace_bytes, void* stream);

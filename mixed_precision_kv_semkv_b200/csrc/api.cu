@@ -181,6 +181,7 @@ int semkv_decode_attention(const semkv_cache_t* c, const uint16_t* q, float soft
     int r = validate(c);
     if (r != SEMKV_OK) return r;
     if (!q || !out || !std::isfinite(softmax_scale)) return SEMKV_ERR_INVALID_ARG;
+    if (((uintptr_t)q) & 15u) return SEMKV_ERR_INVALID_ARG;  // query rows are read 16 bytes at a time
     size_t need = 0;
     semkv_workspace_bytes(c, &need);
     if (workspace_bytes < need || (need > 0 && !workspace)) return SEMKV_ERR_INVALID_ARG;

@@ -138,18 +138,25 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         if (t0 < t1) issue_fetch(t0, 0);
         if (t0 + 1 < t1) issue_fetch(t0 + 1, 1);
     }
+    // the GQ query rows: loads issued first, their latency hidden behind the table build; staged in
+    // the B_P area (zeroed once B_Q is built)
+    uint16_t* qs = reinterpret_cast<uint16_t*>(bp);
+    constexpr int QV = GQ * D / 8;  // 16-byte pieces of the query rows
+    uint4 qv[(QV + 127) / 128];
+    {
+        const uint4* qu = reinterpret_cast<const uint4*>(q + ((size_t)b * Hq + (size_t)hk * GQ) * D);
+#pragma unroll
+        for (int e = 0; e < (QV + 127) / 128; ++e)
+            if (tid + 128 * e < QV) qv[e] = __ldg(qu + tid + 128 * e);
+    }
     for (int i = tid; i < L * L * 32; i += 128) {
         const int P = i >> 5;
         const __half2 pr = __floats2half2_rn((float)(P / L) - MID, (float)(P % L) - MID);  // exact: |x| <= 7.5
         lut[i] = *reinterpret_cast<const uint32_t*>(&pr);
     }
-    // the GQ query rows staged in the B_P area (zeroed once B_Q is built)
-    uint16_t* qs = reinterpret_cast<uint16_t*>(bp);
-    {
-        const uint16_t* qu = q + ((size_t)b * Hq + (size_t)hk * GQ) * D;
-        for (int i = tid; i < GQ * D / 8; i += 128)
-            reinterpret_cast<uint4*>(qs)[i] = __ldg(reinterpret_cast<const uint4*>(qu) + i);
-    }
+#pragma unroll
+    for (int e = 0; e < (QV + 127) / 128; ++e)
+        if (tid + 128 * e < QV) reinterpret_cast<uint4*>(qs)[tid + 128 * e] = qv[e];
     __syncthreads();
     for (int ks = tid; ks < KSLOTS; ks += 128) {
         const int col = ks >> 1, h2 = ks & 1, j = col / NPAIR, pp = col % NPAIR;
@@ -162,11 +169,23 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
             *reinterpret_cast<uint16_t*>(bq + core_off(nrow, ks, C::LBO_Q, C::SBO_Q)) = v;
         }
     }
-    if (tid < NG * GQ) {
-        const int grp = tid / GQ, h = tid % GQ;
-        float s = 0.f;
-        for (int d = grp * G; d < (grp + 1) * G; ++d) s += h2f(qs[h * D + d]);
-        qsum[tid] = s;
+    {
+        // per-group query sums: 8 threads per (group, head), G/8 channels each
+        const int si = tid >> 3, part = tid & 7;
+        float a = 0.f;
+        if (si < NG * GQ) {
+            const int grp = si / GQ, h = si % GQ;
+            const __half2* qp = reinterpret_cast<const __half2*>(qs + h * D + grp * G + part * (G / 8));
+#pragma unroll
+            for (int e = 0; e < G / 16; ++e) {
+                const float2 f2 = __half22float2(qp[e]);
+                a += f2.x + f2.y;
+            }
+        }
+        a += __shfl_xor_sync(0xffffffffu, a, 4);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        if (si < NG * GQ && part == 0) qsum[si] = a;
     }
     __syncthreads();
     for (int i = tid; i < (int)((NV / 8) * C::SBO_P / 16); i += 128) reinterpret_cast<uint4*>(bp)[i] = make_uint4(0, 0, 0, 0);
@@ -196,20 +215,23 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     uint32_t ph_k = 0, ph_v = 0;
     bool timeout = false;
 
-    const uint32_t* lut_lane = lut + lane;  // this lane's copy: entry P at lut_lane[32 * P]
-    // W words (from shared memory) -> KCP TMEM columns of this thread's lane
-    auto unpack_to_tmem = [&](const uint32_t* words) {
+    const uint32_t lut_lane = smem_u32(lut + lane);  // this lane's copy: entry P at + 128 P bytes
+    // W words (shared address `words` + 4 tid, stride 512 B) -> KCP TMEM columns of this thread's lane
+    auto unpack_to_tmem = [&](uint32_t words) {
+        uint32_t wv[W];
+#pragma unroll
+        for (int j = 0; j < W; ++j) wv[j] = lds_u32_after_wait(words + (uint32_t)(j * 512 + 4 * tid));
         uint32_t chunk[8];
         int ci = 0;
         uint32_t cbase = C::COL_A;
 #pragma unroll
         for (int j = 0; j < W; ++j) {
-            uint32_t f = to_fraction<L>(words[j * 128 + tid]);
+            uint32_t f = to_fraction<L>(wv[j]);
 #pragma unroll
             for (int pp = 0; pp < NPAIR; ++pp) {
                 const unsigned long long t = (unsigned long long)f * (unsigned long long)(L * L);
                 f = (uint32_t)t;
-                chunk[ci++] = lut_lane[(uint32_t)(t >> 32) << 5];
+                chunk[ci++] = lds_u32(lut_lane + ((uint32_t)(t >> 32) << 7));
                 if (ci == 8) {
                     tmem_st8(lane_base + cbase, chunk);
                     cbase += 8;
@@ -230,7 +252,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         if (!mbar_wait(&mbar[2 + stg], (uint32_t)(it >> 1) & 1u)) timeout = true;
 
         // ---- K codes -> TMEM, q.k
-        unpack_to_tmem(reinterpret_cast<const uint32_t*>(sb + C::STAGE_K));
+        unpack_to_tmem(smem_u32(sb + C::STAGE_K));
         tc_wait_st();
         tc_fence_before();
         __syncthreads();
@@ -300,7 +322,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
             }
         }
         // ---- V codes -> TMEM (same columns: the q.k product has completed), p.V
-        unpack_to_tmem(reinterpret_cast<const uint32_t*>(sb + C::STAGE_V));
+        unpack_to_tmem(smem_u32(sb + C::STAGE_V));
         tc_wait_st();
         fence_async_smem();
         tc_fence_before();

@@ -62,6 +62,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase)
     return false;
 }
 
+// 32-bit loads from a shared-memory address (as returned by smem_u32).  lds_u32_after_wait is
+// ordered after earlier volatile asm (an mbarrier wait that made the data visible); lds_u32 may be
+// scheduled freely and is for data written before the CTA's set-up barrier (tables).
+__device__ __forceinline__ uint32_t lds_u32_after_wait(uint32_t saddr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr)
+{
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
+
 // ------------------------------------------------------------------ bulk async copy (no multicast)
 
 // global -> shared, `bytes` a multiple of 16, both addresses 16-byte aligned; completes on `bar`.

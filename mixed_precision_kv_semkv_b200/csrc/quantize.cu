@@ -169,11 +169,17 @@ __device__ __forceinline__ bool gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok
             }
         }
     }
-    const bool arrived = mbar_wait(bar, 0);
+    // one thread waits for the copies (the others sleep in the barrier instead of polling); the
+    // barrier then orders the landed rows before every thread's reads
+    __shared__ int arrived_s;
+    if (tid == 0) arrived_s = mbar_wait(bar, 0) ? 1 : 0;
     __syncthreads();
-    if (!arrived) {  // copies did not land in time: report, wait once more for them, and stop
-        if (tid == 0) atomicOr(status, SEMKV_STATUS_TIMEOUT);
-        mbar_wait(bar, 0);
+    if (!arrived_s) {  // copies did not land in time: report, wait once more for them, and stop
+        if (tid == 0) {
+            atomicOr(status, SEMKV_STATUS_TIMEOUT);
+            mbar_wait(bar, 0);
+        }
+        __syncthreads();
         return false;
     }
     return true;
