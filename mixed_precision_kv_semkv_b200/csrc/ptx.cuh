@@ -78,6 +78,20 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t saddr)
     return v;
 }
 
+// ------------------------------------------------------------------ 16-byte async copies (cp.async)
+
+// 16 bytes global -> shared without a register round trip (L2 only: .cg); both addresses 16-byte aligned
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+
+// wait until every cp.async this thread issued has landed
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ bulk async copy (no multicast)
 
 // global -> shared, `bytes` a multiple of 16, both addresses 16-byte aligned; completes on `bar`.

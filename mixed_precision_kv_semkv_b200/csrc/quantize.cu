@@ -8,9 +8,9 @@
 // One launch covers both segments; one CTA (4 warps) per 128-slot output tile (the compile-time
 // path uses two CTAs per tile, one for its K rows and one for its V rows):
 //   1. warp 0 maps the tile's slots to token indices (32-ary search of the rank directory for the
-//      first bitmap word, then a ballot scan), and fetches each token's K and V row (256 B each)
-//      with one cp.async.bulk per row into shared memory, completing on an mbarrier; the other
-//      warps zero the rows of slots past the segment's end meanwhile;
+//      first bitmap word, then a ballot scan); all threads then copy each token's K and V row
+//      (256 B each) into shared memory in 16-byte cp.async pieces (rows of slots past the
+//      segment's end are zeroed);
 //   2. thread t quantizes K row t and packs it along the channels;
 //   3. thread t writes the scale/zero of V row t; after a barrier thread d packs channel d of
 //      every slot along the tile's slots.
@@ -119,70 +119,37 @@ __device__ __forceinline__ void map_slots_warp(int* tok, bool is_hi, int s0, int
 
 // Slots [s0, s0 + nv) of a segment of unit u -> token indices (tok), and each token's K row and V
 // row (256 B each; V/Vs may be null) into shared memory: warp 0 searches the rank directory
-// (32-ary) for the first bitmap word, scans the following words with ballots, and issues one
-// cp.async.bulk per row on `bar`; rows of slots past nv are zeroed.  Returns false (status set)
-// if the copies timed out.
-__device__ __forceinline__ bool gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok, uint64_t* bar, bool is_hi, int u,
-                                            int s0, int nv, const uint16_t* __restrict__ K,
-                                            const uint16_t* __restrict__ V, const uint32_t* __restrict__ bitmap,
-                                            const uint32_t* __restrict__ rank, int T, int words_cap,
-                                            int32_t* __restrict__ status)
+// (32-ary) for the first bitmap word and scans the following words with ballots; then all 128
+// threads move the rows in 16-byte cp.async pieces (16 consecutive threads per row, so every
+// warp reads two whole rows per instruction); rows of slots past nv are zeroed.
+__device__ __forceinline__ void gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok, bool is_hi, int u, int s0, int nv,
+                                            const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
+                                            const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ rank,
+                                            int T, int words_cap)
 {
     constexpr int D = 128;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-    }
+    const int tid = threadIdx.x, warp = tid >> 5;
     tok[tid] = -1;
     __syncthreads();
-
-    if (warp == 0) {
+    if (warp == 0)
         map_slots_warp(tok, is_hi, s0, nv, bitmap + (size_t)u * words_cap, rank + (size_t)u * words_cap, T);
-        __syncwarp();
-        // ---- row fetch: one bulk copy per row; rows of unmapped slots are zeroed instead
-        int valid_rows = 0;
-        for (int r = lane; r < nv; r += 32) valid_rows += (tok[r] >= 0 && tok[r] < T);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) valid_rows += __shfl_xor_sync(0xffffffffu, valid_rows, o);
-        const uint32_t mats = V ? 2u : 1u;
-        if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)valid_rows * mats * D * 2u);
-        __syncwarp();
-        for (int r = lane; r < nv; r += 32) {
-            const int t = tok[r];
-            if (t >= 0 && t < T) {
-                const size_t off = ((size_t)u * T + t) * D;
-                bulk_g2s(Ks + r * QROW, K + off, D * 2, bar);
-                if (V) bulk_g2s(Vs + r * QROW, V + off, D * 2, bar);
-            } else {
-                for (int i = 0; i < D; i += 8) {
-                    *reinterpret_cast<uint4*>(Ks + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
-                    if (V) *reinterpret_cast<uint4*>(Vs + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-        }
-    } else {
-        for (int r = nv + (tid - 32); r < TILE; r += 96) {
-            for (int i = 0; i < D; i += 8) {
-                *reinterpret_cast<uint4*>(Ks + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
-                if (V) *reinterpret_cast<uint4*>(Vs + r * QROW + i) = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-    }
-    // one thread waits for the copies (the others sleep in the barrier instead of polling); the
-    // barrier then orders the landed rows before every thread's reads
-    __shared__ int arrived_s;
-    if (tid == 0) arrived_s = mbar_wait(bar, 0) ? 1 : 0;
     __syncthreads();
-    if (!arrived_s) {  // copies did not land in time: report, wait once more for them, and stop
-        if (tid == 0) {
-            atomicOr(status, SEMKV_STATUS_TIMEOUT);
-            mbar_wait(bar, 0);
+    for (int c = tid; c < TILE * (D / 8); c += 128) {
+        const int r = c >> 4, part = (c & 15) * 8;
+        const int t = r < nv ? tok[r] : -1;
+        uint16_t* dk = Ks + r * QROW + part;
+        uint16_t* dv = Vs ? Vs + r * QROW + part : nullptr;
+        if (t >= 0 && t < T) {
+            const size_t off = ((size_t)u * T + t) * D + part;
+            cp_async16(dk, K + off);
+            if (dv) cp_async16(dv, V + off);
+        } else {
+            *reinterpret_cast<uint4*>(dk) = make_uint4(0u, 0u, 0u, 0u);
+            if (dv) *reinterpret_cast<uint4*>(dv) = make_uint4(0u, 0u, 0u, 0u);
         }
-        __syncthreads();
-        return false;
     }
-    return true;
+    cp_async_wait_all();
+    __syncthreads();
 }
 
 __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
@@ -212,9 +179,7 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     uint16_t* Vs = Ks + TILE * QROW;
     int* tok = reinterpret_cast<int*>(Vs + TILE * QROW);
     float4* vgrid = reinterpret_cast<float4*>(tok + TILE);  // [TILE][NG] (s, r, z, -)
-    __shared__ __align__(8) uint64_t bar;
-
-    if (!gather_rows(Ks, Vs, tok, &bar, is_hi, u, s0, nv, K, V, bitmap, rank, T, words_cap, status)) return;
+    gather_rows(Ks, Vs, tok, is_hi, u, s0, nv, K, V, bitmap, rank, T, words_cap);
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     uint32_t* kw = seg.k + tile_base * WK * TILE;
@@ -512,10 +477,8 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
     extern __shared__ __align__(128) unsigned char smem[];
     uint16_t* Xs = reinterpret_cast<uint16_t*>(smem);  // this CTA's rows: K rows or V rows
     int* tok = reinterpret_cast<int*>(Xs + TILE * QROW);
-    __shared__ __align__(8) uint64_t bar;
-    if (!gather_rows(Xs, nullptr, tok, &bar, is_hi, u, s0, min(TILE, n - s0), part ? V : K, nullptr, bitmap, rank, T,
-                     words_cap, status))
-        return;
+    gather_rows(Xs, nullptr, tok, is_hi, u, s0, min(TILE, n - s0), part ? V : K, nullptr, bitmap, rank, T,
+                words_cap);
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     const int W_hi = ceil_div(D, radix_k(LH)), W_lo = ceil_div(D, radix_k(LL));
