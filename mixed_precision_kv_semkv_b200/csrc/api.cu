@@ -64,7 +64,8 @@ int sm_count()
 }
 
 // Split-K factor per segment: one wave of four CTAs per SM over the whole decode, shared between
-// the segments in proportion to their capacity in tiles, at most one split per tile.
+// the segments in proportion to their capacity in tiles (rounded down, so that the two grids
+// together never need a second wave), at least one and at most one split per tile.
 void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
 {
     const int units = c->B * c->H;
@@ -72,7 +73,7 @@ void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
     const long target = 4L * sm_count();
     auto pick = [&](int tiles) -> int {
         if (tiles == 0) return 0;
-        long s = (target * tiles + (long)units * total - 1) / ((long)units * total);
+        long s = (target * tiles) / ((long)units * total);
         if (s < 1) s = 1;
         if (s > tiles) s = tiles;
         return (int)s;
