@@ -214,32 +214,39 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
 // Log-sum-exp merge of the split partials of one (unit, query head): all splits' maxima are read
 // in parallel, the weights 2^(m_s - M) go to shared memory, then four slices of 128 threads each
 // sum a quarter of the splits of o_s[d] with independent loads, and the slices are added.
-constexpr int MERGE_SLICES = 4;
+// Merge of the split-K partials: one CTA per (unit, query head, 32-channel slice); its 512 threads
+// first reduce the splits' maxima and denominators, then each of 16 warps sums a 16th of the
+// splits for the slice's 32 channels, so every thread makes only a few independent loads.
+constexpr int MERGE_CH = 32, MERGE_PARTS = 16;
 
-__global__ void __launch_bounds__(128 * MERGE_SLICES) k_decode_merge(const float* __restrict__ ws, int g,
-                                                                      int nsplit_total, float* __restrict__ out)
+__global__ void __launch_bounds__(32 * MERGE_PARTS) k_decode_merge(const float* __restrict__ ws, int g,
+                                                                  int nsplit_total, float* __restrict__ out)
 {
-    constexpr int D = 128, NT = 128 * MERGE_SLICES;
+    constexpr int D = 128, NT = 32 * MERGE_PARTS;
     // launched as a programmatic dependent of the split kernels: wait for them (and their writes)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int u = blockIdx.x / g, h = blockIdx.x % g;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, d = tid & (D - 1), slice = tid / D;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float* base = ws + (size_t)u * nsplit_total * g * (D + 2) + h * (D + 2);
     const size_t stride = (size_t)g * (D + 2);
-    extern __shared__ float wts[];  // [nsplit_total]
-    __shared__ float red[NT / 32], redl[NT / 32], part[MERGE_SLICES][D];
+    extern __shared__ float wts[];  // [nsplit_total]: the splits' maxima, then their weights
+    __shared__ float red[MERGE_PARTS], redl[MERGE_PARTS], part[MERGE_PARTS][MERGE_CH];
     const float NEG = -__int_as_float(0x7f800000);
     float M = NEG;
-    for (int s = tid; s < nsplit_total; s += NT) M = fmaxf(M, base[s * stride + D]);
+    for (int s = tid; s < nsplit_total; s += NT) {
+        const float m = base[s * stride + D];
+        wts[s] = m;
+        M = fmaxf(M, m);
+    }
     M = warp_max(M);
     if (lane == 0) red[warp] = M;
     __syncthreads();
     M = NEG;
 #pragma unroll
-    for (int i = 0; i < NT / 32; ++i) M = fmaxf(M, red[i]);
+    for (int i = 0; i < MERGE_PARTS; ++i) M = fmaxf(M, red[i]);
     float l = 0.f;
     for (int s = tid; s < nsplit_total; s += NT) {
-        const float w = M == NEG ? 0.f : exp2f(base[s * stride + D] - M);
+        const float w = M == NEG ? 0.f : exp2f(wts[s] - M);
         wts[s] = w;
         l += w * base[s * stride + D + 1];
     }
@@ -249,22 +256,17 @@ __global__ void __launch_bounds__(128 * MERGE_SLICES) k_decode_merge(const float
     __syncthreads();
     float Ls = 0.f;
 #pragma unroll
-    for (int i = 0; i < NT / 32; ++i) Ls += redl[i];
-    float O0 = 0.f, O1 = 0.f;
-    int s = slice;
-#pragma unroll 4
-    for (; s + MERGE_SLICES < nsplit_total; s += 2 * MERGE_SLICES) {  // two independent loads per step
-        O0 += wts[s] * base[s * stride + d];
-        O1 += wts[s + MERGE_SLICES] * base[(s + MERGE_SLICES) * stride + d];
-    }
-    for (; s < nsplit_total; s += MERGE_SLICES) O0 += wts[s] * base[s * stride + d];
-    part[slice][d] = O0 + O1;
+    for (int i = 0; i < MERGE_PARTS; ++i) Ls += redl[i];
+    const int d = blockIdx.y * MERGE_CH + lane;
+    float O = 0.f;
+    for (int s = warp; s < nsplit_total; s += MERGE_PARTS) O += wts[s] * base[s * stride + d];
+    part[warp][lane] = O;
     __syncthreads();
-    if (slice == 0) {
-        float O = 0.f;
+    if (warp == 0) {
+        float t = 0.f;
 #pragma unroll
-        for (int i = 0; i < MERGE_SLICES; ++i) O += part[i][d];
-        out[((size_t)u * g + h) * D + d] = Ls > 0.f ? O / Ls : 0.f;
+        for (int i = 0; i < MERGE_PARTS; ++i) t += part[i][lane];
+        out[((size_t)u * g + h) * D + d] = Ls > 0.f ? t / Ls : 0.f;
     }
 }
 
@@ -305,8 +307,8 @@ void launch_decode_merge(const float* ws, int units, int H, int g, int D, int ns
     (void)H;
     (void)D;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * g));
-    cfg.blockDim = dim3(128 * MERGE_SLICES);
+    cfg.gridDim = dim3((unsigned)(units * g), 128 / MERGE_CH);
+    cfg.blockDim = dim3(32 * MERGE_PARTS);
     cfg.dynamicSmemBytes = (size_t)(nsplit_total > 0 ? nsplit_total : 1) * sizeof(float);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
