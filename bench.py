@@ -57,18 +57,28 @@ def radix_words(L: int, n: int = 128) -> int:
     return -(-n // k)
 
 
-def alg_bytes(w, T: int, n_hi: int) -> dict:
-    """Algorithmic bytes of one layer, per hot-path step (measurement)."""
+# this library's kernel launches in one step: select 1, quantize 1, append 1, decode 3 (hi and lo
+# segments, merge); the committed ncu launch list of the step shows the same kernels
+LAUNCHES_PER_STEP = 6
+
+
+def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False) -> dict:
+    """Algorithmic bytes of one layer, per hot-path step (measurement).  With
+    `appended`, one generated token per unit follows the prefill (`new_hi` of them on the L_hi grid)
+    and the decode reads the cache including it."""
     units = w.B * w.H
     ng = w.D // w.G
     rec = lambda L: 2 * (4 * radix_words(L, w.D) + 4 * ng)  # noqa: E731  K + V record of one token
     cache = units * (n_hi * rec(w.L_hi) + (T - n_hi) * rec(w.L_lo))
     bitmap_rank = units * 2 * 4 * ((T + 31) // 32)
     q = w.B * w.Hq * w.D * 2
+    new = new_hi * rec(w.L_hi) + (units - new_hi) * rec(w.L_lo) if appended else 0
     return {
         "select": units * 4 * T + bitmap_rank,
         "quantize": units * T * w.D * 2 * 2 + bitmap_rank + cache,
-        "decode": cache + q,
+        # the new token's k, v rows and score read, its record written
+        "append": units * (w.D * 2 * 2 + 4) + new if appended else 0,
+        "decode": cache + new + q,
         "cache": cache,
     }
 
@@ -160,30 +170,37 @@ def oracle_sample(w, seconds_target: float = 15.0, max_units: int = 8):
     from mixed_precision_kv_semkv_b200 import synth
 
     if w.name not in _SAMPLE_INPUTS:
-        _SAMPLE_INPUTS[w.name] = synth.layer_cpu(w, 0, B=1)
+        d0 = synth.layer_cpu(w, 0, B=1)
+        gen = synth.gen_steps_cpu(w, d0["K"], 0, 0, 1)
+        d0.update(kn=gen["k"][0], vn=gen["v"][0], sn=gen["scores"][0])
+        _SAMPLE_INPUTS[w.name] = d0
     d = _SAMPLE_INPUTS[w.name]
     g = w.Hq // w.H
     T = w.T
     n_hi = oracle.n_hi(w.p, T)
-    tiles_hi, tiles_lo = max(1, -(-n_hi // 128)), max(1, -(-(T - n_hi) // 128))
-    done, t0 = 0, time.perf_counter()
+    tiles_hi, tiles_lo = -(-(n_hi + 1) // 128), -(-(T - n_hi + 1) // 128)
+    done, new_hi, t0 = 0, 0, time.perf_counter()
     while done < min(max_units, w.H):
         h = done
         bm, rk, nh, tau, _ = oracle.select(d["scores"][0, h], w.p)
         hi, lo, _ = oracle.quantize_pack_unit(d["K"][0, h].view(np.uint16), d["V"][0, h].view(np.uint16), bm, w.G,
                                               w.L_hi, w.L_lo, tiles_hi, tiles_lo)
-        Kh, Vh = oracle.dequantize_unit(T, w.D, w.G, w.L_hi, w.L_lo, bm, hi, lo)
+        st = oracle.UnitState(T + 1, bm, rk, nh, T - nh, tau, hi, lo)
+        oracle.append_unit(st, d["kn"][0, h].view(np.uint16), d["vn"][0, h].view(np.uint16), float(d["sn"][0, h]),
+                           w.G, w.L_hi, w.L_lo)
+        new_hi += st.n_hi - nh
+        Kh, Vh = oracle.dequantize_unit(T + 1, w.D, w.G, w.L_hi, w.L_lo, st.bitmap, hi, lo)
         oracle.attention_fp64(d["q"][0, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, synth.sm_scale())
         done += 1
         if time.perf_counter() - t0 > seconds_target:
             break
     el = time.perf_counter() - t0
-    per_unit = alg_bytes(w, T, n_hi)
     units_layer = w.B * w.H
-    step_bytes = (per_unit["select"] + per_unit["quantize"] + per_unit["decode"]) / units_layer * done
+    per = alg_bytes(w, T, n_hi, new_hi * units_layer // max(done, 1), appended=True)
+    step_bytes = (per["select"] + per["quantize"] + per["append"] + per["decode"]) / units_layer * done
     return {"seconds": el, "units": done, "bytes": step_bytes, "gbs": step_bytes / el / 1e9,
-            "sample": f"{done} unit(s) (one batch row x kv head each, T={T}) of workload {w.name}: select + "
-                      f"quantize/pack + dequantize + fp64 attention, oracle as it stands, 1 thread"}
+            "sample": f"{done} unit(s) (one batch row x kv head each, T={T} + 1 appended) of workload {w.name}: "
+                      f"select + quantize/pack + append + dequantize + fp64 attention, oracle as it stands, 1 thread"}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -224,8 +241,8 @@ def run_reference(args):
 def run_semkv(args):
     import torch
 
-    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_assign_precision, semkv_decode_attention,
-                                               semkv_quantize_pack, synth)
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_append_token, semkv_assign_precision,
+                                               semkv_decode_attention, semkv_quantize_pack, synth)
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
@@ -242,25 +259,39 @@ def run_semkv(args):
     T = w.T
     d = synth.layer_gpu(w, seed=rank_seed(rank))
     K, V, S, q = d["K"], d["V"], d["scores"], d["q"]
-    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p)
+    # one generated token per unit: its k, v rows and score (appended after the prefill every step)
+    gen = synth.gen_steps_gpu(w, K, seed=rank_seed(rank), layer=0, steps=1)
+    kn, vn, sn = (gen[x][0].contiguous() for x in ("k", "v", "scores"))
+    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=1)
     ws = cache.workspace()
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
     scale = synth.sm_scale(w.D)
     from mixed_precision_kv_semkv_b200.cache import n_hi_for
 
-    nb = alg_bytes(w, T, n_hi_for(w.p, T))
-    step_bytes = nb["select"] + nb["quantize"] + nb["decode"]
     stream = torch.cuda.current_stream()
 
     # each C-ABI call is captured once into its own CUDA graph: replaying it costs the host a few
     # microseconds, so the device timings below are not bounded by Python/ctypes enqueue time
     calls = [lambda: semkv_assign_precision(cache, S, T, w.p),
              lambda: semkv_quantize_pack(cache, K, V, T),
+             lambda: semkv_append_token(cache, kn, vn, sn),
              lambda: semkv_decode_attention(cache, q, scale, out, ws)]
+    names = ("select", "quantize", "append", "decode_in_step")
     for c in calls:  # eager once: module loading and kernel attributes happen outside capture
         c()
     torch.cuda.synchronize()
+    # which units' new token went to the L_hi grid (the same every step: same inputs)
+    n_hi0 = n_hi_for(w.p, T)
+    new_hi = int((cache.bufs["n_hi"] - n_hi0).sum().item())
+    nb = alg_bytes(w, T, n_hi0, new_hi, appended=True)
+    step_bytes = nb["select"] + nb["quantize"] + nb["append"] + nb["decode"]
+    # the step as one CUDA graph (as a serving loop would capture it): the timed `value`; and each
+    # call in a graph of its own: the per-call split (each then also pays its own graph launch)
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph, capture_error_mode="relaxed"):
+        for c in calls:
+            c()
     graphs = []
     for c in calls:
         gr = torch.cuda.CUDAGraph()
@@ -269,12 +300,17 @@ def run_semkv(args):
         graphs.append(gr)
 
     def step(ev=None):
-        for i, gr in enumerate(graphs):
-            if ev is not None:
-                ev[i].record(stream)
-            gr.replay()
         if ev is not None:
-            ev[3].record(stream)
+            ev[0].record(stream)
+        step_graph.replay()
+        if ev is not None:
+            ev[1].record(stream)
+
+    def step_split(ev):
+        for i, gr in enumerate(graphs):
+            ev[i].record(stream)
+            gr.replay()
+        ev[len(graphs)].record(stream)
 
     steps = 3 if args.profile else args.steps
     warm = max(args.warmup, 3)
@@ -284,7 +320,7 @@ def run_semkv(args):
     torch.cuda.synchronize()
     assert cache.status() == 0, f"device status {cache.status()}"
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     clocks = Clocks(local)
     if not args.profile:
         clocks.start()
@@ -299,11 +335,17 @@ def run_semkv(args):
     if dist is not None:
         dist.barrier()
     ck = clocks.stop() if not args.profile else {}
-    t_sel = sum(e[0].elapsed_time(e[1]) for e in evs)
-    t_q = sum(e[1].elapsed_time(e[2]) for e in evs)
-    t_dec = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms = max_over_ranks(t_sel + t_q + t_dec, dist, "cuda")
+    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), dist, "cuda")
     value = weak_scaling_value(world, step_bytes, steps, total_ms)
+
+    # per-call split, outside the timed region
+    split_steps = min(steps, 300)
+    evs_split = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(split_steps)]
+    for i in range(split_steps):
+        flush.zero_()
+        step_split(evs_split[i])
+    torch.cuda.synchronize()
+    t_call = [sum(e[i].elapsed_time(e[i + 1]) for e in evs_split) * steps / split_steps for i in range(len(graphs))]
 
     # decode alone over an L2-cold cache (decode-attn HBM GB/s of the metric)
     dec_ms = []
@@ -311,7 +353,7 @@ def run_semkv(args):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        graphs[2].replay()
+        graphs[3].replay()
         e1.record(stream)
         dec_ms.append((e0, e1))
     torch.cuda.synchronize()
@@ -325,14 +367,16 @@ def run_semkv(args):
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     peak_note = "measured" if "hbm_gbs" in peaks else "fallback"
     per_kernel = {
-        "select": {"ms": t_sel / steps, "gbs": nb["select"] / (t_sel / steps * 1e-3) / 1e9},
-        "quantize": {"ms": t_q / steps, "gbs": nb["quantize"] / (t_q / steps * 1e-3) / 1e9},
-        "decode_in_step": {"ms": t_dec / steps, "gbs": nb["decode"] / (t_dec / steps * 1e-3) / 1e9},
-        "decode_l2_cold": {"ms": dec_cold, "gbs": nb["decode"] / (dec_cold * 1e-3) / 1e9},
+        nm: {"ms": t / steps, "gbs": nb[nm.replace("_in_step", "")] / (t / steps * 1e-3) / 1e9}
+        for nm, t in zip(names, t_call)
     }
+    per_kernel.update({
+        "decode_l2_cold": {"ms": dec_cold, "gbs": nb["decode"] / (dec_cold * 1e-3) / 1e9},
+    })
     dom = max(("select", "quantize", "decode_in_step"), key=lambda k: per_kernel[k]["ms"])
-    dom_name = {"select": "semkv_assign_precision (k_select)", "quantize": "semkv_quantize_pack (k_quantize)",
-                "decode_in_step": "semkv_decode_attention (k_decode_split + k_decode_merge)"}[dom]
+    dom_name = {"select": "semkv_assign_precision (k_select_cluster)",
+                "quantize": "semkv_quantize_pack (k_quantize_fast)",
+                "decode_in_step": "semkv_decode_attention (k_decode_tc x 2 + k_decode_merge)"}[dom]
     ach = per_kernel[dom]["gbs"]
     traffic = None  # DRAM bytes per launch from the committed ncu capture, if the kernel is unchanged since
     try:
@@ -349,7 +393,7 @@ def run_semkv(args):
 
     e2e = None
     if not args.no_e2e and not args.profile:
-        hK, hV, hS, hq = (t.cpu().pin_memory() for t in (K, V, S, q))
+        hK, hV, hS, hq, hk, hv, hs = (t.cpu().pin_memory() for t in (K, V, S, q, kn, vn, sn))
         hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
         e2e_steps = min(steps, 20)
         el = 0.0
@@ -361,13 +405,16 @@ def run_semkv(args):
             V.copy_(hV, non_blocking=True)
             S.copy_(hS, non_blocking=True)
             q.copy_(hq, non_blocking=True)
+            kn.copy_(hk, non_blocking=True)
+            vn.copy_(hv, non_blocking=True)
+            sn.copy_(hs, non_blocking=True)
             step()
             hout.copy_(out, non_blocking=True)
             e1.record(stream)
             e1.synchronize()
             if i >= 2:
                 el += e0.elapsed_time(e1)
-        h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hS, hq))
+        h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hS, hq, hk, hv, hs))
         e2e = {"value": world * step_bytes * e2e_steps / (el * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * 4,
                "ms_per_step": el / e2e_steps}
@@ -384,7 +431,10 @@ def run_semkv(args):
         "config": {"workload": f"{w.name}: Llama-3.1-8B-shaped layer, B{w.B} H{w.H} Hq{w.Hq} T{T} D{w.D}, "
                                f"G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}",
                    "l2": "flushed between steps (512 MB write)", "parallelism": f"dp{world} (independent units)",
-                   "step": "assign_precision + quantize_pack + decode_attention"},
+                   "timing": "step = one CUDA graph of the four calls; per_kernel = each call replayed from a graph "
+                             "of its own (so each also pays a graph launch)",
+                   "step": "assign_precision + quantize_pack + append_token (one generated token per unit) + "
+                           "decode_attention"},
         "per_kernel": per_kernel,
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                      "frac": ach / hbm_peak, "peak_kind": peak_note, "traffic": traffic,
@@ -392,7 +442,7 @@ def run_semkv(args):
         "decode_roofline": {"achieved": per_kernel["decode_l2_cold"]["gbs"], "peak": hbm_peak,
                             "frac": per_kernel["decode_l2_cold"]["gbs"] / hbm_peak,
                             "frac_of_8000": per_kernel["decode_l2_cold"]["gbs"] / 8000.0},
-        "clocks": ck, "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 6 * steps,
+        "clocks": ck, "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": LAUNCHES_PER_STEP * steps,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

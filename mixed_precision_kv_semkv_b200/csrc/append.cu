@@ -16,15 +16,18 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
                                                  const uint16_t* __restrict__ vnew, const float* __restrict__ score)
 {
     constexpr int D = 128;
-    const int u = blockIdx.x, d = threadIdx.x;
+    const int u = blockIdx.x, d = threadIdx.x, lane = d & 31, warp = d >> 5;
     const int G = c.G, NG = D / G;
-    __shared__ float kr[D], vr[D];
     __shared__ int kc[D + 32];
-    __shared__ float gs[2][16], gz[2][16];
+    __shared__ float gmn[2][4], gmx[2][4];  // per-warp partial extrema of groups wider than a warp
 
+    // every independent load first: the unit's state and this thread's channel of the new rows
     const float sc = score[u];
-    const bool hi = sc > c.tau[u];  // NaN compares false: the token goes lo
+    const float tau = c.tau[u];
     const int nh = c.n_hi[u], nl = c.n_lo[u];
+    const float kx = h2f(knew[(size_t)u * D + d]);
+    const float vx = h2f(vnew[(size_t)u * D + d]);
+    const bool hi = sc > tau;  // NaN compares false: the token goes lo
     const int T = nh + nl;
     const int slot = hi ? nh : nl;
     const int cap = hi ? c.cap_hi : c.cap_lo;
@@ -42,31 +45,43 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
     uint32_t* vw = (hi ? c.v_hi : c.v_lo) + tb * WV * D;
     uint32_t* kz = (hi ? c.kz_hi : c.kz_lo) + tb * NG * TILE;
     uint32_t* vz = (hi ? c.vz_hi : c.vz_lo) + tb * NG * TILE;
-
-    kr[d] = h2f(knew[(size_t)u * D + d]);
-    vr[d] = h2f(vnew[(size_t)u * D + d]);
     if (d < 32) kc[D + d] = 0;  // padding digits of the last K word
-    __syncthreads();
 
-    bool bad = !isfinite(kr[d]) || !isfinite(vr[d]);
-    if (d < 2 * NG) {  // threads 0..NG-1: K groups, NG..2NG-1: V groups
-        const int which = d / NG, grp = d % NG;
-        const float* x = which ? vr : kr;
-        float mn = __int_as_float(0x7f800000), mx = -mn;
-        for (int i = 0; i < G; ++i) {
-            mn = fminf(mn, x[grp * G + i]);
-            mx = fmaxf(mx, x[grp * G + i]);
-        }
-        uint16_t s16 = scale_half_ru(__fdiv_rn(__fsub_rn(mx, mn), (float)(L - 1)));
-        uint16_t z16 = zero_half(mn);
-        gs[which][grp] = h2f(s16);
-        gz[which][grp] = h2f(z16);
-        (which ? vz : kz)[grp * TILE + tt] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+    // group extrema: butterfly over the group's lanes (min and max are exact in any order)
+    const int width = G < 32 ? G : 32;
+    float kmn = kx, kmx = kx, vmn = vx, vmx = vx;
+    for (int o = width >> 1; o > 0; o >>= 1) {
+        kmn = fminf(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+        kmx = fmaxf(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+        vmn = fminf(vmn, __shfl_xor_sync(0xffffffffu, vmn, o));
+        vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
     }
-    __syncthreads();
+    if (G > 32) {  // combine the group's warps
+        if (lane == 0) {
+            gmn[0][warp] = kmn;
+            gmx[0][warp] = kmx;
+            gmn[1][warp] = vmn;
+            gmx[1][warp] = vmx;
+        }
+        __syncthreads();
+        const int w0 = (d / G) * (G / 32);
+        for (int i = 0; i < G / 32; ++i) {
+            kmn = fminf(kmn, gmn[0][w0 + i]);
+            kmx = fmaxf(kmx, gmx[0][w0 + i]);
+            vmn = fminf(vmn, gmn[1][w0 + i]);
+            vmx = fmaxf(vmx, gmx[1][w0 + i]);
+        }
+    }
+    const uint16_t ks16 = scale_half_ru(__fdiv_rn(__fsub_rn(kmx, kmn), (float)(L - 1))), kz16 = zero_half(kmn);
+    const uint16_t vs16 = scale_half_ru(__fdiv_rn(__fsub_rn(vmx, vmn), (float)(L - 1))), vz16 = zero_half(vmn);
     const int grp = d / G;
-    kc[d] = quant_code(kr[d], gz[0][grp], gs[0][grp], L);
-    const uint32_t cv = (uint32_t)quant_code(vr[d], gz[1][grp], gs[1][grp], L);
+    if (d % G == 0) {
+        kz[grp * TILE + tt] = (uint32_t)ks16 | ((uint32_t)kz16 << 16);
+        vz[grp * TILE + tt] = (uint32_t)vs16 | ((uint32_t)vz16 << 16);
+    }
+    kc[d] = quant_code(kx, h2f(kz16), h2f(ks16), L);
+    const uint32_t cv = (uint32_t)quant_code(vx, h2f(vz16), h2f(vs16), L);
+    const bool bad = !isfinite(kx) || !isfinite(vx);
     __syncthreads();
 
     if (d < WK) {  // K word d: Horner over its k digits, top digit first
@@ -75,6 +90,8 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
         kw[d * TILE + tt] = w;
     }
     {
+        // V channel d: a fresh word at the first slot of a word; otherwise the digit is added in
+        // place (it was zero), with a reduction that needs no read
         const int pos = tt % k;
         uint32_t* p = vw + (size_t)(tt / k) * D + d;
         if (pos == 0) {
@@ -82,7 +99,7 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
         } else {
             uint32_t pw = 1u;
             for (int i = 0; i < pos; ++i) pw *= (uint32_t)L;
-            *p = *p + cv * pw;
+            atomicAdd(p, cv * pw);
         }
     }
     if (__syncthreads_or(bad) && d == 0) atomicOr(c.status, SEMKV_STATUS_NONFINITE_KV);
@@ -96,7 +113,7 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
             bm[w] = hi ? 1u : 0u;
             rk[w] = (uint32_t)nh;
         } else if (hi) {
-            bm[w] |= 1u << (T % 32);
+            atomicOr(bm + w, 1u << (T % 32));
         }
         if (hi) c.n_hi[u] = nh + 1;
         else c.n_lo[u] = nl + 1;
