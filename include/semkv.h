@@ -43,6 +43,10 @@
  *                            that holds a live slot always has zero digits at the slots past n.
  *   tau     [B*H] float      precision threshold of the unit (the n_hi-th largest score)
  *   status  [1] int32        device status word (SEMKV_STATUS_* bits)
+ *   slot_token [B*H][cap_hi + cap_lo] int32   token index of each prefill slot (L_hi segment
+ *                            first, then L_lo): the inverse of the slot map, written by
+ *                            semkv_assign_precision for slots < n and read by
+ *                            semkv_quantize_pack; appends do not update it
  * Code c of value x on a group with scale s and zero z dequantizes to fmaf((float)c, s, z).
  */
 #ifndef SEMKV_H
@@ -92,13 +96,14 @@ typedef struct semkv_cache {
     int32_t *n_hi, *n_lo;
     float *tau;
     int32_t *status;
+    int32_t *slot_token; /* [B*H][cap_hi + cap_lo], see the layout above */
 } semkv_cache_t;
 
 enum {
     SEMKV_BUF_K_HI = 0, SEMKV_BUF_V_HI, SEMKV_BUF_KZ_HI, SEMKV_BUF_VZ_HI,
     SEMKV_BUF_K_LO, SEMKV_BUF_V_LO, SEMKV_BUF_KZ_LO, SEMKV_BUF_VZ_LO,
     SEMKV_BUF_BITMAP, SEMKV_BUF_RANK, SEMKV_BUF_N_HI, SEMKV_BUF_N_LO, SEMKV_BUF_TAU, SEMKV_BUF_STATUS,
-    SEMKV_NBUF
+    SEMKV_BUF_SLOT_TOKEN, SEMKV_NBUF
 };
 
 /* Byte size of each of the SEMKV_NBUF buffers of a cache with the shape fields of `shape`
@@ -112,7 +117,8 @@ SEMKV_API int semkv_workspace_bytes(const semkv_cache_t* shape, size_t* bytes);
 /* Precision assignment (SemKV page, Abstract: tokens ranked by an internal score; the top fraction
  * gets the finer of two neighbouring grids).  scores: device fp32 [B][H][T].  For every unit:
  * n_hi = floor(p*T) (p in [0,1], computed in double); the n_hi tokens with the largest scores
- * (equal scores: lower token index first; -0 == +0) get bit 1 in the bitmap; rank[] is filled;
+ * (equal scores: lower token index first; -0 == +0) get bit 1 in the bitmap; rank[] and
+ * slot_token[] are filled;
  * n_lo = T - n_hi; tau = the n_hi-th largest score (+inf if n_hi = 0).  Requires T <= T_cap,
  * n_hi <= cap_hi and T - n_hi <= cap_lo (else SEMKV_ERR_CAPACITY).  NaN scores set
  * SEMKV_STATUS_NAN_SCORE.  Bitmap words past the last token are cleared. */

@@ -27,7 +27,7 @@ STATUS_TIMEOUT = 16
 
 SHAPE_FIELDS = ("B", "H", "Hq", "D", "G", "L_hi", "L_lo", "cap_hi", "cap_lo", "T_cap")
 BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
-             "bitmap", "rank", "n_hi", "n_lo", "tau", "status")
+             "bitmap", "rank", "n_hi", "n_lo", "tau", "status", "slot_token")
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
             "semkv_append_token", "semkv_decode_attention", "semkv_decode_attention_noalloc", "semkv_dequantize",
             "semkv_status_string", "semkv_radix_digits")

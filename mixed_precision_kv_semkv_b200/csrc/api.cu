@@ -30,7 +30,7 @@ int validate_shape(const semkv_cache_t* c)
 int validate_ptrs(const semkv_cache_t* c)
 {
     const void* p[] = {c->k_hi, c->v_hi, c->kz_hi, c->vz_hi, c->k_lo, c->v_lo, c->kz_lo, c->vz_lo,
-                       c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau, c->status};
+                       c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau, c->status, c->slot_token};
     for (const void* x : p)
         if (!x) return SEMKV_ERR_INVALID_ARG;
     return SEMKV_OK;
@@ -128,6 +128,7 @@ int semkv_cache_bytes(const semkv_cache_t* c, size_t sizes[SEMKV_NBUF])
     sizes[SEMKV_BUF_N_LO] = units * 4;
     sizes[SEMKV_BUF_TAU] = units * 4;
     sizes[SEMKV_BUF_STATUS] = 4;
+    sizes[SEMKV_BUF_SLOT_TOKEN] = units * (size_t)(c->cap_hi + c->cap_lo) * 4;
     return SEMKV_OK;
 }
 
@@ -150,7 +151,7 @@ int semkv_assign_precision(const semkv_cache_t* c, const float* scores, int32_t 
     const int n_hi = (int)std::floor((double)p * (double)T);
     if (n_hi > c->cap_hi || T - n_hi > c->cap_lo) return SEMKV_ERR_CAPACITY;
     launch_select(scores, c->B * c->H, T, n_hi, c->T_cap / 32, c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau,
-                  c->status, (cudaStream_t)stream);
+                  c->status, c->slot_token, c->cap_hi, c->cap_lo, (cudaStream_t)stream);
     return launch_status();
 }
 
@@ -161,8 +162,8 @@ int semkv_quantize_pack(const semkv_cache_t* c, const uint16_t* K, const uint16_
     if (T < 0 || T > c->T_cap || ((!K || !V) && T > 0)) return SEMKV_ERR_INVALID_ARG;
     if (T == 0) return SEMKV_OK;
     if ((((uintptr_t)K) | ((uintptr_t)V)) & 15u) return SEMKV_ERR_INVALID_ARG;  // rows are fetched by bulk copies
-    launch_quantize(seg_view(c, true), seg_view(c, false), K, V, c->bitmap, c->rank, c->B * c->H, T, c->D, c->G,
-                    c->T_cap / 32, c->status, (cudaStream_t)stream);
+    launch_quantize(seg_view(c, true), seg_view(c, false), K, V, c->slot_token, c->B * c->H, T, c->D, c->G,
+                    c->status, (cudaStream_t)stream);
     return launch_status();
 }
 

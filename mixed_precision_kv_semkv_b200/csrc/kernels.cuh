@@ -20,12 +20,14 @@ struct SegView {
     int is_hi;      // 1: L_hi segment (bitmap bit 1), 0: L_lo segment
 };
 
+// also writes slot_token [units][cap_hi + cap_lo]: the token index of every prefill slot
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
-                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st);
+                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
+                   int cap_hi, int cap_lo, cudaStream_t st);
 
+// reads the slot map (slot_token) that launch_select wrote
 void launch_quantize(const SegView& hi, const SegView& lo, const uint16_t* K, const uint16_t* V,
-                     const uint32_t* bitmap, const uint32_t* rank, int units, int T, int D, int G, int words_cap,
-                     int32_t* status, cudaStream_t st);
+                     const int32_t* slot_token, int units, int T, int D, int G, int32_t* status, cudaStream_t st);
 
 void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, cudaStream_t st);
 

@@ -7,10 +7,10 @@
 //
 // One launch covers both segments; one CTA (4 warps) per 128-slot output tile (the compile-time
 // path uses two CTAs per tile, one for its K rows and one for its V rows):
-//   1. warp 0 maps the tile's slots to token indices (32-ary search of the rank directory for the
-//      first bitmap word, then a ballot scan); all threads then copy each token's K and V row
-//      (256 B each) into shared memory in 16-byte cp.async pieces (rows of slots past the
-//      segment's end are zeroed);
+//   1. each warp reads the tokens of its 32 slots from the slot map (written by the precision
+//      assignment) and copies their K and V rows (256 B each) into shared memory in 16-byte
+//      cp.async pieces (rows of slots past the segment's end are zeroed); no warp waits for
+//      another;
 //   2. thread t quantizes K row t and packs it along the channels;
 //   3. thread t writes the scale/zero of V row t; after a barrier thread d packs channel d of
 //      every slot along the tile's slots.
@@ -32,6 +32,8 @@ constexpr int QROW = 136;  // halves per shared row: 128 + 8; rows 272 B apart k
 struct QuantSeg {
     uint32_t *k, *v, *kz, *vz;
     const int32_t* n;
+    const int32_t* map;  // slot -> token of unit 0; unit u at + u * map_stride
+    int map_stride;
     int L, k_digits, tiles_cap, is_hi;
 };
 
@@ -74,71 +76,24 @@ __device__ __forceinline__ uint32_t code_of(float x, const Grid& g, float top)
     return __float_as_uint(__fadd_rn(q, 12582912.0f)) - 0x4B400000u;
 }
 
-// One warp: slots [s0, s0 + nv) of a segment -> token indices in tok[] (entries not found stay as
-// they were).  A 32-ary search of the rank directory finds the last bitmap word whose count of
-// earlier tokens of the class is <= s0; a ballot scan of the following words emits the tokens.
-__device__ __forceinline__ void map_slots_warp(int* tok, bool is_hi, int s0, int nv, const uint32_t* __restrict__ bm,
-                                               const uint32_t* __restrict__ rk, int T)
-{
-    const int lane = threadIdx.x & 31;
-    const int nwords = (T + 31) / 32;
-    auto before = [&](int w) -> int { return is_hi ? (int)rk[w] : 32 * w - (int)rk[w]; };
-    int lo_w = 0, hi_w = nwords;  // the last word with before() <= s0 lies in [lo_w, hi_w)
-    while (hi_w - lo_w > 1) {
-        const int step = (hi_w - lo_w + 31) / 32;
-        const int probe = lo_w + lane * step;
-        const bool ok = probe < hi_w && before(probe) <= s0;
-        const unsigned m = __ballot_sync(0xffffffffu, ok);
-        lo_w += (31 - __clz(m)) * step;
-        hi_w = min(hi_w, lo_w + step);
-    }
-    int cur = lo_w, base = before(lo_w);
-    while (true) {
-        const int w = cur + lane;
-        uint32_t m = 0u;
-        if (w < nwords) {
-            const uint32_t b = bm[w];
-            const uint32_t valid = (32 * (w + 1) <= T) ? 0xffffffffu : ((1u << (T - 32 * w)) - 1u);
-            m = is_hi ? b : (~b & valid);
-        }
-        const int cnt = __popc(m);
-        const int inc = (int)warp_incl_scan((uint32_t)cnt);
-        int my = base + inc - cnt;
-        while (m) {
-            const int bit = __ffs(m) - 1;
-            m &= m - 1u;
-            if (my >= s0 && my < s0 + nv) tok[my - s0] = 32 * w + bit;
-            ++my;
-        }
-        base += __shfl_sync(0xffffffffu, inc, 31);
-        cur += 32;
-        if (base >= s0 + nv || cur >= nwords) break;
-    }
-    __syncwarp();
-}
-
-// Slots [s0, s0 + nv) of a segment of unit u -> token indices (tok), and each token's K row and V
-// row (256 B each; V/Vs may be null) into shared memory: warp 0 searches the rank directory
-// (32-ary) for the first bitmap word and scans the following words with ballots; then all 128
-// threads move the rows in 16-byte cp.async pieces (16 consecutive threads per row, so every
-// warp reads two whole rows per instruction); rows of slots past nv are zeroed.
-__device__ __forceinline__ void gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok, bool is_hi, int u, int s0, int nv,
-                                            const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
-                                            const uint32_t* __restrict__ bitmap, const uint32_t* __restrict__ rank,
-                                            int T, int words_cap)
+// This warp's 32 slots of the tile (slots s0 + 32 w .. s0 + 32 w + 31, those past nv empty): their
+// tokens from the slot map, and those tokens' K row and V row (256 B each; V/Vs may be null) into
+// shared memory in 16-byte cp.async pieces (16 lanes per row, so every instruction reads two
+// whole rows); rows of empty slots are zeroed.  Only the calling warp waits: the warps of a CTA
+// fetch and start on their rows independently.
+__device__ __forceinline__ void gather_rows_warp(uint16_t* Ks, uint16_t* Vs, const QuantSeg& seg, int u, int s0, int nv,
+                                                 const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
+                                                 int T)
 {
     constexpr int D = 128;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    tok[tid] = -1;
-    __syncthreads();
-    if (warp == 0)
-        map_slots_warp(tok, is_hi, s0, nv, bitmap + (size_t)u * words_cap, rank + (size_t)u * words_cap, T);
-    __syncthreads();
-    for (int c = tid; c < TILE * (D / 8); c += 128) {
-        const int r = c >> 4, part = (c & 15) * 8;
-        const int t = r < nv ? tok[r] : -1;
-        uint16_t* dk = Ks + r * QROW + part;
-        uint16_t* dv = Vs ? Vs + r * QROW + part : nullptr;
+    const int lane = threadIdx.x & 31, r0 = 32 * (threadIdx.x >> 5);
+    const int mine = r0 + lane < nv ? __ldg(seg.map + (size_t)u * seg.map_stride + s0 + r0 + lane) : -1;
+#pragma unroll 4
+    for (int c = lane; c < 32 * (D / 8); c += 32) {
+        const int rr = c >> 4, part = (c & 15) * 8;
+        const int t = __shfl_sync(0xffffffffu, mine, rr);
+        uint16_t* dk = Ks + (r0 + rr) * QROW + part;
+        uint16_t* dv = Vs ? Vs + (r0 + rr) * QROW + part : nullptr;
         if (t >= 0 && t < T) {
             const size_t off = ((size_t)u * T + t) * D + part;
             cp_async16(dk, K + off);
@@ -149,13 +104,12 @@ __device__ __forceinline__ void gather_rows(uint16_t* Ks, uint16_t* Vs, int* tok
         }
     }
     cp_async_wait_all();
-    __syncthreads();
+    __syncwarp();
 }
 
 __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
                                                    const uint16_t* __restrict__ V,
-                                                   const uint32_t* __restrict__ bitmap,
-                                                   const uint32_t* __restrict__ rank, int T, int G, int words_cap,
+                                                   int T, int G,
                                                    int32_t* __restrict__ status)
 {
     constexpr int D = 128;
@@ -177,9 +131,8 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     extern __shared__ __align__(128) unsigned char smem[];
     uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
     uint16_t* Vs = Ks + TILE * QROW;
-    int* tok = reinterpret_cast<int*>(Vs + TILE * QROW);
-    float4* vgrid = reinterpret_cast<float4*>(tok + TILE);  // [TILE][NG] (s, r, z, -)
-    gather_rows(Ks, Vs, tok, is_hi, u, s0, nv, K, V, bitmap, rank, T, words_cap);
+    float4* vgrid = reinterpret_cast<float4*>(Vs + TILE * QROW);  // [TILE][NG] (s, r, z, -)
+    gather_rows_warp(Ks, Vs, seg, u, s0, nv, K, V, T);
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     uint32_t* kw = seg.k + tile_base * WK * TILE;
@@ -457,8 +410,7 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
 template <int LH, int LL, int G>
 __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
                                                         const uint16_t* __restrict__ V,
-                                                        const uint32_t* __restrict__ bitmap,
-                                                        const uint32_t* __restrict__ rank, int T, int words_cap,
+                                                        int T,
                                                         int32_t* __restrict__ status)
 {
     constexpr int D = 128, NG = D / G;
@@ -476,9 +428,7 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
 
     extern __shared__ __align__(128) unsigned char smem[];
     uint16_t* Xs = reinterpret_cast<uint16_t*>(smem);  // this CTA's rows: K rows or V rows
-    int* tok = reinterpret_cast<int*>(Xs + TILE * QROW);
-    gather_rows(Xs, nullptr, tok, is_hi, u, s0, min(TILE, n - s0), part ? V : K, nullptr, bitmap, rank, T,
-                words_cap);
+    gather_rows_warp(Xs, nullptr, seg, u, s0, min(TILE, n - s0), part ? V : K, nullptr, T);
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     const int W_hi = ceil_div(D, radix_k(LH)), W_lo = ceil_div(D, radix_k(LL));
@@ -500,17 +450,18 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
 
 static size_t quantize_smem(int G)
 {
-    return (size_t)2 * TILE * QROW * 2 + TILE * 4 + (size_t)TILE * (128 / G) * 16;
+    return (size_t)2 * TILE * QROW * 2 + (size_t)TILE * (128 / G) * 16;
 }
 
 void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, const uint16_t* V,
-                     const uint32_t* bitmap, const uint32_t* rank, int units, int T, int D, int G, int words_cap,
+                     const int32_t* slot_token, int units, int T, int D, int G,
                      int32_t* status, cudaStream_t st)
 {
     (void)D;
     const int per_unit = shi.tiles_cap + slo.tiles_cap;
     if (per_unit == 0 || units == 0) return;
-    auto conv = [](const SegView& s) {
+    const int map_stride = (shi.tiles_cap + slo.tiles_cap) * TILE;
+    auto conv = [&](const SegView& s, const int32_t* map) {
         QuantSeg q;
         q.k = s.k;
         q.v = s.v;
@@ -521,16 +472,18 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
         q.k_digits = radix_k(s.L);
         q.tiles_cap = s.tiles_cap;
         q.is_hi = s.is_hi;
+        q.map = map;
+        q.map_stride = map_stride;
         return q;
     };
     const unsigned grid = (unsigned)units * per_unit;
-    const QuantSeg qh = conv(shi), ql = conv(slo);
+    const QuantSeg qh = conv(shi, slot_token), ql = conv(slo, slot_token + shi.tiles_cap * TILE);
     // compile-time level pairs and group sizes of the common configurations
 #define SEMKV_QF(LH, LL, GG)                                                                                  \
     if (shi.L == LH && slo.L == LL && G == GG) {                                                              \
-        const size_t sm = (size_t)TILE * QROW * 2 + TILE * 4;                                                 \
+        const size_t sm = (size_t)TILE * QROW * 2;                                                            \
         cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, words_cap, status); \
+        k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, status);                      \
         return;                                                                                               \
     }
 #define SEMKV_QF_G(LH, LL) SEMKV_QF(LH, LL, 32) SEMKV_QF(LH, LL, 64) SEMKV_QF(LH, LL, 128)
@@ -539,7 +492,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
 #undef SEMKV_QF
     const size_t sm = quantize_smem(G);
     cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_quantize<<<grid, 128, sm, st>>>(qh, ql, K, V, bitmap, rank, T, G, words_cap, status);
+    k_quantize<<<grid, 128, sm, st>>>(qh, ql, K, V, T, G, status);
 }
 
 }  // namespace semkv

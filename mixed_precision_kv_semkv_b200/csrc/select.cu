@@ -31,17 +31,41 @@ __device__ __forceinline__ float key_score(uint32_t k)
 
 // One CTA of 1024 threads per unit.  CACHED: the keys are first copied into shared memory (T up to
 // 48K tokens), otherwise every pass streams them from global memory (L2).
+// The slot map of a warp's 32 consecutive bitmap words (lane l holds word w0 + l, its bits and the
+// number of L_hi tokens before it): for each word in turn, lane i places token 32 w + i at its slot,
+// rank within its class, so each word gives two contiguous runs of stores.  Words at or past
+// `w_end` are not this warp's (or hold no token).
+__device__ __forceinline__ void emit_slot_tokens(int32_t* __restrict__ st_hi, int32_t* __restrict__ st_lo, int w0,
+                                                 int w_end, uint32_t word, uint32_t ones_before, int T)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < 32; ++j) {
+        const int w = w0 + j;
+        if (w >= w_end) break;  // uniform over the warp
+        const uint32_t bits = __shfl_sync(0xffffffffu, word, j);
+        const uint32_t ob = __shfl_sync(0xffffffffu, ones_before, j);
+        const int t = 32 * w + lane;
+        if (t < T) {
+            if ((bits >> lane) & 1u) st_hi[ob + __popc(bits & below)] = t;
+            else st_lo[32 * w - (int)ob + __popc(~bits & below)] = t;
+        }
+    }
+}
+
 template <bool CACHED>
 __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ scores, int T, int n_hi, int words_cap,
                                                   uint32_t* __restrict__ bitmap, uint32_t* __restrict__ rank,
                                                   int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
-                                                  float* __restrict__ tau_out, int32_t* __restrict__ status)
+                                                  float* __restrict__ tau_out, int32_t* __restrict__ status,
+                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo)
 {
     const int u = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const float* s = scores + (size_t)u * T;
     uint32_t* bm = bitmap + (size_t)u * words_cap;
     uint32_t* rk = rank + (size_t)u * words_cap;
+    int32_t* st_hi = slot_token + (size_t)u * (cap_hi + cap_lo);
 
     __shared__ uint32_t hist[256];
     __shared__ uint32_t scan_tmp[33];
@@ -151,6 +175,7 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
             bm[w] = word;
             rk[w] = ones_before;
         }
+        emit_slot_tokens(st_hi, st_hi + cap_hi, c + (tid & ~31), nwords, w < nwords ? word : 0u, ones_before, T);
     }
     for (int w = nwords + tid; w < words_cap; w += blockDim.x) {
         bm[w] = 0u;
@@ -182,7 +207,8 @@ template <int KPT>
 __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     k_select_cluster(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
                      uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
-                     float* __restrict__ tau_out, int32_t* __restrict__ status)
+                     float* __restrict__ tau_out, int32_t* __restrict__ status,
+                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo)
 {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -363,6 +389,11 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
         bm[w0 + tid] = word;
         rk[w0 + tid] = ones_before;
     }
+    {
+        int32_t* st_hi = slot_token + (size_t)u * (cap_hi + cap_lo);
+        emit_slot_tokens(st_hi, st_hi + cap_hi, w0 + (tid & ~31), min(nwords, w0 + nw), tid < nw ? word : 0u,
+                         ones_before, T);
+    }
     for (int w = nwords + c * SEL_THREADS + tid; w < words_cap; w += SEL_CS * SEL_THREADS) {
         bm[w] = 0u;
         rk[w] = (uint32_t)n_hi;
@@ -387,7 +418,8 @@ template <int KPT>
 __global__ void __launch_bounds__(SELR_THREADS)
     k_select_reg(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
                  uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
-                 float* __restrict__ tau_out, int32_t* __restrict__ status)
+                 float* __restrict__ tau_out, int32_t* __restrict__ status,
+                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo)
 {
     const int u = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -486,6 +518,10 @@ __global__ void __launch_bounds__(SELR_THREADS)
         bm[tid] = word;
         rk[tid] = ones_before;
     }
+    {
+        int32_t* st_hi = slot_token + (size_t)u * (cap_hi + cap_lo);
+        emit_slot_tokens(st_hi, st_hi + cap_hi, tid & ~31, nwords, tid < nwords ? word : 0u, ones_before, T);
+    }
     for (int w = nwords + tid; w < words_cap; w += SELR_THREADS) {
         bm[w] = 0u;
         rk[w] = (uint32_t)n_hi;
@@ -498,11 +534,12 @@ __global__ void __launch_bounds__(SELR_THREADS)
 }
 
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
-                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, cudaStream_t st)
+                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
+                   int cap_hi, int cap_lo, cudaStream_t st)
 {
     if (T <= SELR_THREADS) {  // one key per thread: a single CTA
         k_select_reg<1><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out,
-                                                        n_lo_out, tau, status);
+                                                        n_lo_out, tau, status, slot_token, cap_hi, cap_lo);
         return;
     }
     const int nwords = (T + 31) / 32;
@@ -512,14 +549,14 @@ void launch_select(const float* scores, int units, int T, int n_hi, int words_ca
 #define SEMKV_SEL(K)                                                                                           \
     if (kpt <= K) {                                                                                            \
         k_select_cluster<K><<<grid, SEL_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, \
-                                                          n_lo_out, tau, status);                             \
+                                                          n_lo_out, tau, status, slot_token, cap_hi, cap_lo);                             \
         return;                                                                                                \
     }
     SEMKV_SEL(1) SEMKV_SEL(2) SEMKV_SEL(4) SEMKV_SEL(8) SEMKV_SEL(16) SEMKV_SEL(32)
 #undef SEMKV_SEL
     // more keys than a cluster holds in registers: one CTA per unit streams the scores from L2
     k_select<false><<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
-                                            status);
+                                            status, slot_token, cap_hi, cap_lo);
 }
 
 }  // namespace semkv

@@ -41,6 +41,9 @@ def unit_views(cache: SemkvCache, bufs: dict, u: int):
     out["n_hi"] = int(bufs["n_hi"][u])
     out["n_lo"] = int(bufs["n_lo"][u])
     out["tau"] = np.float32(bufs["tau"].view(np.float32)[u])
+    caps = cache.cap_hi + cache.cap_lo
+    st = bufs["slot_token"].view(np.int32)[: units * caps].reshape(units, caps)[u]
+    out["slot_hi"], out["slot_lo"] = st[: cache.cap_hi], st[cache.cap_hi:]
     return out
 
 
@@ -99,6 +102,11 @@ def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = "
     assert np.array_equal(g["rank"][:nw], o["rank"][:nw]), f"rank {where}"
     assert g["n_hi"] == o["n_hi"] and g["n_lo"] == T - o["n_hi"], f"counts {where}"
     assert np.float32(g["tau"]).view(np.uint32) == np.float32(o["tau"]).view(np.uint32), f"tau {where}"
+    if strict_tail and "slot_hi" in g:  # after a prefill: the slot map is the inverse of the ranks
+        bits = np.unpackbits(o["bitmap"][:nw].view(np.uint8), bitorder="little")[:T].astype(bool)
+        tokens = np.arange(T)
+        assert np.array_equal(g["slot_hi"][: o["n_hi"]], tokens[bits]), f"slot map hi {where}"
+        assert np.array_equal(g["slot_lo"][: T - o["n_hi"]], tokens[~bits]), f"slot map lo {where}"
     for seg, n, L in (("hi", o["n_hi"], L_hi), ("lo", T - o["n_hi"], L_lo)):
         if strict_tail:
             nt = -(-n // 128)
