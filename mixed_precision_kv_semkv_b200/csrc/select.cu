@@ -389,10 +389,27 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
         bm[w0 + tid] = word;
         rk[w0 + tid] = ones_before;
     }
+    // slot map: every thread places the tokens of its own keys (bitmap words and their counts of
+    // L_hi tokens before them staged in shared memory; gtm/eqm are free again)
+    if (tid < nw) {
+        gtm[tid] = word;
+        eqm[tid] = ones_before;
+    }
+    __syncthreads();
     {
         int32_t* st_hi = slot_token + (size_t)u * (cap_hi + cap_lo);
-        emit_slot_tokens(st_hi, st_hi + cap_hi, w0 + (tid & ~31), min(nwords, w0 + nw), tid < nw ? word : 0u,
-                         ones_before, T);
+        int32_t* st_lo = st_hi + cap_hi;
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int j = 0; j < KPT; ++j) {
+            const int t = tok0 + j * SEL_THREADS + tid;
+            if (t < 32 * w1 && t < T) {
+                const int wl = j * SEL_WARPS + wid;  // the word of token t, within this CTA
+                const uint32_t wd = gtm[wl], ob = eqm[wl];
+                if ((wd >> lane) & 1u) st_hi[ob + __popc(wd & below)] = t;
+                else st_lo[32 * (w0 + wl) - (int)ob + __popc(~wd & below)] = t;
+            }
+        }
     }
     for (int w = nwords + c * SEL_THREADS + tid; w < words_cap; w += SEL_CS * SEL_THREADS) {
         bm[w] = 0u;
