@@ -189,6 +189,17 @@ SEMKV_API const char* semkv_status_string(int code);
  * Pure host function; returns 0 for L outside [2, 256]. */
 SEMKV_API int32_t semkv_radix_digits(int32_t L);
 
+/* Fraction of tokens the finer grid can take under a storage budget (SemKV page, Abstract: measure
+ * the quality cliff, then interpolate above it).  Physical bits per cached value are
+ *   bits(p) = [p*32*W(L_hi) + (1-p)*32*W(L_lo)]/D + 32/G + 1/(2D)
+ * (code words, fp16 scale + zero per group, the precision bitmap shared by K and V), with
+ * W(L) = ceil(D/k(L)) words per row.  *p receives the largest p in [0,1] with 16/bits(p) >= ratio,
+ * to be passed to semkv_assign_precision (which puts floor(p*T) tokens on the finer grid, never
+ * more).  Pure host function.  Returns SEMKV_ERR_INVALID_ARG (null p, ratio not > 0, D or G not
+ * positive, G not dividing D), SEMKV_ERR_UNSUPPORTED (L outside [2, 256]) or SEMKV_ERR_CAPACITY
+ * (even p = 0 gives a smaller reduction than `ratio`). */
+SEMKV_API int semkv_p_for_ratio(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, double ratio, double* p);
+
 #ifdef __cplusplus
 }
 #endif

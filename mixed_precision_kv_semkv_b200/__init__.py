@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     semkv_decode_attention_noalloc,
     semkv_dequantize,
     semkv_quantize_pack,
+    semkv_p_for_ratio,
     semkv_radix_digits,
     semkv_workspace_bytes,
     status_string,

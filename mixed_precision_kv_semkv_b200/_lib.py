@@ -30,7 +30,7 @@ BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
              "bitmap", "rank", "n_hi", "n_lo", "tau", "status", "slot_token")
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
             "semkv_append_token", "semkv_decode_attention", "semkv_decode_attention_noalloc", "semkv_dequantize",
-            "semkv_status_string", "semkv_radix_digits")
+            "semkv_status_string", "semkv_radix_digits", "semkv_p_for_ratio")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.semkv_status_string.restype = ctypes.c_char_p
         L.semkv_radix_digits.argtypes = [i32]
         L.semkv_radix_digits.restype = i32
+        L.semkv_p_for_ratio.argtypes = [i32, i32, i32, i32, ctypes.c_double, ctypes.POINTER(ctypes.c_double)]
         for n in EXPORTED:
             if n not in ("semkv_status_string", "semkv_radix_digits"):
                 getattr(L, n).restype = ctypes.c_int
@@ -104,6 +105,14 @@ def _struct(cache) -> CacheStruct:
 
 def semkv_radix_digits(L: int) -> int:
     return int(lib().semkv_radix_digits(int(L)))
+
+
+def semkv_p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float) -> float:
+    """Largest fraction p on the L_hi grid whose storage reduction vs fp16 is still >= ratio."""
+    p = ctypes.c_double()
+    _check("semkv_p_for_ratio", lib().semkv_p_for_ratio(int(D), int(G), int(L_hi), int(L_lo), float(ratio),
+                                                       ctypes.byref(p)))
+    return p.value
 
 
 def semkv_cache_bytes(cache) -> list[int]:

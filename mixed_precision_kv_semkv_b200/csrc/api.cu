@@ -107,6 +107,24 @@ extern "C" {
 
 int32_t semkv_radix_digits(int32_t L) { return level_ok(L) ? radix_k(L) : 0; }
 
+int semkv_p_for_ratio(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, double ratio, double* p)
+{
+    if (!p || !(ratio > 0.0) || !std::isfinite(ratio) || D < 1 || G < 1 || D % G) return SEMKV_ERR_INVALID_ARG;
+    if (!level_ok(L_hi) || !level_ok(L_lo)) return SEMKV_ERR_UNSUPPORTED;
+    // bits(p) = a + b p, linear in p; the budget is 16 / ratio bits per value
+    const double w_hi = ceil_div(D, radix_k(L_hi)), w_lo = ceil_div(D, radix_k(L_lo));
+    const double a = 32.0 * w_lo / D + 32.0 / G + 1.0 / (2.0 * D), b = 32.0 * (w_hi - w_lo) / D;
+    const double budget = 16.0 / ratio;
+    if (a + b <= budget) {  // p = 1 fits (also every b <= 0 case that fits at all)
+        *p = 1.0;
+        return SEMKV_OK;
+    }
+    if (b <= 0.0 || a > budget) return SEMKV_ERR_CAPACITY;
+    const double x = (budget - a) / b;  // in [0, 1) here
+    *p = x < 0.0 ? 0.0 : x;
+    return SEMKV_OK;
+}
+
 int semkv_cache_bytes(const semkv_cache_t* c, size_t sizes[SEMKV_NBUF])
 {
     int r = validate_shape(c);

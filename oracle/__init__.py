@@ -255,6 +255,31 @@ def attention_fp64(q16, Khat, Vhat, sm_scale: float) -> np.ndarray:
     return out
 
 
+def p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float, iters: int = 200):
+    """Largest fraction p in [0, 1] of tokens on the L_hi grid whose storage reduction against
+    fp16 (16 bits / storage_bits_per_value) is still at least `ratio`; None if even p = 0 misses
+    it.  SemKV page, Abstract: the recipe is to measure the quality cliff and then interpolate
+    above it -- the finer grid's share is what a storage budget leaves room for.  Plain bisection
+    on the buffer-derived storage above (no closed-form inversion)."""
+    if not ratio > 0.0:
+        return None
+    ok = lambda p: 16.0 / storage_bits_per_value(D, G, L_hi, L_lo, p) >= ratio  # noqa: E731
+    if ok(1.0):
+        return 1.0
+    if not ok(0.0):
+        return None
+    lo, hi = 0.0, 1.0  # ok(lo), not ok(hi)
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        if ok(mid):
+            lo = mid
+        else:
+            hi = mid
+        if hi - lo < 1e-15:
+            break
+    return lo
+
+
 def storage_bits_per_value(D: int, G: int, L_hi: int, L_lo: int, p_real: float) -> float:
     """Physical bits per cached value (K or V), from the oracle's own buffer sizes per full tile.
 

@@ -18,3 +18,14 @@ def orc():
 
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def semkv():
+    """The library's Python binding (builds libsemkv.so first if it is stale; loads without a GPU)."""
+    from mixed_precision_kv_semkv_b200 import build
+
+    build.build()
+    import mixed_precision_kv_semkv_b200 as m
+
+    return m

@@ -11,16 +11,6 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.fixture(scope="module")
-def semkv():
-    from mixed_precision_kv_semkv_b200 import build
-
-    build.build()
-    import mixed_precision_kv_semkv_b200 as m
-
-    return m
-
-
 def _declared_symbols():
     names = set()
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
