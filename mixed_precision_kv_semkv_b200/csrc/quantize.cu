@@ -414,13 +414,17 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
                                                         int32_t* __restrict__ status)
 {
     constexpr int D = 128, NG = D / G;
-    const int per_unit = hi.tiles_cap + lo.tiles_cap;
+    // segment-major order (every unit's L_lo tiles, then every unit's L_hi tiles): the CTAs
+    // resident at any time mostly run one segment's two code paths, which keeps instruction
+    // fetch local
     const int part = blockIdx.x & 1;  // 0: K rows, 1: V rows of the tile
-    const int u = (blockIdx.x >> 1) / per_unit;
-    int tile = (blockIdx.x >> 1) % per_unit;
-    const bool is_hi = tile < hi.tiles_cap;
+    const int units = (int)(gridDim.x / 2) / (hi.tiles_cap + lo.tiles_cap);
+    const int item = blockIdx.x >> 1, n_lo_items = units * lo.tiles_cap;
+    const bool is_hi = item >= n_lo_items;
     const QuantSeg& seg = is_hi ? hi : lo;
-    if (!is_hi) tile -= hi.tiles_cap;
+    const int it = is_hi ? item - n_lo_items : item;
+    const int u = it / seg.tiles_cap;
+    const int tile = it % seg.tiles_cap;
     const int tid = threadIdx.x;
     const int n = seg.n[u];
     const int s0 = tile * TILE;
