@@ -47,6 +47,9 @@
  *                            first, then L_lo): the inverse of the slot map, written by
  *                            semkv_assign_precision for slots < n and read by
  *                            semkv_quantize_pack; appends do not update it
+ *   score_keys [B*H][T_cap] uint32   every token's score as an order-preserving key (-0 as +0;
+ *                            key order = score order), written by semkv_assign_precision and by
+ *                            every append; semkv_append_token_running ranks a new token by it
  * Code c of value x on a group with scale s and zero z dequantizes to fmaf((float)c, s, z).
  */
 #ifndef SEMKV_H
@@ -96,14 +99,15 @@ typedef struct semkv_cache {
     int32_t *n_hi, *n_lo;
     float *tau;
     int32_t *status;
-    int32_t *slot_token; /* [B*H][cap_hi + cap_lo], see the layout above */
+    int32_t *slot_token;  /* [B*H][cap_hi + cap_lo], see the layout above */
+    uint32_t *score_keys; /* [B*H][T_cap], see the layout above */
 } semkv_cache_t;
 
 enum {
     SEMKV_BUF_K_HI = 0, SEMKV_BUF_V_HI, SEMKV_BUF_KZ_HI, SEMKV_BUF_VZ_HI,
     SEMKV_BUF_K_LO, SEMKV_BUF_V_LO, SEMKV_BUF_KZ_LO, SEMKV_BUF_VZ_LO,
     SEMKV_BUF_BITMAP, SEMKV_BUF_RANK, SEMKV_BUF_N_HI, SEMKV_BUF_N_LO, SEMKV_BUF_TAU, SEMKV_BUF_STATUS,
-    SEMKV_BUF_SLOT_TOKEN, SEMKV_NBUF
+    SEMKV_BUF_SLOT_TOKEN, SEMKV_BUF_SCORE_KEYS, SEMKV_NBUF
 };
 
 /* Byte size of each of the SEMKV_NBUF buffers of a cache with the shape fields of `shape`
@@ -143,6 +147,16 @@ SEMKV_API int semkv_quantize_pack(const semkv_cache_t* cache, const uint16_t* K,
  * SEMKV_STATUS_APPEND_OVERFLOW; a NaN score sets SEMKV_STATUS_NAN_SCORE (the token goes lo). */
 SEMKV_API int semkv_append_token(const semkv_cache_t* cache, const uint16_t* k, const uint16_t* v, const float* score,
                        void* stream);
+
+/* semkv_append_token with the exact running top-p rule instead of the fixed threshold tau: the
+ * new token goes on the L_hi grid iff it is among the floor(p*(T+1)) largest of the unit's T+1
+ * scores (equal scores: lower token index first, so the new token loses ties), i.e. iff fewer than
+ * floor(p*(T+1)) earlier tokens have a score >= its score.  Earlier tokens keep their grid (their
+ * original values are gone), so n_hi may differ from floor(p*(T+1)).  p in [0,1] (else
+ * SEMKV_ERR_INVALID_ARG); reads the unit's score_keys (4 B per token); otherwise as
+ * semkv_append_token. */
+SEMKV_API int semkv_append_token_running(const semkv_cache_t* cache, const uint16_t* k, const uint16_t* v,
+                                         const float* score, float p, void* stream);
 
 /* GQA decode attention over the packed cache.  q: device fp16 [B][Hq][D]; out: device fp32
  * [B][Hq][D].  Query head qh attends with kv head qh / (Hq/H) over all n_hi + n_lo tokens of its

@@ -7,6 +7,7 @@ binding (`_lib`, same function names as the C entry points), a torch-allocated c
 from ._lib import (  # noqa: F401
     SemkvError,
     semkv_append_token,
+    semkv_append_token_running,
     semkv_assign_precision,
     semkv_cache_bytes,
     semkv_decode_attention,

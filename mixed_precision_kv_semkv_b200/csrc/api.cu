@@ -30,7 +30,8 @@ int validate_shape(const semkv_cache_t* c)
 int validate_ptrs(const semkv_cache_t* c)
 {
     const void* p[] = {c->k_hi, c->v_hi, c->kz_hi, c->vz_hi, c->k_lo, c->v_lo, c->kz_lo, c->vz_lo,
-                       c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau, c->status, c->slot_token};
+                       c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau, c->status, c->slot_token,
+                       c->score_keys};
     for (const void* x : p)
         if (!x) return SEMKV_ERR_INVALID_ARG;
     return SEMKV_OK;
@@ -147,6 +148,7 @@ int semkv_cache_bytes(const semkv_cache_t* c, size_t sizes[SEMKV_NBUF])
     sizes[SEMKV_BUF_TAU] = units * 4;
     sizes[SEMKV_BUF_STATUS] = 4;
     sizes[SEMKV_BUF_SLOT_TOKEN] = units * (size_t)(c->cap_hi + c->cap_lo) * 4;
+    sizes[SEMKV_BUF_SCORE_KEYS] = units * (size_t)c->T_cap * 4;
     return SEMKV_OK;
 }
 
@@ -169,7 +171,7 @@ int semkv_assign_precision(const semkv_cache_t* c, const float* scores, int32_t 
     const int n_hi = (int)std::floor((double)p * (double)T);
     if (n_hi > c->cap_hi || T - n_hi > c->cap_lo) return SEMKV_ERR_CAPACITY;
     launch_select(scores, c->B * c->H, T, n_hi, c->T_cap / 32, c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau,
-                  c->status, c->slot_token, c->cap_hi, c->cap_lo, (cudaStream_t)stream);
+                  c->status, c->slot_token, c->cap_hi, c->cap_lo, c->score_keys, (cudaStream_t)stream);
     return launch_status();
 }
 
@@ -191,7 +193,17 @@ int semkv_append_token(const semkv_cache_t* c, const uint16_t* k, const uint16_t
     int r = validate(c);
     if (r != SEMKV_OK) return r;
     if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
-    launch_append(*c, k, v, score, (cudaStream_t)stream);
+    launch_append(*c, k, v, score, -1.0f, (cudaStream_t)stream);
+    return launch_status();
+}
+
+int semkv_append_token_running(const semkv_cache_t* c, const uint16_t* k, const uint16_t* v, const float* score,
+                               float p, void* stream)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (!k || !v || !score || !(p >= 0.0f && p <= 1.0f)) return SEMKV_ERR_INVALID_ARG;
+    launch_append(*c, k, v, score, p, (cudaStream_t)stream);
     return launch_status();
 }
 

@@ -12,8 +12,11 @@
 
 namespace semkv {
 
+// p < 0: the token goes on the L_hi grid iff score > tau.  p >= 0 (running top-p): iff fewer than
+// floor(p (T+1)) earlier tokens have a score >= its score (the newest token loses ties).
 __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t* __restrict__ knew,
-                                                 const uint16_t* __restrict__ vnew, const float* __restrict__ score)
+                                                 const uint16_t* __restrict__ vnew, const float* __restrict__ score,
+                                                 float p)
 {
     constexpr int D = 128;
     const int u = blockIdx.x, d = threadIdx.x, lane = d & 31, warp = d >> 5;
@@ -27,8 +30,28 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
     const int nh = c.n_hi[u], nl = c.n_lo[u];
     const float kx = h2f(knew[(size_t)u * D + d]);
     const float vx = h2f(vnew[(size_t)u * D + d]);
-    const bool hi = sc > tau;  // NaN compares false: the token goes lo
     const int T = nh + nl;
+    const uint32_t key = order_key(sc);
+    bool hi;
+    if (p < 0.0f) {
+        hi = sc > tau;  // NaN compares false: the token goes lo
+    } else {
+        // rank of the new token among all T + 1 scores: earlier keys >= its key, 4 per load
+        __shared__ int cnt_s[4];
+        const uint32_t* keys = c.score_keys + (size_t)u * c.T_cap;
+        int cnt = 0;
+        for (int t = 4 * d; t < T; t += 4 * 128) {  // t + 3 < T_cap: T < T_cap, T_cap % 32 == 0
+            const uint4 k4 = *reinterpret_cast<const uint4*>(keys + t);
+            cnt += (k4.x >= key) + (t + 1 < T && k4.y >= key) + (t + 2 < T && k4.z >= key) + (t + 3 < T && k4.w >= key);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) cnt_s[warp] = cnt;
+        __syncthreads();
+        const int total = cnt_s[0] + cnt_s[1] + cnt_s[2] + cnt_s[3];
+        const double target = floor((double)p * (double)(T + 1));
+        hi = !isnan(sc) && (double)total < target;
+    }
     const int slot = hi ? nh : nl;
     const int cap = hi ? c.cap_hi : c.cap_lo;
     if (slot >= cap || T >= c.T_cap) {
@@ -117,12 +140,14 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
         }
         if (hi) c.n_hi[u] = nh + 1;
         else c.n_lo[u] = nl + 1;
+        c.score_keys[(size_t)u * c.T_cap + T] = key;
     }
 }
 
-void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, cudaStream_t st)
+void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, float p,
+                   cudaStream_t st)
 {
-    k_append<<<c.B * c.H, 128, 0, st>>>(c, k, v, score);
+    k_append<<<c.B * c.H, 128, 0, st>>>(c, k, v, score, p);
 }
 
 }  // namespace semkv

@@ -15,6 +15,7 @@
 
 #include <cuda_fp16.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace semkv {
 
@@ -160,6 +161,15 @@ __device__ __forceinline__ float warp_max(float v)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
+}
+
+// Order-preserving uint32 image of a score (-0 taken as +0): a > b as floats iff key(a) > key(b)
+__host__ __device__ __forceinline__ uint32_t order_key(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7fffffffu) == 0u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 }  // namespace semkv

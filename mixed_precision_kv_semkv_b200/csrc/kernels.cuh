@@ -23,13 +23,15 @@ struct SegView {
 // also writes slot_token [units][cap_hi + cap_lo]: the token index of every prefill slot
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
-                   int cap_hi, int cap_lo, cudaStream_t st);
+                   int cap_hi, int cap_lo, uint32_t* score_keys, cudaStream_t st);
 
 // reads the slot map (slot_token) that launch_select wrote
 void launch_quantize(const SegView& hi, const SegView& lo, const uint16_t* K, const uint16_t* V,
                      const int32_t* slot_token, int units, int T, int D, int G, int32_t* status, cudaStream_t st);
 
-void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, cudaStream_t st);
+// p < 0: the fixed threshold rule (score > tau); p in [0, 1]: the running top-p rule
+void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, float p,
+                   cudaStream_t st);
 
 // decode: split partials of one segment go to splits [split_off, split_off + nsplit) of each unit
 void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H, int g, int D, int G,

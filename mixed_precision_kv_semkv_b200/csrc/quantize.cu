@@ -414,17 +414,20 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
                                                         int32_t* __restrict__ status)
 {
     constexpr int D = 128, NG = D / G;
-    // segment-major order (every unit's L_lo tiles, then every unit's L_hi tiles): the CTAs
-    // resident at any time mostly run one segment's two code paths, which keeps instruction
-    // fetch local
-    const int part = blockIdx.x & 1;  // 0: K rows, 1: V rows of the tile
+    // order: the L_lo segment's K rows, its V rows, then the L_hi segment's K rows and V rows
+    // (every unit's tiles in each): the CTAs resident at any time mostly run one code path,
+    // which keeps instruction fetch local
     const int units = (int)(gridDim.x / 2) / (hi.tiles_cap + lo.tiles_cap);
-    const int item = blockIdx.x >> 1, n_lo_items = units * lo.tiles_cap;
-    const bool is_hi = item >= n_lo_items;
+    const int n_lo = units * lo.tiles_cap;  // CTAs of one part of the L_lo segment
+    int item = blockIdx.x;
+    const bool is_hi = item >= 2 * n_lo;
+    if (is_hi) item -= 2 * n_lo;
     const QuantSeg& seg = is_hi ? hi : lo;
-    const int it = is_hi ? item - n_lo_items : item;
-    const int u = it / seg.tiles_cap;
-    const int tile = it % seg.tiles_cap;
+    const int n_seg = units * seg.tiles_cap;
+    const int part = item >= n_seg ? 1 : 0;  // 0: K rows, 1: V rows of the tile
+    if (part) item -= n_seg;
+    const int u = item / seg.tiles_cap;
+    const int tile = item % seg.tiles_cap;
     const int tid = threadIdx.x;
     const int n = seg.n[u];
     const int s0 = tile * TILE;

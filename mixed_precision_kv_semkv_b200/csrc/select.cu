@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
                                                   uint32_t* __restrict__ bitmap, uint32_t* __restrict__ rank,
                                                   int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
                                                   float* __restrict__ tau_out, int32_t* __restrict__ status,
-                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo)
+                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo, uint32_t* __restrict__ score_keys)
 {
     const int u = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -76,9 +76,11 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
     {
         bool bad = false;
 #pragma unroll 8
+        uint32_t* sk = score_keys + (size_t)u * 32 * words_cap;
         for (int t = tid; t < T; t += blockDim.x) {
             const float f = s[t];
             bad |= isnan(f);
+            sk[t] = score_key(f);
             if (CACHED) kcache[t] = score_key(f);
         }
         if (__syncthreads_or(bad) && tid == 0) atomicOr(status, SEMKV_STATUS_NAN_SCORE);
@@ -208,7 +210,7 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     k_select_cluster(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
                      uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
                      float* __restrict__ tau_out, int32_t* __restrict__ status,
-                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo)
+                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo, uint32_t* __restrict__ score_keys)
 {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -233,12 +235,14 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     bool bad = false;
     uint32_t kand = 0xffffffffu, kor = 0u;
 #pragma unroll
+    uint32_t* sk = score_keys + (size_t)u * 32 * words_cap;
     for (int j = 0; j < KPT; ++j) {
         const int t = tok0 + j * SEL_THREADS + tid;
         const bool in = t < 32 * w1 && t < T;
         const float f = in ? s[t] : 0.f;
         bad |= in && isnan(f);
         key[j] = in ? score_key(f) : 0u;
+        if (in) sk[t] = key[j];
         if (in) {
             kand &= key[j];
             kor |= key[j];
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(SELR_THREADS)
     k_select_reg(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
                  uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
                  float* __restrict__ tau_out, int32_t* __restrict__ status,
-                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo)
+                 int32_t* __restrict__ slot_token, int cap_hi, int cap_lo, uint32_t* __restrict__ score_keys)
 {
     const int u = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -450,11 +454,13 @@ __global__ void __launch_bounds__(SELR_THREADS)
     uint32_t key[KPT];
     bool bad = false;
 #pragma unroll
+    uint32_t* sk = score_keys + (size_t)u * 32 * words_cap;
     for (int j = 0; j < KPT; ++j) {
         const int t = j * SELR_THREADS + tid;
         const float f = t < T ? s[t] : 0.f;
         bad |= t < T && isnan(f);
         key[j] = score_key(f);
+        if (t < T) sk[t] = key[j];
     }
     if (__syncthreads_or(bad) && tid == 0) atomicOr(status, SEMKV_STATUS_NAN_SCORE);
 
@@ -552,11 +558,11 @@ __global__ void __launch_bounds__(SELR_THREADS)
 
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
-                   int cap_hi, int cap_lo, cudaStream_t st)
+                   int cap_hi, int cap_lo, uint32_t* score_keys, cudaStream_t st)
 {
     if (T <= SELR_THREADS) {  // one key per thread: a single CTA
         k_select_reg<1><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out,
-                                                        n_lo_out, tau, status, slot_token, cap_hi, cap_lo);
+                                                        n_lo_out, tau, status, slot_token, cap_hi, cap_lo, score_keys);
         return;
     }
     const int nwords = (T + 31) / 32;
@@ -566,14 +572,14 @@ void launch_select(const float* scores, int units, int T, int n_hi, int words_ca
 #define SEMKV_SEL(K)                                                                                           \
     if (kpt <= K) {                                                                                            \
         k_select_cluster<K><<<grid, SEL_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, \
-                                                          n_lo_out, tau, status, slot_token, cap_hi, cap_lo);                             \
+                                                          n_lo_out, tau, status, slot_token, cap_hi, cap_lo, score_keys);                             \
         return;                                                                                                \
     }
     SEMKV_SEL(1) SEMKV_SEL(2) SEMKV_SEL(4) SEMKV_SEL(8) SEMKV_SEL(16) SEMKV_SEL(32)
 #undef SEMKV_SEL
     // more keys than a cluster holds in registers: one CTA per unit streams the scores from L2
     k_select<false><<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
-                                            status, slot_token, cap_hi, cap_lo);
+                                            status, slot_token, cap_hi, cap_lo, score_keys);
 }
 
 }  // namespace semkv

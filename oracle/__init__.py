@@ -255,6 +255,28 @@ def attention_fp64(q16, Khat, Vhat, sm_scale: float) -> np.ndarray:
     return out
 
 
+def running_is_hi(scores_prev, score_new: float, p: float) -> bool:
+    """Exact running top-p for a generated token (reading of the running threshold): select again
+    over all T + 1 scores, the new token last, and read the new token's bit.  Earlier tokens keep
+    their grid; only the new token's assignment is taken from this selection."""
+    allsc = np.concatenate([np.asarray(scores_prev, np.float32), np.float32([score_new])])
+    T = allsc.shape[0] - 1
+    bm, _, _, _, _ = select(allsc, p)
+    return bool((int(bm[T // 32]) >> (T % 32)) & 1)
+
+
+def append_unit_running(state: UnitState, k16, v16, score: float, p: float, scores_prev, G: int, L_hi: int,
+                        L_lo: int) -> int:
+    """append_unit with the running top-p rule: the grid comes from running_is_hi (the fixed tau
+    of the state is left as it was)."""
+    tau = state.tau
+    state.tau = np.float32(-np.inf) if running_is_hi(scores_prev, score, p) else np.float32(np.inf)
+    try:
+        return append_unit(state, k16, v16, score, G, L_hi, L_lo)
+    finally:
+        state.tau = tau
+
+
 def p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float, iters: int = 200):
     """Largest fraction p in [0, 1] of tokens on the L_hi grid whose storage reduction against
     fp16 (16 bits / storage_bits_per_value) is still at least `ratio`; None if even p = 0 misses

@@ -58,6 +58,7 @@ def test_cache_bytes_match_oracle_layout(semkv, orc, L_hi, L_lo, G):
     assert sizes["n_hi"] == sizes["n_lo"] == sizes["tau"] == units * 4
     assert sizes["status"] == 4
     assert sizes["slot_token"] == units * (256 + 768) * 4
+    assert sizes["score_keys"] == units * 1024 * 4
 
 
 @pytest.mark.parametrize("bad,code", [
