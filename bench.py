@@ -78,6 +78,8 @@ def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False) -> 
         "quantize": units * T * w.D * 2 * 2 + bitmap_rank + cache,
         # the new token's k, v rows and score read, its record written
         "append": units * (w.D * 2 * 2 + 4) + new if appended else 0,
+        # the running rule also reads every stored score key and writes the new one
+        "append_running": units * (w.D * 2 * 2 + 4) + new + units * 4 * (T + 1) if appended else 0,
         "decode": cache + new + q,
         "cache": cache,
     }
@@ -241,8 +243,9 @@ def run_reference(args):
 def run_semkv(args):
     import torch
 
-    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_append_token, semkv_assign_precision,
-                                               semkv_decode_attention, semkv_quantize_pack, synth)
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_append_token, semkv_append_token_running,
+                                               semkv_assign_precision, semkv_decode_attention, semkv_quantize_pack,
+                                               synth)
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
@@ -298,6 +301,15 @@ def run_semkv(args):
         with torch.cuda.graph(gr, capture_error_mode="relaxed"):
             c()
         graphs.append(gr)
+    # the running top-p append (the same token, ranked against every stored score) for the split
+    run_call = lambda: semkv_append_token_running(cache, kn, vn, sn, w.p)  # noqa: E731
+    calls[0]()  # a fresh prefill first: the cache holds room for one appended token
+    calls[1]()
+    run_call()
+    torch.cuda.synchronize()
+    run_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(run_graph, capture_error_mode="relaxed"):
+        run_call()
 
     def step(ev=None):
         if ev is not None:
@@ -346,6 +358,23 @@ def run_semkv(args):
         step_split(evs_split[i])
     torch.cuda.synchronize()
     t_call = [sum(e[i].elapsed_time(e[i + 1]) for e in evs_split) * steps / split_steps for i in range(len(graphs))]
+    # running append: after a fresh prefill (select + quantize replayed untimed), its own graph
+    t_run = 0.0
+    for i in range(split_steps):
+        flush.zero_()
+        graphs[0].replay()
+        graphs[1].replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+        t_run += e0.elapsed_time(e1)
+    t_run /= split_steps
+    # leave the cache as a timed step leaves it (prefill + the fixed-threshold append)
+    for gr in graphs[:3]:
+        gr.replay()
+    torch.cuda.synchronize()
 
     # decode alone over an L2-cold cache (decode-attn HBM GB/s of the metric)
     dec_ms = []
@@ -372,6 +401,7 @@ def run_semkv(args):
     }
     per_kernel.update({
         "decode_l2_cold": {"ms": dec_cold, "gbs": nb["decode"] / (dec_cold * 1e-3) / 1e9},
+        "append_running": {"ms": t_run, "gbs": nb["append_running"] / (t_run * 1e-3) / 1e9},
     })
     dom = max(("select", "quantize", "decode_in_step"), key=lambda k: per_kernel[k]["ms"])
     dom_name = {"select": "semkv_assign_precision (k_select_cluster)",

@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(128) k_append(semkv_cache_t c, const uint16_t*
         __shared__ int cnt_s[4];
         const uint32_t* keys = c.score_keys + (size_t)u * c.T_cap;
         int cnt = 0;
+#pragma unroll 8
         for (int t = 4 * d; t < T; t += 4 * 128) {  // t + 3 < T_cap: T < T_cap, T_cap % 32 == 0
             const uint4 k4 = *reinterpret_cast<const uint4*>(keys + t);
             cnt += (k4.x >= key) + (t + 1 < T && k4.y >= key) + (t + 2 < T && k4.z >= key) + (t + 3 < T && k4.w >= key);
