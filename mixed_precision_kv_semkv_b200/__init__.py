@@ -6,6 +6,7 @@ binding (`_lib`, same function names as the C entry points), a torch-allocated c
 """
 from ._lib import (  # noqa: F401
     SemkvError,
+    semkv_append_decode,
     semkv_append_token,
     semkv_append_token_running,
     semkv_assign_precision,

@@ -29,7 +29,7 @@ SHAPE_FIELDS = ("B", "H", "Hq", "D", "G", "L_hi", "L_lo", "cap_hi", "cap_lo", "T
 BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
              "bitmap", "rank", "n_hi", "n_lo", "tau", "status", "slot_token", "score_keys")
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
-            "semkv_append_token", "semkv_append_token_running", "semkv_decode_attention",
+            "semkv_append_token", "semkv_append_token_running", "semkv_append_decode", "semkv_decode_attention",
             "semkv_decode_attention_noalloc", "semkv_dequantize", "semkv_status_string", "semkv_radix_digits",
             "semkv_p_for_ratio")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.semkv_quantize_pack.argtypes = [cp, vp, vp, i32, vp]
         L.semkv_append_token.argtypes = [cp, vp, vp, vp, vp]
         L.semkv_append_token_running.argtypes = [cp, vp, vp, vp, f32, vp]
+        L.semkv_append_decode.argtypes = [cp, vp, vp, vp, vp, f32, vp, vp, sz, vp]
         L.semkv_decode_attention.argtypes = [cp, vp, f32, vp, vp, sz, vp]
         L.semkv_decode_attention_noalloc.argtypes = [cp, vp, f32, vp, vp]
         L.semkv_dequantize.argtypes = [cp, vp, vp, i32, vp]
@@ -150,6 +151,17 @@ def semkv_append_token_running(cache, k, v, score, p: float, stream=None) -> int
     return _check("semkv_append_token_running",
                   lib().semkv_append_token_running(ctypes.byref(_struct(cache)), _ptr(k), _ptr(v), _ptr(score),
                                                    float(p), _stream(stream)))
+
+
+def semkv_append_decode(cache, k, v, score, q, softmax_scale: float, out, workspace,
+                        workspace_bytes: int | None = None, stream=None) -> int:
+    """append_token then decode_attention in one pass over the cache."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _check("semkv_append_decode",
+                  lib().semkv_append_decode(ctypes.byref(_struct(cache)), _ptr(k), _ptr(v), _ptr(score), _ptr(q),
+                                            float(softmax_scale), _ptr(out), _ptr(workspace), int(workspace_bytes),
+                                            _stream(stream)))
 
 
 def semkv_decode_attention(cache, q, softmax_scale: float, out, workspace, workspace_bytes: int | None = None,

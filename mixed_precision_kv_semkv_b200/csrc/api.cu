@@ -104,6 +104,43 @@ int launch_status()
 
 }  // namespace
 
+namespace {
+
+// decode, with an appended token first when app.k is set (both segments on the tensor-core kernel)
+static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_scale, float* out, void* workspace,
+                       size_t workspace_bytes, const AppendIn& app, cudaStream_t st)
+{
+    int r = validate(c);
+    if (r != SEMKV_OK) return r;
+    if (!q || !out || !std::isfinite(softmax_scale)) return SEMKV_ERR_INVALID_ARG;
+    if (((uintptr_t)q) & 15u) return SEMKV_ERR_INVALID_ARG;  // query rows are read 16 bytes at a time
+    size_t need = 0;
+    semkv_workspace_bytes(c, &need);
+    if (workspace_bytes < need || (need > 0 && !workspace)) return SEMKV_ERR_INVALID_ARG;
+    int nh, nl;
+    decode_splits(c, &nh, &nl);
+    const int units = c->B * c->H, g = c->Hq / c->H;
+    const float scale_log2 = softmax_scale * 1.4426950408889634f;
+    float* ws = static_cast<float*>(workspace);
+    bool dependent = false;
+    for (int hi = 1; hi >= 0; --hi) {
+        const SegView sv = seg_view(c, hi != 0);
+        const int ns = hi ? nh : nl, off = hi ? 0 : nh;
+        if (ns == 0) continue;
+        if (decode_tc_supported(sv.L, c->G, g)) {
+            launch_decode_tc(sv, q, units, c->H, g, c->G, scale_log2, ns, off, nh + nl, ws, c->status, dependent, app,
+                             st);
+        } else {
+            launch_decode_split(sv, q, units, c->H, g, c->D, c->G, scale_log2, ns, off, nh + nl, ws, st);
+        }
+        dependent = true;
+    }
+    launch_decode_merge(ws, units, c->H, g, c->D, nh + nl, out, app, st);
+    return launch_status();
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t semkv_radix_digits(int32_t L) { return level_ok(L) ? radix_k(L) : 0; }
@@ -207,36 +244,31 @@ int semkv_append_token_running(const semkv_cache_t* c, const uint16_t* k, const 
     return launch_status();
 }
 
+
 int semkv_decode_attention(const semkv_cache_t* c, const uint16_t* q, float softmax_scale, float* out,
                            void* workspace, size_t workspace_bytes, void* stream)
 {
+    const AppendIn none = {};
+    return decode_impl(c, q, softmax_scale, out, workspace, workspace_bytes, none, (cudaStream_t)stream);
+}
+
+int semkv_append_decode(const semkv_cache_t* c, const uint16_t* k, const uint16_t* v, const float* score,
+                        const uint16_t* q, float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                        void* stream)
+{
     int r = validate(c);
     if (r != SEMKV_OK) return r;
-    if (!q || !out || !std::isfinite(softmax_scale)) return SEMKV_ERR_INVALID_ARG;
-    if (((uintptr_t)q) & 15u) return SEMKV_ERR_INVALID_ARG;  // query rows are read 16 bytes at a time
-    size_t need = 0;
-    semkv_workspace_bytes(c, &need);
-    if (workspace_bytes < need || (need > 0 && !workspace)) return SEMKV_ERR_INVALID_ARG;
-    int nh, nl;
-    decode_splits(c, &nh, &nl);
-    const int units = c->B * c->H, g = c->Hq / c->H;
-    const float scale_log2 = softmax_scale * 1.4426950408889634f;
-    float* ws = static_cast<float*>(workspace);
-    cudaStream_t st = (cudaStream_t)stream;
-    bool dependent = false;
-    for (int hi = 1; hi >= 0; --hi) {
-        const SegView sv = seg_view(c, hi != 0);
-        const int ns = hi ? nh : nl, off = hi ? 0 : nh;
-        if (ns == 0) continue;
-        if (decode_tc_supported(sv.L, c->G, g)) {
-            launch_decode_tc(sv, q, units, c->H, g, c->G, scale_log2, ns, off, nh + nl, ws, c->status, dependent, st);
-        } else {
-            launch_decode_split(sv, q, units, c->H, g, c->D, c->G, scale_log2, ns, off, nh + nl, ws, st);
-        }
-        dependent = true;
+    if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
+    const int g = c->Hq / c->H;
+    if (!decode_tc_supported(c->L_hi, c->G, g) || !decode_tc_supported(c->L_lo, c->G, g)) {
+        // shapes the fused path does not cover: the two calls, in order
+        launch_append(*c, k, v, score, -1.0f, (cudaStream_t)stream);
+        r = launch_status();
+        if (r != SEMKV_OK) return r;
+        return semkv_decode_attention(c, q, softmax_scale, out, workspace, workspace_bytes, stream);
     }
-    launch_decode_merge(ws, units, c->H, g, c->D, nh + nl, out, st);
-    return launch_status();
+    const AppendIn app = {*c, k, v, score};
+    return decode_impl(c, q, softmax_scale, out, workspace, workspace_bytes, app, (cudaStream_t)stream);
 }
 
 int semkv_dequantize(const semkv_cache_t* c, float* K, float* V, int32_t T, void* stream)

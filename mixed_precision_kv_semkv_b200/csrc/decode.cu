@@ -13,6 +13,7 @@
 // sum_t p_h(t) s_V(t) (c_td - m), and the zero terms sum_t p_h(t) (z_V + m s_V) are summed per
 // (group, head).  Each CTA writes (m_h, l_h, o_h[D]) to the workspace; a second kernel merges the
 // splits with log-sum-exp weights.
+#include "append.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -220,13 +221,24 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
 constexpr int MERGE_CH = 32, MERGE_PARTS = 16;
 
 __global__ void __launch_bounds__(32 * MERGE_PARTS) k_decode_merge(const float* __restrict__ ws, int g,
-                                                                  int nsplit_total, float* __restrict__ out)
+                                                                  int nsplit_total, float* __restrict__ out,
+                                                                  semkv_cache_t cache,
+                                                                  const uint16_t* __restrict__ knew,
+                                                                  const float* __restrict__ snew)
 {
     constexpr int D = 128, NT = 32 * MERGE_PARTS;
     // launched as a programmatic dependent of the split kernels: wait for them (and their writes)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int u = blockIdx.x / g, h = blockIdx.x % g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (knew && h == 0 && blockIdx.y == 0 && tid == 0) {
+        // the appended token's bookkeeping: every decode CTA has read the counts by now
+        const float sc = snew[u];
+        const int nh = cache.n_hi[u], nl = cache.n_lo[u];
+        const bool hi = sc > cache.tau[u];
+        if (append_fits(cache, hi, nh, nl)) append_state(cache, u, hi, nh, nl, sc);
+        else atomicOr(cache.status, SEMKV_STATUS_APPEND_OVERFLOW | (isnan(sc) ? SEMKV_STATUS_NAN_SCORE : 0));
+    }
     const float* base = ws + (size_t)u * nsplit_total * g * (D + 2) + h * (D + 2);
     const size_t stride = (size_t)g * (D + 2);
     extern __shared__ float wts[];  // [nsplit_total]: the splits' maxima, then their weights
@@ -302,7 +314,7 @@ void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H
 }
 
 void launch_decode_merge(const float* ws, int units, int H, int g, int D, int nsplit_total, float* out,
-                         cudaStream_t st)
+                         const AppendIn& app, cudaStream_t st)
 {
     (void)H;
     (void)D;
@@ -316,7 +328,7 @@ void launch_decode_merge(const float* ws, int units, int H, int g, int D, int ns
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, k_decode_merge, ws, g, nsplit_total, out);
+    cudaLaunchKernelEx(&cfg, k_decode_merge, ws, g, nsplit_total, out, app.cache, app.k, app.score);
 }
 
 }  // namespace semkv

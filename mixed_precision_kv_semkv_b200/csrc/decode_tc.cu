@@ -26,6 +26,7 @@
 //            The zero terms sum_t p (z_V + m s_V) and the denominators stay on the CUDA cores.
 // Each CTA writes (max, sum, unnormalized o) per query head to the workspace; k_decode_merge
 // combines the splits.  Every mbarrier wait is bounded; a timeout sets SEMKV_STATUS_TIMEOUT.
+#include "append.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -87,7 +88,10 @@ template <int L, int GQ, int NG>
 __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_t* __restrict__ q, int H,
                                                        float scale_log2, int nsplit, int split_off, int nsplit_total,
                                                        float* __restrict__ ws, int32_t* __restrict__ status,
-                                                       int wait_for_prior)
+                                                       int wait_for_prior, semkv_cache_t cache,
+                                                       const uint16_t* __restrict__ knew,
+                                                       const uint16_t* __restrict__ vnew,
+                                                       const float* __restrict__ snew)
 {
     using C = Tc<L, GQ, NG>;
     constexpr int D = 128, W = C::W, NPAIR = C::NPAIR, KC = C::KC, KSTEPS = C::KSTEPS, KSLOTS = C::KSLOTS;
@@ -111,10 +115,30 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     __shared__ __align__(8) uint64_t mbar[4];                // 0: q.k done, 1: p.V done, 2/3: stage full
     __shared__ uint32_t tmem_base_s;
 
-    const int n = seg.n[u];
+    // append and attend in one pass (knew != nullptr): every CTA works out the new token's grid
+    // and its segment's new length from the inputs alone (the counts are updated by the merge,
+    // after every CTA has read them); the CTA whose tiles hold the new slot writes the row first
+    int n = seg.n[u];
+    int append_tile = -1;
+    bool app_hi = false;
+    int app_nh = 0, app_nl = 0;
+    if (knew) {
+        app_nh = cache.n_hi[u];
+        app_nl = cache.n_lo[u];
+        app_hi = snew[u] > cache.tau[u];  // NaN compares false: the token goes lo
+        if (append_fits(cache, app_hi, app_nh, app_nl) && app_hi == (seg.is_hi != 0)) append_tile = n++ / TILE;
+    }
     const int tiles = min(ceil_div(n, TILE), seg.tiles_cap);
     const int per = ceil_div(tiles, nsplit);
     const int t0 = split * per, t1 = min(tiles, t0 + per);
+    if (append_tile >= t0 && append_tile < t1) {
+        const bool bad = append_row(cache, u, app_hi, app_nh, app_nl, h2f(knew[(size_t)u * D + tid]),
+                                    h2f(vnew[(size_t)u * D + tid]));
+        if (bad && tid == 0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
+        // the row's words (plain stores and reductions) before this CTA's bulk copies read the tile
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncthreads();
+    }
 
     auto issue_fetch = [&](int tile, int stg) {  // one thread
         unsigned char* dst = stage0 + stg * C::STAGE_BYTES;
@@ -397,7 +421,8 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
 
 template <int L, int GQ, int NG>
 static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, float scale_log2, int nsplit,
-                      int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent, cudaStream_t st)
+                      int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
+                      const AppendIn& app, cudaStream_t st)
 {
     using C = Tc<L, GQ, NG>;
     // at most four CTAs per SM: each holds 128 of the SM's 512 TMEM columns
@@ -414,7 +439,7 @@ static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, f
     cfg.attrs = attr;
     cfg.numAttrs = dependent ? 1 : 0;
     cudaLaunchKernelEx(&cfg, k_decode_tc<L, GQ, NG>, seg, q, H, scale_log2, nsplit, split_off, nsplit_total, ws,
-                       status, dependent ? 1 : 0);
+                       status, dependent ? 1 : 0, app.cache, app.k, app.v, app.score);
 }
 
 // instantiated shapes: L in {4, 5, 6, 8, 16} x (g, groups) whose accumulators fit 128 TMEM columns
@@ -435,14 +460,14 @@ bool decode_tc_supported(int L, int G, int g)
 
 void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, int g, int G, float scale_log2,
                       int nsplit, int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
-                      cudaStream_t st)
+                      const AppendIn& app, cudaStream_t st)
 {
     if (nsplit == 0 || units == 0) return;
     const int ng = 128 / G;
 #define SEMKV_TC_GO(LL, GG, NN)                                                                                   \
     if (seg.L == LL && g == GG && ng == NN) {                                                                     \
         launch_tc<LL, GG, NN>(seg, q, units, H, scale_log2, nsplit, split_off, nsplit_total, ws, status, dependent, \
-                              st);                                                                                \
+                              app, st);                                                                           \
         return;                                                                                                   \
     }
     SEMKV_TC_LEVELS(SEMKV_TC_GO)

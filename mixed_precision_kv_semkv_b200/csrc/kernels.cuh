@@ -20,6 +20,14 @@ struct SegView {
     int is_hi;      // 1: L_hi segment (bitmap bit 1), 0: L_lo segment
 };
 
+// A generated token to append while decoding (k == nullptr: none); the fixed-threshold rule.
+struct AppendIn {
+    semkv_cache_t cache;
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* score;
+};
+
 // also writes slot_token [units][cap_hi + cap_lo]: the token index of every prefill slot
 void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
                    int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
@@ -36,8 +44,10 @@ void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v,
 // decode: split partials of one segment go to splits [split_off, split_off + nsplit) of each unit
 void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H, int g, int D, int G,
                          float scale_log2, int nsplit, int split_off, int nsplit_total, float* ws, cudaStream_t st);
+// with app.k != nullptr the merge also does the appended tokens' bookkeeping (counts, bitmap, rank,
+// score keys, status), once every decode CTA has read the counts
 void launch_decode_merge(const float* ws, int units, int H, int g, int D, int nsplit_total, float* out,
-                         cudaStream_t st);
+                         const AppendIn& app, cudaStream_t st);
 
 // tcgen05 decode (decode_tc.cu): supported for L in {2, 4..8, 10..16}, G >= 32, g <= 8.
 bool decode_tc_supported(int L, int G, int g);
@@ -45,7 +55,7 @@ bool decode_tc_supported(int L, int G, int g);
 // start while that kernel drains, and waits for it to complete before it exits).
 void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, int g, int G, float scale_log2,
                       int nsplit, int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
-                      cudaStream_t st);
+                      const AppendIn& app, cudaStream_t st);
 
 void launch_dequantize(const semkv_cache_t& c, int T, float* K, float* V, cudaStream_t st);
 
