@@ -64,22 +64,27 @@ def lib():
         L.oracle_scale_half.restype = _c.c_uint16
         L.oracle_n_hi.argtypes = [_c.c_float, _c.c_int32]
         L.oracle_n_hi.restype = _c.c_int32
-        L.oracle_select.argtypes = [_f32p, _c.c_int32, _c.c_float, _u32p, _u32p,
+        L.oracle_select.argtypes = [_f32p, _c.c_int32, _c.c_float, _c.c_int32, _u32p, _u32p,
                                     _c.POINTER(_c.c_int32), _c.POINTER(_c.c_float)]
         L.oracle_select.restype = _c.c_int
         L.oracle_quantize_group.argtypes = [_u16p, _c.c_int, _c.c_int, _u8p,
                                             _c.POINTER(_c.c_uint16), _c.POINTER(_c.c_uint16)]
         L.oracle_quantize_group.restype = _c.c_int
+        L.oracle_quantize_group_clip.argtypes = [_u16p, _c.c_int, _c.c_int, _c.c_float, _u8p,
+                                                 _c.POINTER(_c.c_uint16), _c.POINTER(_c.c_uint16)]
+        L.oracle_quantize_group_clip.restype = _c.c_int
+        L.oracle_float_to_half_rn.argtypes = [_c.c_float]
+        L.oracle_float_to_half_rn.restype = _c.c_uint16
         L.oracle_pack_word.argtypes = [_u8p, _c.c_int, _c.c_int]
         L.oracle_pack_word.restype = _c.c_uint32
         L.oracle_unpack_word.argtypes = [_c.c_uint32, _c.c_int, _c.c_int, _u8p]
         L.oracle_quantize_pack_unit.argtypes = [_u16p, _u16p, _c.c_int32, _c.c_int, _c.c_int, _c.c_int,
-                                                _c.c_int, _u32p, _c.c_int, _c.c_int] + [_u32p] * 8
+                                                _c.c_int, _c.c_float, _u32p, _c.c_int, _c.c_int] + [_u32p] * 8
         L.oracle_quantize_pack_unit.restype = _c.c_int
         L.oracle_dequantize_unit.argtypes = [_c.c_int32, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _u32p] + \
             [_u32p] * 8 + [_f32p, _f32p]
         L.oracle_append_unit.argtypes = [_u16p, _u16p, _c.c_float, _c.c_float, _c.c_int, _c.c_int, _c.c_int,
-                                         _c.c_int, _c.c_int32, _u32p, _u32p, _c.POINTER(_c.c_int32),
+                                         _c.c_int, _c.c_float, _c.c_int32, _u32p, _u32p, _c.POINTER(_c.c_int32),
                                          _c.POINTER(_c.c_int32), _c.c_int, _c.c_int] + [_u32p] * 8
         L.oracle_append_unit.restype = _c.c_int
         L.oracle_attention_fp64.argtypes = [_u16p, _c.c_int, _f32p, _f32p, _c.c_int32, _c.c_int, _c.c_float,
@@ -121,6 +126,11 @@ def float_to_half_up(f) -> np.ndarray:
     return out
 
 
+def half_rn(f: float) -> int:
+    """binary16 bits nearest to the fp32 value f (ties to even)."""
+    return int(lib().oracle_float_to_half_rn(float(f)))
+
+
 def scale_half(sf: float) -> int:
     return int(lib().oracle_scale_half(float(sf)))
 
@@ -129,8 +139,9 @@ def n_hi(p: float, T: int) -> int:
     return int(lib().oracle_n_hi(float(p), int(T)))
 
 
-def select(score, p: float):
-    """Precision assignment of one unit. Returns (bitmap, rank, n_hi, tau, status)."""
+def select(score, p: float, window: int = 0):
+    """Precision assignment of one unit (window: the last `window` tokens also go to the finer
+    grid). Returns (bitmap, rank, n_hi, tau, status)."""
     score = np.ascontiguousarray(score, dtype=np.float32)
     T = score.shape[0]
     nw = max((T + 31) // 32, 1)
@@ -138,18 +149,19 @@ def select(score, p: float):
     rank = np.zeros(nw, np.uint32)
     nh = _c.c_int32(0)
     tau = _c.c_float(0)
-    st = lib().oracle_select(score, T, float(p), bitmap, rank, _c.byref(nh), _c.byref(tau))
+    st = lib().oracle_select(score, T, float(p), int(window), bitmap, rank, _c.byref(nh), _c.byref(tau))
     nwt = (T + 31) // 32
     return bitmap[:nwt], rank[:nwt], nh.value, np.float32(tau.value), st
 
 
-def quantize_group(x16, L: int):
-    """Quantize one group of fp16 bit patterns. Returns (codes uint8, scale16, zero16, status)."""
+def quantize_group(x16, L: int, clip: float = 1.0):
+    """Quantize one group of fp16 bit patterns (clip in (0, 1]: the clipped-range variant).
+    Returns (codes uint8, scale16, zero16, status)."""
     x16 = np.ascontiguousarray(x16, dtype=np.uint16)
     codes = np.zeros(x16.shape[0], np.uint8)
     s = _c.c_uint16(0)
     z = _c.c_uint16(0)
-    st = lib().oracle_quantize_group(x16, x16.shape[0], L, codes, _c.byref(s), _c.byref(z))
+    st = lib().oracle_quantize_group_clip(x16, x16.shape[0], L, float(clip), codes, _c.byref(s), _c.byref(z))
     return codes, s.value, z.value, st
 
 
@@ -183,7 +195,8 @@ def _seg_args(hi, lo):
             lo["k"].ravel(), lo["v"].ravel(), lo["kz"].ravel(), lo["vz"].ravel()]
 
 
-def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi: int, tiles_lo: int):
+def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi: int, tiles_lo: int,
+                       clip: float = 1.0):
     """Quantize and place one unit. K16, V16: [T][D] uint16. Returns (hi, lo, status)."""
     K16 = np.ascontiguousarray(K16, dtype=np.uint16)
     V16 = np.ascontiguousarray(V16, dtype=np.uint16)
@@ -192,7 +205,8 @@ def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi:
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
     n = min(len(bitmap), len(bm))
     bm[:n] = bitmap[:n]
-    st = lib().oracle_quantize_pack_unit(K16.ravel(), V16.ravel(), T, D, G, L_hi, L_lo, bm, tiles_hi, tiles_lo,
+    st = lib().oracle_quantize_pack_unit(K16.ravel(), V16.ravel(), T, D, G, L_hi, L_lo, float(clip), bm, tiles_hi,
+                                         tiles_lo,
                                          *_seg_args(hi, lo))
     return hi, lo, st
 
@@ -225,14 +239,15 @@ class UnitState:
         self.lo = lo
 
 
-def append_unit(state: UnitState, k16, v16, score: float, G: int, L_hi: int, L_lo: int) -> int:
-    """Append one token to a unit in place. Returns status bits."""
+def append_unit(state: UnitState, k16, v16, score: float, G: int, L_hi: int, L_lo: int, clip: float = 1.0) -> int:
+    """Append one token to a unit in place (clip: as in quantize_group). Returns status bits."""
     k16 = np.ascontiguousarray(k16, dtype=np.uint16)
     v16 = np.ascontiguousarray(v16, dtype=np.uint16)
     D = k16.shape[0]
     nh = _c.c_int32(state.n_hi)
     nl = _c.c_int32(state.n_lo)
-    st = lib().oracle_append_unit(k16, v16, float(score), float(state.tau), D, G, L_hi, L_lo, state.T_cap,
+    st = lib().oracle_append_unit(k16, v16, float(score), float(state.tau), D, G, L_hi, L_lo, float(clip),
+                                  state.T_cap,
                                   state.bitmap, state.rank, _c.byref(nh), _c.byref(nl),
                                   state.hi["k"].shape[0], state.lo["k"].shape[0], *_seg_args(state.hi, state.lo))
     state.n_hi = nh.value
@@ -266,13 +281,13 @@ def running_is_hi(scores_prev, score_new: float, p: float) -> bool:
 
 
 def append_unit_running(state: UnitState, k16, v16, score: float, p: float, scores_prev, G: int, L_hi: int,
-                        L_lo: int) -> int:
+                        L_lo: int, clip: float = 1.0) -> int:
     """append_unit with the running top-p rule: the grid comes from running_is_hi (the fixed tau
     of the state is left as it was)."""
     tau = state.tau
     state.tau = np.float32(-np.inf) if running_is_hi(scores_prev, score, p) else np.float32(np.inf)
     try:
-        return append_unit(state, k16, v16, score, G, L_hi, L_lo)
+        return append_unit(state, k16, v16, score, G, L_hi, L_lo, clip)
     finally:
         state.tau = tau
 

@@ -38,6 +38,11 @@
  *               quantization at generation time too) is hi iff its score > tau of its unit
  *               (strict) [reading]; it is quantized alone and placed at the next slot.
  *   dequantize  x^ = fmaf((float)c, s, z).
+ *   variants    two quantizer variants of prior art that the pages summarise (the SKVQ abstract):
+ *               a clip ratio that shrinks each group's range before the grid is fitted, and a
+ *               window of the most recent tokens forced onto the finer grid at selection.  Both
+ *               are off by default; the formulas are readings, given at oracle_quantize_group_clip
+ *               and oracle_select.
  *   attention   fp64: o = sum_t softmax_t(sigma * q.k^_t) v^_t over all tokens of the unit, for
  *               each of the g query heads that share the kv head (GQA); no mask.
  *
@@ -129,6 +134,28 @@ uint16_t oracle_float_to_half_up(float f)
     return encode_half(neg, k * ulp);
 }
 
+/* binary32 -> binary16 rounded to nearest, ties to the even significand (IEEE 754 default
+ * rounding).  Only finite |f| <= 65504 is asked of it here (the clipped zero); larger magnitudes
+ * give infinity, NaN gives the quiet NaN. */
+uint16_t oracle_float_to_half_rn(float f)
+{
+    if (isnan(f)) return 0x7E00;
+    if (f == 0.0f) return signbit(f) ? 0x8000 : 0x0000;
+    int neg = f < 0.0f;
+    double a = fabs((double)f);
+    if (a >= 65520.0) return neg ? 0xFC00 : 0x7C00; /* halfway to 2^16 and beyond: infinity */
+    int e;
+    frexp(a, &e);
+    int E = e - 1; /* a in [2^E, 2^(E+1)) */
+    if (E < -14) E = -14;
+    double ulp = ldexp(1.0, E - 10);
+    double n = a / ulp; /* exact */
+    double k = floor(n);
+    double rem = n - k;
+    if (rem > 0.5 || (rem == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0; /* nearest; a tie goes to even */
+    return encode_half(neg, k * ulp);
+}
+
 /* the fp16 scale of a group: rounded up, saturated at the largest finite binary16 [reading] */
 uint16_t oracle_scale_half(float sf)
 {
@@ -159,11 +186,16 @@ int32_t oracle_n_hi(float p, int32_t T) { return (int32_t)floor((double)p * (dou
  * Order the T scores of one unit and assign the two precisions (SemKV page, Abstract: tokens
  * are ordered by a model-internal score and split between two neighbouring precisions).
  * Writes bitmap[0..ceil(T/32)) and rank[0..ceil(T/32)).  Returns status bits.
+ *
+ * window (prior-art variant, the SKVQ abstract on the same pages: the most recent tokens are
+ * kept at high precision) [reading]: after the selection by score, the last min(window, T)
+ * tokens are put on the finer grid too; n_hi is then the number of tokens on it.  tau stays the
+ * score threshold of the selection by score.  window = 0 is the plain method.
  */
-int oracle_select(const float* score, int32_t T, float p, uint32_t* bitmap, uint32_t* rank,
+int oracle_select(const float* score, int32_t T, float p, int32_t window, uint32_t* bitmap, uint32_t* rank,
                   int32_t* n_hi_out, float* tau_out)
 {
-    if (T < 0 || !(p >= 0.0f && p <= 1.0f)) return OR_BAD_ARG;
+    if (T < 0 || !(p >= 0.0f && p <= 1.0f) || window < 0) return OR_BAD_ARG;
     int status = 0;
     int32_t nw = (T + 31) / 32;
     scored_t* v = (scored_t*)malloc(sizeof(scored_t) * (size_t)(T > 0 ? T : 1));
@@ -176,6 +208,7 @@ int oracle_select(const float* score, int32_t T, float p, uint32_t* bitmap, uint
     int32_t n_hi = oracle_n_hi(p, T);
     memset(bitmap, 0, sizeof(uint32_t) * (size_t)nw);
     for (int32_t i = 0; i < n_hi; i++) bitmap[v[i].t / 32] |= 1u << (v[i].t % 32);
+    for (int32_t t = (window < T ? T - window : 0); t < T; t++) bitmap[t / 32] |= 1u << (t % 32);
     uint32_t acc = 0;
     for (int32_t w = 0; w < nw; w++) {
         rank[w] = acc;
@@ -185,7 +218,7 @@ int oracle_select(const float* score, int32_t T, float p, uint32_t* bitmap, uint
             acc++;
         }
     }
-    *n_hi_out = n_hi;
+    *n_hi_out = (int32_t)acc; /* = n_hi when window = 0 */
     /* -0 and +0 are the same score; the threshold is stored as +0 */
     *tau_out = n_hi > 0 ? v[n_hi - 1].s + 0.0f : INFINITY;
     free(v);
@@ -198,9 +231,16 @@ int oracle_select(const float* score, int32_t T, float p, uint32_t* bitmap, uint
  * Affine quantization of one group of G fp16 values to L levels (SemKV page, Abstract: a uniform
  * affine grid whose level count need not be a power of two).  Writes G codes, the fp16 scale and
  * the fp16 zero.
+ *
+ * clip (prior-art variant, the SKVQ abstract on the same pages: clipped dynamic quantization of
+ * each group): clip = 1 is the plain grid over [mn, mx].  For 0 < clip < 1 [reading -- the pages
+ * give neither the formula nor a value]: the extrema are first scaled by clip in fp32
+ * (mn' = clip*mn, mx' = clip*mx); z = the binary16 nearest to mn' (ties to even, -0 stored as
+ * +0); s = fp16 rounded up of (mx' - z)/(L - 1), taken as 0 if that is negative; values outside
+ * the clipped range get the end codes through the clamp below.
  */
-int oracle_quantize_group(const uint16_t* x, int G, int L, uint8_t* code, uint16_t* scale_out,
-                          uint16_t* zero_out)
+int oracle_quantize_group_clip(const uint16_t* x, int G, int L, float clip, uint8_t* code, uint16_t* scale_out,
+                               uint16_t* zero_out)
 {
     int status = 0;
     float mn = INFINITY, mx = -INFINITY;
@@ -210,11 +250,22 @@ int oracle_quantize_group(const uint16_t* x, int G, int L, uint8_t* code, uint16
         if (v < mn) mn = v;
         if (v > mx) mx = v;
     }
-    float sf = (mx - mn) / (float)(L - 1);
-    uint16_t s16 = oracle_scale_half(sf);
+    uint16_t s16, z16;
+    if (clip == 1.0f) {
+        float sf = (mx - mn) / (float)(L - 1);
+        s16 = oracle_scale_half(sf);
+        float z0 = mn + 0.0f;                   /* -0 becomes +0: one zero for both signs */
+        z16 = oracle_float_to_half_up(z0);      /* exact: mn is a binary16 value */
+    } else {
+        float mnc = clip * mn, mxc = clip * mx; /* one fp32 multiply each */
+        z16 = oracle_float_to_half_rn(mnc);
+        if (z16 == 0x8000) z16 = 0x0000;        /* -0 becomes +0 */
+        float sf = (mxc - oracle_half_to_float(z16)) / (float)(L - 1);
+        if (sf < 0.0f) sf = 0.0f;               /* mn == mx and z rounded above clip*mx */
+        s16 = oracle_scale_half(sf);
+    }
     float s = oracle_half_to_float(s16);
-    float z = mn + 0.0f; /* -0 becomes +0: one zero for both signs */
-    uint16_t z16 = oracle_float_to_half_up(z); /* exact: mn is a binary16 value */
+    float z = oracle_half_to_float(z16);
     for (int i = 0; i < G; i++) {
         float v = oracle_half_to_float(x[i]);
         int c = 0;
@@ -230,6 +281,12 @@ int oracle_quantize_group(const uint16_t* x, int G, int L, uint8_t* code, uint16
     *scale_out = s16;
     *zero_out = z16;
     return status;
+}
+
+int oracle_quantize_group(const uint16_t* x, int G, int L, uint8_t* code, uint16_t* scale_out,
+                          uint16_t* zero_out)
+{
+    return oracle_quantize_group_clip(x, G, L, 1.0f, code, scale_out, zero_out);
 }
 
 /* word = sum_i c_i L^i over k codes (base-L positional notation, lowest index least significant) */
@@ -297,11 +354,12 @@ static void pack_segment(const uint8_t* ck, const uint8_t* cv, int tiles, int D,
  * Segment buffers must hold tiles_hi (tiles_lo) tiles; slots past n_seg are written as zeros.
  */
 int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, int D, int G, int L_hi,
-                              int L_lo, const uint32_t* bitmap, int tiles_hi, int tiles_lo,
+                              int L_lo, float clip, const uint32_t* bitmap, int tiles_hi, int tiles_lo,
                               uint32_t* k_hi, uint32_t* v_hi, uint32_t* kz_hi, uint32_t* vz_hi,
                               uint32_t* k_lo, uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo)
 {
-    if (D <= 0 || G <= 0 || D % G != 0 || L_hi < 2 || L_lo < 2 || L_hi > 256 || L_lo > 256)
+    if (D <= 0 || G <= 0 || D % G != 0 || L_hi < 2 || L_lo < 2 || L_hi > 256 || L_lo > 256 ||
+        !(clip > 0.0f && clip <= 1.0f))
         return OR_BAD_ARG;
     int status = 0, NG = D / G;
     int tiles[2] = {tiles_hi, tiles_lo};
@@ -330,11 +388,11 @@ int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, i
         int tile = slot / OR_TILE, tt = slot % OR_TILE;
         for (int grp = 0; grp < NG; grp++) {
             uint16_t s16, z16;
-            status |= oracle_quantize_group(K + (size_t)t * D + grp * G, G, Ls[seg],
-                                            ck[seg] + (size_t)slot * D + grp * G, &s16, &z16);
+            status |= oracle_quantize_group_clip(K + (size_t)t * D + grp * G, G, Ls[seg], clip,
+                                                 ck[seg] + (size_t)slot * D + grp * G, &s16, &z16);
             kz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
-            status |= oracle_quantize_group(V + (size_t)t * D + grp * G, G, Ls[seg],
-                                            cv[seg] + (size_t)slot * D + grp * G, &s16, &z16);
+            status |= oracle_quantize_group_clip(V + (size_t)t * D + grp * G, G, Ls[seg], clip,
+                                                 cv[seg] + (size_t)slot * D + grp * G, &s16, &z16);
             vz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
         }
     }
@@ -408,12 +466,12 @@ void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, const u
 /*
  * Quantization at generation time of one new token of one unit (SemKV page, Abstract: the same
  * cliff is reported when tokens are quantized as they are generated).  hi iff score > tau
- * [reading].  The token is
- * quantized alone and written at the next slot of its segment; older tokens are untouched.
+ * [reading].  The token is quantized alone (with the prefill's clip) and written at the next
+ * slot of its segment; older tokens are untouched.
  * State (bitmap, rank, n_hi, n_lo) is updated in place.  Returns status bits.
  */
 int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float tau, int D, int G,
-                       int L_hi, int L_lo, int32_t T_cap, uint32_t* bitmap, uint32_t* rank,
+                       int L_hi, int L_lo, float clip, int32_t T_cap, uint32_t* bitmap, uint32_t* rank,
                        int32_t* n_hi, int32_t* n_lo, int tiles_hi, int tiles_lo, uint32_t* k_hi,
                        uint32_t* v_hi, uint32_t* kz_hi, uint32_t* vz_hi, uint32_t* k_lo,
                        uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo)
@@ -441,9 +499,9 @@ int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float 
     int tile = slot / OR_TILE, tt = slot % OR_TILE;
     for (int grp = 0; grp < NG; grp++) {
         uint16_t s16, z16;
-        status |= oracle_quantize_group(k + grp * G, G, L, kc + grp * G, &s16, &z16);
+        status |= oracle_quantize_group_clip(k + grp * G, G, L, clip, kc + grp * G, &s16, &z16);
         kz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
-        status |= oracle_quantize_group(v + grp * G, G, L, vc + grp * G, &s16, &z16);
+        status |= oracle_quantize_group_clip(v + grp * G, G, L, clip, vc + grp * G, &s16, &z16);
         vz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
     }
     for (int j = 0; j < WK; j++) kw[k_word_index(tile, j, tt, WK)] = oracle_pack_word(kc + j * kdig, kdig, L);
