@@ -57,9 +57,11 @@ def radix_words(L: int, n: int = 128) -> int:
     return -(-n // k)
 
 
-# this library's kernel launches in one step: select 1, quantize 1, append 1, decode 3 (hi and lo
-# segments, merge); the committed ncu launch list of the step shows the same kernels
-LAUNCHES_PER_STEP = 6
+# this library's kernel launches in one step: select 1, quantize 1, append+decode 3 (the hi and lo
+# segments, then the merge); the committed ncu launch list of the step shows the same kernels
+LAUNCHES_PER_STEP = 5
+# the quantizer variants timed beside the step (recent window of the selection; clipped range)
+WINDOW, CLIP = 128, 0.9
 
 
 def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False) -> dict:
@@ -243,9 +245,9 @@ def run_reference(args):
 def run_semkv(args):
     import torch
 
-    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_append_token, semkv_append_token_running,
-                                               semkv_assign_precision, semkv_decode_attention, semkv_quantize_pack,
-                                               synth)
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_append_decode, semkv_append_token,
+                                               semkv_append_token_running, semkv_assign_precision,
+                                               semkv_decode_attention, semkv_quantize_pack, synth)
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
@@ -265,9 +267,10 @@ def run_semkv(args):
     # one generated token per unit: its k, v rows and score (appended after the prefill every step)
     gen = synth.gen_steps_gpu(w, K, seed=rank_seed(rank), layer=0, steps=1)
     kn, vn, sn = (gen[x][0].contiguous() for x in ("k", "v", "scores"))
-    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=1)
+    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=1, window=WINDOW)
     ws = cache.workspace()
-    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")  # the step's attention output
+    out_s = torch.empty_like(out)  # the same, from the separate append and decode calls
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
     scale = synth.sm_scale(w.D)
     from mixed_precision_kv_semkv_b200.cache import n_hi_for
@@ -279,7 +282,7 @@ def run_semkv(args):
     calls = [lambda: semkv_assign_precision(cache, S, T, w.p),
              lambda: semkv_quantize_pack(cache, K, V, T),
              lambda: semkv_append_token(cache, kn, vn, sn),
-             lambda: semkv_decode_attention(cache, q, scale, out, ws)]
+             lambda: semkv_decode_attention(cache, q, scale, out_s, ws)]
     names = ("select", "quantize", "append", "decode_in_step")
     for c in calls:  # eager once: module loading and kernel attributes happen outside capture
         c()
@@ -288,12 +291,19 @@ def run_semkv(args):
     n_hi0 = n_hi_for(w.p, T)
     new_hi = int((cache.bufs["n_hi"] - n_hi0).sum().item())
     nb = alg_bytes(w, T, n_hi0, new_hi, appended=True)
-    step_bytes = nb["select"] + nb["quantize"] + nb["append"] + nb["decode"]
+    step_bytes = nb["select"] + nb["quantize"] + nb["append"] + nb["decode"]  # the three calls below do this
     # the step as one CUDA graph (as a serving loop would capture it): the timed `value`; and each
     # call in a graph of its own: the per-call split (each then also pays its own graph launch)
+    fused_call = lambda: semkv_append_decode(cache, kn, vn, sn, q, scale, out, ws)  # noqa: E731
+    step_calls = (calls[0], calls[1], fused_call)
+    calls[0]()  # a fresh prefill first: the cache holds room for one appended token
+    calls[1]()
+    fused_call()
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_s), "append+decode in one pass differs from append then decode"
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph, capture_error_mode="relaxed"):
-        for c in calls:
+        for c in step_calls:
             c()
     graphs = []
     for c in calls:
@@ -310,6 +320,10 @@ def run_semkv(args):
     run_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(run_graph, capture_error_mode="relaxed"):
         run_call()
+    # append + decode in one pass (the step's last call) on its own, likewise after a fresh prefill
+    fused_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(fused_graph, capture_error_mode="relaxed"):
+        fused_call()
 
     def step(ev=None):
         if ev is not None:
@@ -358,19 +372,60 @@ def run_semkv(args):
         step_split(evs_split[i])
     torch.cuda.synchronize()
     t_call = [sum(e[i].elapsed_time(e[i + 1]) for e in evs_split) * steps / split_steps for i in range(len(graphs))]
-    # running append: after a fresh prefill (select + quantize replayed untimed), its own graph
-    t_run = 0.0
-    for i in range(split_steps):
-        flush.zero_()
-        graphs[0].replay()
-        graphs[1].replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        run_graph.replay()
-        e1.record(stream)
-        e1.synchronize()
-        t_run += e0.elapsed_time(e1)
-    t_run /= split_steps
+    # running append and fused append+decode: each after a fresh prefill (select + quantize
+    # replayed untimed), from a graph of its own
+    def after_prefill(gr):
+        t = 0.0
+        for i in range(split_steps):
+            flush.zero_()
+            graphs[0].replay()
+            graphs[1].replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            e1.synchronize()
+            t += e0.elapsed_time(e1)
+        return t / split_steps
+
+    t_run = after_prefill(run_graph)
+    t_fused = after_prefill(fused_graph)
+    # the quantizer variants on the same workload, each call in a graph of its own: the selection
+    # with a recent window of WINDOW tokens, the quantization with a clipped range (clip CLIP,
+    # which runs the generic quantize kernel)
+    cache.struct.window = WINDOW
+    win_graph = torch.cuda.CUDAGraph()
+    calls[0]()
+    with torch.cuda.graph(win_graph, capture_error_mode="relaxed"):
+        calls[0]()
+    cache.struct.window = 0
+    calls[0]()
+    cache.struct.clip = CLIP
+    clip_graph = torch.cuda.CUDAGraph()
+    calls[1]()
+    with torch.cuda.graph(clip_graph, capture_error_mode="relaxed"):
+        calls[1]()
+    cache.struct.clip = 0.0
+    torch.cuda.synchronize()
+
+    def timed(gr, before=()):
+        t = 0.0
+        for i in range(split_steps):
+            flush.zero_()
+            for b in before:
+                b.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            e1.synchronize()
+            t += e0.elapsed_time(e1)
+        return t / split_steps
+
+    t_win = timed(win_graph)
+    t_clip = timed(clip_graph, before=(graphs[0],))
+    assert cache.status() == 0, f"device status {cache.status()}"
+    assert torch.equal(out, out_s), "append+decode in one pass differs from append then decode"
     # leave the cache as a timed step leaves it (prefill + the fixed-threshold append)
     for gr in graphs[:3]:
         gr.replay()
@@ -402,11 +457,14 @@ def run_semkv(args):
     per_kernel.update({
         "decode_l2_cold": {"ms": dec_cold, "gbs": nb["decode"] / (dec_cold * 1e-3) / 1e9},
         "append_running": {"ms": t_run, "gbs": nb["append_running"] / (t_run * 1e-3) / 1e9},
+        "append_decode": {"ms": t_fused, "gbs": (nb["append"] + nb["decode"]) / (t_fused * 1e-3) / 1e9},
+        f"select_window{WINDOW}": {"ms": t_win, "gbs": nb["select"] / (t_win * 1e-3) / 1e9},
+        f"quantize_clip{CLIP}": {"ms": t_clip, "gbs": nb["quantize"] / (t_clip * 1e-3) / 1e9},
     })
-    dom = max(("select", "quantize", "decode_in_step"), key=lambda k: per_kernel[k]["ms"])
+    dom = max(("select", "quantize", "append_decode"), key=lambda k: per_kernel[k]["ms"])
     dom_name = {"select": "semkv_assign_precision (k_select_cluster)",
                 "quantize": "semkv_quantize_pack (k_quantize_fast)",
-                "decode_in_step": "semkv_decode_attention (k_decode_tc x 2 + k_decode_merge)"}[dom]
+                "append_decode": "semkv_append_decode (k_decode_tc x 2 + k_decode_merge)"}[dom]
     ach = per_kernel[dom]["gbs"]
     traffic = None  # DRAM bytes per launch from the committed ncu capture, if the kernel is unchanged since
     try:
@@ -461,10 +519,11 @@ def run_semkv(args):
         "config": {"workload": f"{w.name}: Llama-3.1-8B-shaped layer, B{w.B} H{w.H} Hq{w.Hq} T{T} D{w.D}, "
                                f"G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}",
                    "l2": "flushed between steps (512 MB write)", "parallelism": f"dp{world} (independent units)",
-                   "timing": "step = one CUDA graph of the four calls; per_kernel = each call replayed from a graph "
-                             "of its own (so each also pays a graph launch)",
-                   "step": "assign_precision + quantize_pack + append_token (one generated token per unit) + "
-                           "decode_attention"},
+                   "timing": "step = one CUDA graph of its three calls; per_kernel = each call (and the separate "
+                             "append_token and decode_attention) replayed from a graph of its own (so each also pays "
+                             "a graph launch)",
+                   "step": "assign_precision + quantize_pack + append_decode (append_token of one generated token "
+                           "per unit and decode_attention in one pass)"},
         "per_kernel": per_kernel,
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                      "frac": ach / hbm_peak, "peak_kind": peak_note, "traffic": traffic,

@@ -93,6 +93,17 @@ typedef struct semkv_cache {
     int32_t L_hi, L_lo;     /* level counts of the two grids (L_hi is used for the top fraction p) */
     int32_t cap_hi, cap_lo; /* slot capacity of each segment per unit, multiples of 128 */
     int32_t T_cap;          /* token capacity per unit (bitmap/rank length), multiple of 32 */
+    /* Quantizer variants of prior art (the SKVQ abstract on the same pages); zero-initialised
+     * fields give the plain method.
+     *   window: semkv_assign_precision also puts the last min(window, T) tokens of each unit on
+     *           the L_hi grid (recent tokens at high precision); >= 0.
+     *   clip:   0 or 1 = the plain min/max grid.  In (0, 1): each group's min and max are first
+     *           scaled by clip in fp32 (clipped range), the zero is the nearest binary16 of the
+     *           scaled min (-0 stored as +0), the scale is fp16 rounded up of
+     *           (clip*max - zero)/(L - 1) (at least 0); values outside take the end codes.  Used by
+     *           semkv_quantize_pack and every append.  Other values: SEMKV_ERR_INVALID_ARG. */
+    int32_t window;
+    float clip;
     uint32_t *k_hi, *v_hi, *kz_hi, *vz_hi;
     uint32_t *k_lo, *v_lo, *kz_lo, *vz_lo;
     uint32_t *bitmap, *rank;
@@ -120,12 +131,13 @@ SEMKV_API int semkv_workspace_bytes(const semkv_cache_t* shape, size_t* bytes);
 
 /* Precision assignment (SemKV page, Abstract: tokens ranked by an internal score; the top fraction
  * gets the finer of two neighbouring grids).  scores: device fp32 [B][H][T].  For every unit:
- * n_hi = floor(p*T) (p in [0,1], computed in double); the n_hi tokens with the largest scores
- * (equal scores: lower token index first; -0 == +0) get bit 1 in the bitmap; rank[] and
- * slot_token[] are filled;
- * n_lo = T - n_hi; tau = the n_hi-th largest score (+inf if n_hi = 0).  Requires T <= T_cap,
- * n_hi <= cap_hi and T - n_hi <= cap_lo (else SEMKV_ERR_CAPACITY).  NaN scores set
- * SEMKV_STATUS_NAN_SCORE.  Bitmap words past the last token are cleared. */
+ * n_sel = floor(p*T) (p in [0,1], computed in double); the n_sel tokens with the largest scores
+ * (equal scores: lower token index first; -0 == +0) get bit 1 in the bitmap, and so do the last
+ * min(window, T) tokens; n_hi = the number of 1 bits (n_sel when window = 0); rank[] and
+ * slot_token[] are filled; n_lo = T - n_hi; tau = the n_sel-th largest score (+inf if
+ * n_sel = 0).  Requires T <= T_cap, n_sel + min(window, T) <= cap_hi and T - n_sel <= cap_lo
+ * (else SEMKV_ERR_CAPACITY).  NaN scores set SEMKV_STATUS_NAN_SCORE.  Bitmap words past the last
+ * token are cleared. */
 SEMKV_API int semkv_assign_precision(const semkv_cache_t* cache, const float* scores, int32_t T, float p,
                            void* stream);
 
@@ -134,7 +146,8 @@ SEMKV_API int semkv_assign_precision(const semkv_cache_t* cache, const float* sc
  * semkv_assign_precision must have run for this T.  Per token and group of G channels:
  * mn, mx = min, max; s = fp16 rounded up of fp32 (mx - mn)/(L - 1) (saturated at 65504);
  * z = mn; code = clamp(rint((x - z)/s), 0, L - 1) (fp32 subtract and divide, ties to even; 0 if
- * s = 0).  K and V must be 16-byte aligned (rows are fetched with bulk copies).  Codes are packed and placed as described at the top of this file; slots past the
+ * s = 0).  With the clip variant set in the cache, s and z are those of the clipped range (see
+ * semkv_cache_t).  K and V must be 16-byte aligned (rows are fetched with bulk copies).  Codes are packed and placed as described at the top of this file; slots past the
  * segment's length inside its last tile get zero codes and zero scale/zero.  Non-finite inputs
  * set SEMKV_STATUS_NONFINITE_KV. */
 SEMKV_API int semkv_quantize_pack(const semkv_cache_t* cache, const uint16_t* K, const uint16_t* V, int32_t T,

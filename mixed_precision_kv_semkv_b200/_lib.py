@@ -36,8 +36,9 @@ NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
 class CacheStruct(ctypes.Structure):
-    """Mirror of semkv_cache_t."""
-    _fields_ = [(n, ctypes.c_int32) for n in SHAPE_FIELDS] + [(n, ctypes.c_void_p) for n in BUF_NAMES]
+    """Mirror of semkv_cache_t (window, clip: the quantizer variants; 0 = off)."""
+    _fields_ = [(n, ctypes.c_int32) for n in SHAPE_FIELDS] + [("window", ctypes.c_int32), ("clip", ctypes.c_float)] + \
+        [(n, ctypes.c_void_p) for n in BUF_NAMES]
 
 
 class SemkvError(RuntimeError):

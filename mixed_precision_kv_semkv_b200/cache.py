@@ -21,21 +21,24 @@ def round_up(x: int, m: int) -> int:
     return (x + m - 1) // m * m
 
 
-def capacities(T: int, p: float, extra: int = 0):
-    """(cap_hi, cap_lo, T_cap) for a prefill of T tokens at fraction p plus `extra` appends."""
+def capacities(T: int, p: float, extra: int = 0, window: int = 0):
+    """(cap_hi, cap_lo, T_cap) for a prefill of T tokens at fraction p (plus a recent window of
+    `window` tokens on the finer grid) and `extra` appends."""
     nh = n_hi_for(p, T)
-    return round_up(nh + extra, 128), round_up(T - nh + extra, 128), round_up(T + extra, 32)
+    return round_up(nh + min(window, T) + extra, 128), round_up(T - nh + extra, 128), round_up(T + extra, 32)
 
 
 class SemkvCache:
-    """One layer's cache: device buffers + the semkv_cache_t descriptor."""
+    """One layer's cache: device buffers + the semkv_cache_t descriptor.  window and clip select
+    the quantizer variants (recent tokens forced onto the finer grid; clipped group range); 0 is
+    the plain method."""
 
     def __init__(self, B: int, H: int, Hq: int, G: int, L_hi: int, L_lo: int, cap_hi: int, cap_lo: int,
-                 T_cap: int, D: int = 128, device="cuda"):
+                 T_cap: int, D: int = 128, device="cuda", window: int = 0, clip: float = 0.0):
         import torch
 
         self.struct = _lib.CacheStruct(B=B, H=H, Hq=Hq, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=cap_hi,
-                                       cap_lo=cap_lo, T_cap=T_cap)
+                                       cap_lo=cap_lo, T_cap=T_cap, window=window, clip=clip)
         sizes = _lib.semkv_cache_bytes(self.struct)
         self.sizes = dict(zip(_lib.BUF_NAMES, sizes))
         self.bufs = {}
@@ -46,12 +49,12 @@ class SemkvCache:
             setattr(self.struct, name, int(t.data_ptr()))
         self.bufs["status"].zero_()
         self.shape = dict(B=B, H=H, Hq=Hq, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=cap_hi, cap_lo=cap_lo,
-                          T_cap=T_cap)
+                          T_cap=T_cap, window=window, clip=clip)
 
     @classmethod
-    def for_prefill(cls, B, H, Hq, G, L_hi, L_lo, T, p, extra=0, device="cuda"):
-        ch, cl, tc = capacities(T, p, extra)
-        return cls(B, H, Hq, G, L_hi, L_lo, ch, cl, tc, device=device)
+    def for_prefill(cls, B, H, Hq, G, L_hi, L_lo, T, p, extra=0, device="cuda", window=0, clip=0.0):
+        ch, cl, tc = capacities(T, p, extra, window)
+        return cls(B, H, Hq, G, L_hi, L_lo, ch, cl, tc, device=device, window=window, clip=clip)
 
     def __getattr__(self, name):
         shape = self.__dict__.get("shape", {})

@@ -24,6 +24,7 @@ int validate_shape(const semkv_cache_t* c)
     if (!level_ok(c->L_hi) || !level_ok(c->L_lo)) return SEMKV_ERR_UNSUPPORTED;
     if (c->G != 8 && c->G != 16 && c->G != 32 && c->G != 64 && c->G != 128) return SEMKV_ERR_UNSUPPORTED;
     if (c->Hq / c->H > 8) return SEMKV_ERR_UNSUPPORTED;
+    if (c->window < 0 || !(c->clip == 0.0f || (c->clip > 0.0f && c->clip <= 1.0f))) return SEMKV_ERR_INVALID_ARG;
     return SEMKV_OK;
 }
 
@@ -205,9 +206,10 @@ int semkv_assign_precision(const semkv_cache_t* c, const float* scores, int32_t 
     int r = validate(c);
     if (r != SEMKV_OK) return r;
     if (T < 0 || T > c->T_cap || !(p >= 0.0f && p <= 1.0f) || (!scores && T > 0)) return SEMKV_ERR_INVALID_ARG;
-    const int n_hi = (int)std::floor((double)p * (double)T);
-    if (n_hi > c->cap_hi || T - n_hi > c->cap_lo) return SEMKV_ERR_CAPACITY;
-    launch_select(scores, c->B * c->H, T, n_hi, c->T_cap / 32, c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau,
+    const int n_sel = (int)std::floor((double)p * (double)T);
+    const int win = c->window < T ? c->window : T;  // the recent tokens also put on the L_hi grid
+    if (n_sel + win > c->cap_hi || T - n_sel > c->cap_lo) return SEMKV_ERR_CAPACITY;
+    launch_select(scores, c->B * c->H, T, n_sel, win, c->T_cap / 32, c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau,
                   c->status, c->slot_token, c->cap_hi, c->cap_lo, c->score_keys, (cudaStream_t)stream);
     return launch_status();
 }
@@ -220,7 +222,7 @@ int semkv_quantize_pack(const semkv_cache_t* c, const uint16_t* K, const uint16_
     if (T == 0) return SEMKV_OK;
     if ((((uintptr_t)K) | ((uintptr_t)V)) & 15u) return SEMKV_ERR_INVALID_ARG;  // rows are fetched by bulk copies
     launch_quantize(seg_view(c, true), seg_view(c, false), K, V, c->slot_token, c->B * c->H, T, c->D, c->G,
-                    c->status, (cudaStream_t)stream);
+                    clip_ratio(*c), c->status, (cudaStream_t)stream);
     return launch_status();
 }
 

@@ -3,8 +3,8 @@
 // decode kernels that append and attend in one pass.
 //
 // SemKV page, Abstract: the quality cliff also appears for tokens quantized as they are generated.
-// The token is quantized alone with the prefill's affine rule and written at slot n_seg of its
-// segment.  K: the row's W words are written whole.  V: each channel's word that holds the slot
+// The token is quantized alone with the prefill's affine rule (and clip) and written at slot n_seg
+// of its segment.  K: the row's W words are written whole.  V: each channel's word that holds the slot
 // gets its digit -- a fresh word at the first slot of a word, otherwise the word plus
 // code * L^position (the digit was zero: slots are filled in order and the prefill wrote zero
 // digits past the segment's end).
@@ -63,8 +63,10 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
             vmx = fmaxf(vmx, gmx[1][w0 + i]);
         }
     }
-    const uint16_t ks16 = scale_half_ru(__fdiv_rn(__fsub_rn(kmx, kmn), (float)(L - 1))), kz16 = zero_half(kmn);
-    const uint16_t vs16 = scale_half_ru(__fdiv_rn(__fsub_rn(vmx, vmn), (float)(L - 1))), vz16 = zero_half(vmn);
+    const float clip = clip_ratio(c);
+    uint16_t ks16, kz16, vs16, vz16;
+    group_scale_zero(kmn, kmx, L, clip, ks16, kz16);
+    group_scale_zero(vmn, vmx, L, clip, vs16, vz16);
     const int grp = d / G;
     if (d % G == 0) {
         kz[grp * TILE + tt] = (uint32_t)ks16 | ((uint32_t)kz16 << 16);

@@ -112,6 +112,34 @@ __device__ __forceinline__ uint16_t scale_half_ru(float sf)
 // exact binary16 of a value that is itself a binary16 (the group minimum); -0 becomes +0.
 __device__ __forceinline__ uint16_t zero_half(float mn) { return __half_as_ushort(__float2half_rn(mn + 0.0f)); }
 
+// fp16 scale and zero of a group with extrema mn, mx on L levels.  clip = 1: s rounded up from
+// (mx - mn)/(L - 1), z = mn.  clip < 1 (clipped range, the SKVQ abstract): the extrema are scaled
+// by clip, z is the nearest binary16 of clip*mn (-0 as +0) and s is rounded up from
+// (clip*mx - z)/(L - 1), at least 0.  Values outside the clipped grid must be clamped by the caller.
+__device__ __forceinline__ void group_scale_zero(float mn, float mx, int L, float clip, uint16_t& s16, uint16_t& z16)
+{
+    if (clip == 1.0f) {
+        s16 = scale_half_ru(__fdiv_rn(__fsub_rn(mx, mn), (float)(L - 1)));
+        z16 = zero_half(mn);
+        return;
+    }
+    z16 = __half_as_ushort(__float2half_rn(__fmul_rn(clip, mn)));
+    if (z16 == 0x8000u) z16 = 0u;
+    float sf = __fdiv_rn(__fsub_rn(__fmul_rn(clip, mx), h2f(z16)), (float)(L - 1));
+    if (sf < 0.0f) sf = 0.0f;
+    s16 = scale_half_ru(sf);
+}
+
+// Tiles [t0, t1) of split s when `tiles` tiles are shared by nsplit splits: shares differ by at
+// most one tile (every split works when tiles >= nsplit, so each SM carries about the same load),
+// and the later splits take the smaller shares (the last tile, where an appended token lands,
+// is in the last split).
+__device__ __forceinline__ void split_tiles(int tiles, int nsplit, int s, int& t0, int& t1)
+{
+    t0 = tiles - (int)(((long long)tiles * (nsplit - s)) / nsplit);
+    t1 = tiles - (int)(((long long)tiles * (nsplit - 1 - s)) / nsplit);
+}
+
 // code of x on the grid (z, s) with L levels: clamp(rint((x - z)/s), 0, L - 1), IEEE fp32
 // subtract and divide, round half to even; 0 when s == 0.
 __device__ __forceinline__ int quant_code(float x, float z, float s, int L)

@@ -77,8 +77,8 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
 
     const int n = seg.n[u];
     const int tiles = min(ceil_div(n, TILE), seg.tiles_cap);  // never past the segment's capacity
-    const int per = ceil_div(tiles, nsplit);
-    const int t0 = split * per, t1 = min(tiles, t0 + per);
+    int t0, t1;
+    split_tiles(tiles, nsplit, split, t0, t1);
 
     float m[GMAX], acc[GMAX], zacc = 0.f, lacc = 0.f;
 #pragma unroll

@@ -84,7 +84,7 @@ __host__ __device__ constexpr uint32_t core_off(int n, int ks, uint32_t lbo, uin
     return (uint32_t)(n >> 3) * sbo + (uint32_t)(ks >> 3) * lbo + (uint32_t)(n & 7) * 16u + (uint32_t)(ks & 7) * 2u;
 }
 
-template <int L, int GQ, int NG>
+template <int L, int GQ, int NG, bool APP>
 __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_t* __restrict__ q, int H,
                                                        float scale_log2, int nsplit, int split_off, int nsplit_total,
                                                        float* __restrict__ ws, int32_t* __restrict__ status,
@@ -115,23 +115,23 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     __shared__ __align__(8) uint64_t mbar[4];                // 0: q.k done, 1: p.V done, 2/3: stage full
     __shared__ uint32_t tmem_base_s;
 
-    // append and attend in one pass (knew != nullptr): every CTA works out the new token's grid
+    // append and attend in one pass (APP; knew != nullptr): every CTA works out the new token's grid
     // and its segment's new length from the inputs alone (the counts are updated by the merge,
     // after every CTA has read them); the CTA whose tiles hold the new slot writes the row first
     int n = seg.n[u];
     int append_tile = -1;
     bool app_hi = false;
     int app_nh = 0, app_nl = 0;
-    if (knew) {
+    if constexpr (APP) {
         app_nh = cache.n_hi[u];
         app_nl = cache.n_lo[u];
         app_hi = snew[u] > cache.tau[u];  // NaN compares false: the token goes lo
         if (append_fits(cache, app_hi, app_nh, app_nl) && app_hi == (seg.is_hi != 0)) append_tile = n++ / TILE;
     }
     const int tiles = min(ceil_div(n, TILE), seg.tiles_cap);
-    const int per = ceil_div(tiles, nsplit);
-    const int t0 = split * per, t1 = min(tiles, t0 + per);
-    if (append_tile >= t0 && append_tile < t1) {
+    int t0, t1;
+    split_tiles(tiles, nsplit, split, t0, t1);
+    if (APP && append_tile >= t0 && append_tile < t1) {
         const bool bad = append_row(cache, u, app_hi, app_nh, app_nl, h2f(knew[(size_t)u * D + tid]),
                                     h2f(vnew[(size_t)u * D + tid]));
         if (bad && tid == 0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
@@ -427,7 +427,10 @@ static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, f
     using C = Tc<L, GQ, NG>;
     // at most four CTAs per SM: each holds 128 of the SM's 512 TMEM columns
     const size_t sm = C::TOTAL > 48u * 1024u ? C::TOTAL : 48u * 1024u;
-    cudaFuncSetAttribute(k_decode_tc<L, GQ, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    // the plain decode and the one that appends first are separate instantiations, so that the
+    // plain one carries no append code
+    const auto kern = app.k ? k_decode_tc<L, GQ, NG, true> : k_decode_tc<L, GQ, NG, false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)nsplit, (unsigned)units);
     cfg.blockDim = dim3(128);
@@ -438,7 +441,7 @@ static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, f
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = dependent ? 1 : 0;
-    cudaLaunchKernelEx(&cfg, k_decode_tc<L, GQ, NG>, seg, q, H, scale_log2, nsplit, split_off, nsplit_total, ws,
+    cudaLaunchKernelEx(&cfg, kern, seg, q, H, scale_log2, nsplit, split_off, nsplit_total, ws,
                        status, dependent ? 1 : 0, app.cache, app.k, app.v, app.score);
 }
 

@@ -8,6 +8,9 @@
 
 namespace semkv {
 
+// The clip ratio a cache asks for: 0 (unset) means 1, the plain min/max grid.
+__host__ __device__ __forceinline__ float clip_ratio(const semkv_cache_t& c) { return c.clip == 0.0f ? 1.0f : c.clip; }
+
 // One segment (hi or lo) of one layer's cache, as the kernels see it.
 struct SegView {
     uint32_t* k;    // [units][tiles_cap][WK][128]
@@ -29,13 +32,15 @@ struct AppendIn {
 };
 
 // also writes slot_token [units][cap_hi + cap_lo]: the token index of every prefill slot
-void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
-                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
-                   int cap_hi, int cap_lo, uint32_t* score_keys, cudaStream_t st);
+// n_sel tokens by score, then the last `window` tokens (window <= T) also get the L_hi grid
+void launch_select(const float* scores, int units, int T, int n_sel, int window, int words_cap, uint32_t* bitmap,
+                   uint32_t* rank, int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status,
+                   int32_t* slot_token, int cap_hi, int cap_lo, uint32_t* score_keys, cudaStream_t st);
 
 // reads the slot map (slot_token) that launch_select wrote
 void launch_quantize(const SegView& hi, const SegView& lo, const uint16_t* K, const uint16_t* V,
-                     const int32_t* slot_token, int units, int T, int D, int G, int32_t* status, cudaStream_t st);
+                     const int32_t* slot_token, int units, int T, int D, int G, float clip, int32_t* status,
+                     cudaStream_t st);
 
 // p < 0: the fixed threshold rule (score > tau); p in [0, 1]: the running top-p rule
 void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, float p,

@@ -52,11 +52,12 @@ struct Grid {
     float s, r, z;
 };
 
-// per-group grid: scale (fp16, rounded up, saturated), its reciprocal, zero
-__device__ __forceinline__ Grid make_grid(float mn, float mx, int L, uint32_t* packed)
+// per-group grid: scale (fp16, rounded up, saturated), its reciprocal, zero (clip < 1: of the
+// clipped range)
+__device__ __forceinline__ Grid make_grid(float mn, float mx, int L, float clip, uint32_t* packed)
 {
-    const uint16_t s16 = scale_half_ru(__fdiv_rn(__fsub_rn(mx, mn), (float)(L - 1)));
-    const uint16_t z16 = zero_half(mn);
+    uint16_t s16, z16;
+    group_scale_zero(mn, mx, L, clip, s16, z16);
     Grid g;
     g.s = h2f(s16);
     g.z = h2f(z16);
@@ -65,14 +66,14 @@ __device__ __forceinline__ Grid make_grid(float mn, float mx, int L, uint32_t* p
     return g;
 }
 
-// code of x on grid g: rint(RN((x - z)/s)) clamped to L - 1
+// code of x on grid g: rint(RN((x - z)/s)) clamped to [0, L - 1] (below 0 only on a clipped grid)
 __device__ __forceinline__ uint32_t code_of(float x, const Grid& g, float top)
 {
     const float d = __fsub_rn(x, g.z);
     const float q0 = __fmul_rn(d, g.r);
     const float e = __fmaf_rn(-g.s, q0, d);
     float q = __fmaf_rn(e, g.r, q0);
-    q = fminf(q, top);
+    q = fmaxf(fminf(q, top), 0.0f);
     return __float_as_uint(__fadd_rn(q, 12582912.0f)) - 0x4B400000u;
 }
 
@@ -109,7 +110,7 @@ __device__ __forceinline__ void gather_rows_warp(uint16_t* Ks, uint16_t* Vs, con
 
 __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
                                                    const uint16_t* __restrict__ V,
-                                                   int T, int G,
+                                                   int T, int G, float clip,
                                                    int32_t* __restrict__ status)
 {
     constexpr int D = 128;
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
                 }
             }
             uint32_t packed;
-            const Grid g = make_grid(mn, mx, L, &packed);
+            const Grid g = make_grid(mn, mx, L, clip, &packed);
             kz[grp * TILE + tid] = packed;
             for (int i = G - 8; i >= 0; i -= 8) {
                 float f[8];
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
                 }
             }
             uint32_t packed;
-            const Grid g = make_grid(mn, mx, L, &packed);
+            const Grid g = make_grid(mn, mx, L, clip, &packed);
             vgrid[tid * NG + grp] = make_float4(g.s, g.r, g.z, 0.0f);
             vz[grp * TILE + tid] = packed;
         }
@@ -461,7 +462,7 @@ static size_t quantize_smem(int G)
 }
 
 void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, const uint16_t* V,
-                     const int32_t* slot_token, int units, int T, int D, int G,
+                     const int32_t* slot_token, int units, int T, int D, int G, float clip,
                      int32_t* status, cudaStream_t st)
 {
     (void)D;
@@ -486,8 +487,9 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     const unsigned grid = (unsigned)units * per_unit;
     const QuantSeg qh = conv(shi, slot_token), ql = conv(slo, slot_token + shi.tiles_cap * TILE);
     // compile-time level pairs and group sizes of the common configurations
+    // (the clipped-range variant needs codes clamped from below, which only the generic kernel does)
 #define SEMKV_QF(LH, LL, GG)                                                                                  \
-    if (shi.L == LH && slo.L == LL && G == GG) {                                                              \
+    if (clip == 1.0f && shi.L == LH && slo.L == LL && G == GG) {                                                              \
         const size_t sm = (size_t)TILE * QROW * 2;                                                            \
         cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
         k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, status);                      \
@@ -499,7 +501,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
 #undef SEMKV_QF
     const size_t sm = quantize_smem(G);
     cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_quantize<<<grid, 128, sm, st>>>(qh, ql, K, V, T, G, status);
+    k_quantize<<<grid, 128, sm, st>>>(qh, ql, K, V, T, G, clip, status);
 }
 
 }  // namespace semkv

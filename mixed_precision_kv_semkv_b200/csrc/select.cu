@@ -1,4 +1,5 @@
-// Precision assignment: per unit, the n_hi largest of T fp32 scores get the L_hi grid.
+// Precision assignment: per unit, the n_sel largest of T fp32 scores get the L_hi grid (and, in the
+// recent-window variant, the last `window` tokens too; n_hi counts both).
 //
 // SemKV page, Abstract: tokens are ordered by an importance score from inside the model and the
 // top fraction is stored at the finer of two neighbouring precisions.  Ties: equal scores are
@@ -9,6 +10,8 @@
 // shared-memory histograms).  A final pass forms each
 // bitmap word from warp ballots (key > K*, key == K*), takes the first (n_hi - #greater) ties in
 // token order with a block-wide exclusive scan, and writes the rank directory with a second scan.
+// The window (the SKVQ abstract on the same pages: recent tokens kept at high precision) only ORs
+// a suffix of tokens into the words; the selection, its ties and tau do not see it.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -27,6 +30,16 @@ __device__ __forceinline__ float key_score(uint32_t k)
 {
     uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
     return __uint_as_float(u);
+}
+
+// bits of bitmap word w that hold tokens of the window [win_lo, T)
+__device__ __forceinline__ uint32_t window_bits(int w, int T, int win_lo)
+{
+    const int a = win_lo - 32 * w, b = T - 32 * w;  // the window's bit range [a, b) in this word
+    if (b <= 0 || a >= 32 || a >= b) return 0u;
+    const uint32_t below_b = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+    const uint32_t from_a = a <= 0 ? 0xffffffffu : ~((1u << a) - 1u);
+    return below_b & from_a;
 }
 
 // One CTA of 1024 threads per unit.  CACHED: the keys are first copied into shared memory (T up to
@@ -54,7 +67,8 @@ __device__ __forceinline__ void emit_slot_tokens(int32_t* __restrict__ st_hi, in
 }
 
 template <bool CACHED>
-__global__ void __launch_bounds__(1024) k_select(const float* __restrict__ scores, int T, int n_hi, int words_cap,
+__global__ void __launch_bounds__(1024) k_select(const float* __restrict__ scores, int T, int n_hi, int window,
+                                                  int words_cap,
                                                   uint32_t* __restrict__ bitmap, uint32_t* __restrict__ rank,
                                                   int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
                                                   float* __restrict__ tau_out, int32_t* __restrict__ status,
@@ -75,8 +89,8 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
     // NaN scores: flag; their keys sort above +inf (order unspecified, as documented)
     {
         bool bad = false;
-#pragma unroll 8
         uint32_t* sk = score_keys + (size_t)u * 32 * words_cap;
+#pragma unroll 8
         for (int t = tid; t < T; t += blockDim.x) {
             const float f = s[t];
             bad |= isnan(f);
@@ -170,7 +184,7 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
                 take_mask = my_eq & (0xffffffffu >> (31u - pos));
             }
         }
-        uint32_t word = my_gt | take_mask;
+        uint32_t word = my_gt | take_mask | (w < nwords ? window_bits(w, T, T - window) : 0u);
         uint32_t ones_before = carry_ones + block_excl_scan((uint32_t)__popc(word), scan_tmp, &tot);
         carry_ones += tot;
         if (w < nwords) {
@@ -181,11 +195,11 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
     }
     for (int w = nwords + tid; w < words_cap; w += blockDim.x) {
         bm[w] = 0u;
-        rk[w] = (uint32_t)n_hi;
+        rk[w] = carry_ones;
     }
     if (tid == 0) {
-        n_hi_out[u] = n_hi;
-        n_lo_out[u] = T - n_hi;
+        n_hi_out[u] = (int)carry_ones;  // n_hi (selected) plus the window's other tokens
+        n_lo_out[u] = T - (int)carry_ones;
         tau_out[u] = n_hi > 0 ? key_score(kstar) : __int_as_float(0x7f800000);
     }
 }
@@ -207,7 +221,8 @@ constexpr int SEL_CS = 8, SEL_THREADS = 512, SEL_WARPS = SEL_THREADS / 32;
 
 template <int KPT>
 __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
-    k_select_cluster(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
+    k_select_cluster(const float* __restrict__ scores, int T, int n_hi, int window, int words_cap,
+                     uint32_t* __restrict__ bitmap,
                      uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
                      float* __restrict__ tau_out, int32_t* __restrict__ status,
                  int32_t* __restrict__ slot_token, int cap_hi, int cap_lo, uint32_t* __restrict__ score_keys)
@@ -227,15 +242,15 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     __shared__ uint32_t gtm[KPT * SEL_WARPS], eqm[KPT * SEL_WARPS];
     __shared__ uint32_t scan_tmp[33];
     __shared__ uint32_t andor[2];   // this CTA's AND and OR of its keys
-    __shared__ uint32_t totals[2];  // this CTA's ties and strictly-greater counts
+    __shared__ __align__(16) uint32_t totals[4];  // ties, strictly-greater, window-and-not-greater, window ties
     __shared__ uint32_t sh_prefix, sh_remaining, red_and[SEL_WARPS], red_or[SEL_WARPS];
 
     // my keys: tokens tok0 + j*512 + tid (j < KPT) that fall in my CTA's range and below T
     uint32_t key[KPT];
     bool bad = false;
     uint32_t kand = 0xffffffffu, kor = 0u;
-#pragma unroll
     uint32_t* sk = score_keys + (size_t)u * 32 * words_cap;
+#pragma unroll
     for (int j = 0; j < KPT; ++j) {
         const int t = tok0 + j * SEL_THREADS + tid;
         const bool in = t < 32 * w1 && t < T;
@@ -356,23 +371,49 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
         my_gt = gtm[tid];
         my_eq = eqm[tid];
     }
-    uint32_t tot_ties, tot_gt;
+    const uint32_t my_win = tid < nw ? window_bits(w0 + tid, T, T - window) : 0u;
+    uint32_t tot_ties, tot_gt, tot_wng = 0u, tot_wt = 0u;
     uint32_t ties_before = block_excl_scan((uint32_t)__popc(my_eq), scan_tmp, &tot_ties);
     block_excl_scan((uint32_t)__popc(my_gt), scan_tmp, &tot_gt);
+    if (window > 0) {  // uniform over the cluster
+        block_excl_scan((uint32_t)__popc(my_win & ~my_gt), scan_tmp, &tot_wng);
+        block_excl_scan((uint32_t)__popc(my_win & my_eq), scan_tmp, &tot_wt);
+    }
     if (tid == 0) {
         totals[0] = tot_ties;
         totals[1] = tot_gt;
+        totals[2] = tot_wng;
+        totals[3] = tot_wt;
     }
     cluster.sync();
-    // ties and ones of the earlier CTAs
-    uint32_t cta_ties_before = 0u, cta_ones_before = 0u;
-    for (int r = 0; r < c; ++r) {
-        const uint32_t* rt = cluster.map_shared_rank(totals, r);
-        const uint32_t rties = rt[0], rgt = rt[1];
-        const uint32_t taken = cta_ties_before >= take ? 0u : min(rties, take - cta_ties_before);
-        cta_ones_before += rgt + taken;
-        cta_ties_before += rties;
+    // ones (L_hi tokens) of the earlier CTAs, and of all: CTA r holds gt_r greater keys and takes
+    // the ties at global tie positions below `take`; the window is a suffix of the tokens, so its
+    // ties in CTA r are r's last wt_r ties, and the window adds its tokens that are neither
+    // greater nor taken ties.
+    // Lane r < SEL_CS of every warp fetches CTA r's four counts (one 16-byte remote load) and the
+    // warp combines them with scans over the ranks.
+    uint4 tr = make_uint4(0u, 0u, 0u, 0u);
+    if (lane < SEL_CS) tr = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(totals, lane));
+    uint32_t ties_inc = tr.x;
+#pragma unroll
+    for (int o = 1; o < SEL_CS; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, ties_inc, o);
+        if (lane >= o) ties_inc += v;
     }
+    const uint32_t ties_acc = ties_inc - tr.x;  // ties of the CTAs before rank `lane`
+    const uint32_t taken = ties_acc >= take ? 0u : min(tr.x, take - ties_acc);
+    const uint32_t first_wt = ties_acc + tr.x - tr.w;  // global tie position of rank lane's first window tie
+    const uint32_t taken_w = take <= first_wt ? 0u : min(tr.w, take - first_wt);
+    const uint32_t ones = lane < SEL_CS ? tr.y + taken + (tr.z - taken_w) : 0u;
+    uint32_t ones_inc = ones;
+#pragma unroll
+    for (int o = 1; o < SEL_CS; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, ones_inc, o);
+        if (lane >= o) ones_inc += v;
+    }
+    const uint32_t cta_ties_before = __shfl_sync(0xffffffffu, ties_acc, c);
+    const uint32_t cta_ones_before = __shfl_sync(0xffffffffu, ones_inc - ones, c);
+    const uint32_t ones_total = __shfl_sync(0xffffffffu, ones_inc, SEL_CS - 1);
     ties_before += cta_ties_before;
     uint32_t take_mask = 0u;
     if (ties_before < take) {
@@ -384,7 +425,7 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
             take_mask = my_eq & (0xffffffffu >> (31u - pos));
         }
     }
-    const uint32_t word = my_gt | take_mask;
+    const uint32_t word = my_gt | take_mask | my_win;
     uint32_t tot_ones;
     const uint32_t ones_before = cta_ones_before + block_excl_scan((uint32_t)__popc(word), scan_tmp, &tot_ones);
     uint32_t* bm = bitmap + (size_t)u * words_cap;
@@ -417,11 +458,11 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     }
     for (int w = nwords + c * SEL_THREADS + tid; w < words_cap; w += SEL_CS * SEL_THREADS) {
         bm[w] = 0u;
-        rk[w] = (uint32_t)n_hi;
+        rk[w] = ones_total;
     }
     if (c == 0 && tid == 0) {
-        n_hi_out[u] = n_hi;
-        n_lo_out[u] = T - n_hi;
+        n_hi_out[u] = (int)ones_total;
+        n_lo_out[u] = T - (int)ones_total;
         tau_out[u] = n_hi > 0 ? key_score(kstar) : __int_as_float(0x7f800000);
     }
     cluster.sync();  // no CTA leaves while another may still read its shared memory
@@ -437,7 +478,8 @@ constexpr int SELR_THREADS = 1024, SELR_WARPS = SELR_THREADS / 32;
 
 template <int KPT>
 __global__ void __launch_bounds__(SELR_THREADS)
-    k_select_reg(const float* __restrict__ scores, int T, int n_hi, int words_cap, uint32_t* __restrict__ bitmap,
+    k_select_reg(const float* __restrict__ scores, int T, int n_hi, int window, int words_cap,
+                 uint32_t* __restrict__ bitmap,
                  uint32_t* __restrict__ rank, int32_t* __restrict__ n_hi_out, int32_t* __restrict__ n_lo_out,
                  float* __restrict__ tau_out, int32_t* __restrict__ status,
                  int32_t* __restrict__ slot_token, int cap_hi, int cap_lo, uint32_t* __restrict__ score_keys)
@@ -453,8 +495,8 @@ __global__ void __launch_bounds__(SELR_THREADS)
 
     uint32_t key[KPT];
     bool bad = false;
-#pragma unroll
     uint32_t* sk = score_keys + (size_t)u * 32 * words_cap;
+#pragma unroll
     for (int j = 0; j < KPT; ++j) {
         const int t = j * SELR_THREADS + tid;
         const float f = t < T ? s[t] : 0.f;
@@ -533,8 +575,8 @@ __global__ void __launch_bounds__(SELR_THREADS)
             take_mask = my_eq & (0xffffffffu >> (31u - pos));
         }
     }
-    const uint32_t word = my_gt | take_mask;
-    const uint32_t ones_before = block_excl_scan((uint32_t)__popc(word), scan_tmp, &tot);
+    const uint32_t word = my_gt | take_mask | (tid < nwords ? window_bits(tid, T, T - window) : 0u);
+    const uint32_t ones_before = block_excl_scan((uint32_t)__popc(word), scan_tmp, &tot);  // tot: all ones
     uint32_t* bm = bitmap + (size_t)u * words_cap;
     uint32_t* rk = rank + (size_t)u * words_cap;
     if (tid < nwords) {
@@ -547,21 +589,21 @@ __global__ void __launch_bounds__(SELR_THREADS)
     }
     for (int w = nwords + tid; w < words_cap; w += SELR_THREADS) {
         bm[w] = 0u;
-        rk[w] = (uint32_t)n_hi;
+        rk[w] = tot;
     }
     if (tid == 0) {
-        n_hi_out[u] = n_hi;
-        n_lo_out[u] = T - n_hi;
+        n_hi_out[u] = (int)tot;
+        n_lo_out[u] = T - (int)tot;
         tau_out[u] = n_hi > 0 ? key_score(kstar) : __int_as_float(0x7f800000);
     }
 }
 
-void launch_select(const float* scores, int units, int T, int n_hi, int words_cap, uint32_t* bitmap, uint32_t* rank,
-                   int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status, int32_t* slot_token,
-                   int cap_hi, int cap_lo, uint32_t* score_keys, cudaStream_t st)
+void launch_select(const float* scores, int units, int T, int n_hi, int window, int words_cap, uint32_t* bitmap,
+                   uint32_t* rank, int32_t* n_hi_out, int32_t* n_lo_out, float* tau, int32_t* status,
+                   int32_t* slot_token, int cap_hi, int cap_lo, uint32_t* score_keys, cudaStream_t st)
 {
     if (T <= SELR_THREADS) {  // one key per thread: a single CTA
-        k_select_reg<1><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out,
+        k_select_reg<1><<<units, SELR_THREADS, 0, st>>>(scores, T, n_hi, window, words_cap, bitmap, rank, n_hi_out,
                                                         n_lo_out, tau, status, slot_token, cap_hi, cap_lo, score_keys);
         return;
     }
@@ -571,14 +613,14 @@ void launch_select(const float* scores, int units, int T, int n_hi, int words_ca
     const dim3 grid((unsigned)(units * SEL_CS));
 #define SEMKV_SEL(K)                                                                                           \
     if (kpt <= K) {                                                                                            \
-        k_select_cluster<K><<<grid, SEL_THREADS, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, \
+        k_select_cluster<K><<<grid, SEL_THREADS, 0, st>>>(scores, T, n_hi, window, words_cap, bitmap, rank, n_hi_out, \
                                                           n_lo_out, tau, status, slot_token, cap_hi, cap_lo, score_keys);                             \
         return;                                                                                                \
     }
     SEMKV_SEL(1) SEMKV_SEL(2) SEMKV_SEL(4) SEMKV_SEL(8) SEMKV_SEL(16) SEMKV_SEL(32)
 #undef SEMKV_SEL
     // more keys than a cluster holds in registers: one CTA per unit streams the scores from L2
-    k_select<false><<<units, 1024, 0, st>>>(scores, T, n_hi, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
+    k_select<false><<<units, 1024, 0, st>>>(scores, T, n_hi, window, words_cap, bitmap, rank, n_hi_out, n_lo_out, tau,
                                             status, slot_token, cap_hi, cap_lo, score_keys);
 }
 

@@ -54,12 +54,12 @@ def fetch(cache: SemkvCache) -> dict:
     return {n: t.cpu().numpy() for n, t in cache.bufs.items()}
 
 
-def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0):
+def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0):
     import torch
 
     B, H, T, D = K.shape
     Hq = q.shape[1]
-    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra).poison()
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra, window=window, clip=clip).poison()
     dK, dV, dS, dq = to_dev(K), to_dev(V), to_dev(S), to_dev(q)
     semkv_assign_precision(cache, dS, T, p)
     semkv_quantize_pack(cache, dK, dV, T)
@@ -74,11 +74,12 @@ def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0):
     return res
 
 
-def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo):
-    """Oracle results of one unit. K, V [T][D] fp16; S [T]; q [g][D] fp16."""
-    bm, rk, nh, tau, st = oracle.select(S, p)
+def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo, window=0, clip=0.0):
+    """Oracle results of one unit. K, V [T][D] fp16; S [T]; q [g][D] fp16.  window, clip: the
+    quantizer variants as the cache fields state them (clip 0 = 1 = off)."""
+    bm, rk, nh, tau, st = oracle.select(S, p, window=window)
     hi, lo, st2 = oracle.quantize_pack_unit(K.view(np.uint16), V.view(np.uint16), bm, G, L_hi, L_lo, tiles_hi,
-                                            tiles_lo)
+                                            tiles_lo, clip=clip or 1.0)
     T = K.shape[0]
     Kh, Vh = oracle.dequantize_unit(T, K.shape[1], G, L_hi, L_lo, bm, hi, lo)
     o = oracle.attention_fp64(q.view(np.uint16), Kh, Vh, scale)
@@ -133,11 +134,11 @@ def attention_errors(got, ref):
     return max_abs, rel
 
 
-def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None):
+def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0.0):
     """Run the GPU path on a whole case and compare the chosen units (default: all) with the oracle."""
     B, H, T, D = K.shape
     g = q.shape[1] // H
-    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale)
+    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, window=window, clip=clip)
     cache = res["cache"]
     assert res["status"] == 0, f"status {res['status']}"
     units = range(B * H) if units is None else units
@@ -145,7 +146,7 @@ def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None):
     for u in units:
         b, h = divmod(u, H)
         o = oracle_unit(K[b, h], V[b, h], S[b, h], q[b, h * g:(h + 1) * g], p, G, L_hi, L_lo, scale,
-                        cache.cap_hi // 128, cache.cap_lo // 128)
+                        cache.cap_hi // 128, cache.cap_lo // 128, window=window, clip=clip)
         gu = unit_views(cache, res["bufs"], u)
         compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}")
         assert np.array_equal(res["Kh"][b, h].view(np.uint32), o["Kh"].view(np.uint32)), f"Khat unit {u}"

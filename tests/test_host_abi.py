@@ -64,6 +64,7 @@ def test_cache_bytes_match_oracle_layout(semkv, orc, L_hi, L_lo, G):
 @pytest.mark.parametrize("bad,code", [
     (dict(Hq=30), 1), (dict(G=48), 1), (dict(cap_hi=100), 1), (dict(T_cap=1000), 1), (dict(B=0), 1),
     (dict(D=64, G=64), 2), (dict(L_hi=257), 2), (dict(L_lo=1), 2), (dict(G=4), 2), (dict(Hq=8 * 16), 2),
+    (dict(window=-1), 1), (dict(clip=1.5), 1), (dict(clip=-0.25), 1), (dict(clip=float("nan")), 1),
 ])
 def test_bad_shapes_are_rejected(semkv, bad, code):
     with pytest.raises(semkv.SemkvError) as e:
@@ -95,12 +96,20 @@ def test_calls_fail_before_any_launch(semkv):
     assert L.semkv_assign_precision(ref, one, 2000, 0.25, nul) == 1     # T > T_cap
     assert L.semkv_assign_precision(ref, nul, 100, 0.25, nul) == 1      # null scores
     assert L.semkv_assign_precision(ref, one, 1024, 0.5, nul) == 3      # n_hi = 512 > cap_hi = 256
+    s.window = 1
+    assert L.semkv_assign_precision(ref, one, 1024, 0.25, nul) == 3     # 256 selected + 1 window > 256
+    s.window = 0
     assert L.semkv_quantize_pack(ref, nul, one, 10, nul) == 1
     assert L.semkv_append_token(ref, one, one, nul, nul) == 1
     assert L.semkv_decode_attention(ref, one, ctypes.c_float(float("inf")), one, one, 1 << 30, nul) == 1
     assert L.semkv_decode_attention(ref, one, ctypes.c_float(0.1), one, one, 0, nul) == 1  # workspace too small
     assert L.semkv_dequantize(ref, one, nul, 10, nul) == 1
     assert semkv.status_string(3) == "SEMKV_ERR_CAPACITY"
+
+
+def test_variant_fields_accept_their_ranges(semkv):
+    for kw in (dict(window=0, clip=0.0), dict(window=10 ** 6, clip=1.0), dict(clip=1e-6), dict(clip=0.5)):
+        assert len(semkv.semkv_cache_bytes(_shape(**kw))) == len(semkv._lib.BUF_NAMES)
 
 
 def test_workspace_bytes_cover_the_split_partials(semkv):
