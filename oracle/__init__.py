@@ -79,12 +79,13 @@ def lib():
         L.oracle_pack_word.restype = _c.c_uint32
         L.oracle_unpack_word.argtypes = [_c.c_uint32, _c.c_int, _c.c_int, _u8p]
         L.oracle_quantize_pack_unit.argtypes = [_u16p, _u16p, _c.c_int32, _c.c_int, _c.c_int, _c.c_int,
-                                                _c.c_int, _c.c_float, _u32p, _c.c_int, _c.c_int] + [_u32p] * 8
+                                                _c.c_int, _c.c_int, _c.c_int, _c.c_float, _u32p, _c.c_int,
+                                                _c.c_int] + [_u32p] * 8
         L.oracle_quantize_pack_unit.restype = _c.c_int
-        L.oracle_dequantize_unit.argtypes = [_c.c_int32, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _u32p] + \
-            [_u32p] * 8 + [_f32p, _f32p]
+        L.oracle_dequantize_unit.argtypes = [_c.c_int32, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
+                                             _u32p] + [_u32p] * 8 + [_f32p, _f32p]
         L.oracle_append_unit.argtypes = [_u16p, _u16p, _c.c_float, _c.c_float, _c.c_int, _c.c_int, _c.c_int,
-                                         _c.c_int, _c.c_float, _c.c_int32, _u32p, _u32p, _c.POINTER(_c.c_int32),
+                                         _c.c_int, _c.c_int, _c.c_int, _c.c_float, _c.c_int32, _u32p, _u32p, _c.POINTER(_c.c_int32),
                                          _c.POINTER(_c.c_int32), _c.c_int, _c.c_int] + [_u32p] * 8
         L.oracle_append_unit.restype = _c.c_int
         L.oracle_attention_fp64.argtypes = [_u16p, _c.c_int, _f32p, _f32p, _c.c_int32, _c.c_int, _c.c_float,
@@ -176,17 +177,17 @@ def unpack_word(w: int, k: int, L: int) -> np.ndarray:
     return out
 
 
-def segment_shapes(D: int, G: int, L: int, tiles: int):
-    """Shapes of one segment's four buffers in the oracle's layout."""
+def segment_shapes(D: int, G: int, L: int, tiles: int, Lv: int | None = None):
+    """Shapes of one segment's four buffers in the oracle's layout (Lv: the V level count, if not L)."""
     WK = words_per_row(L, D)
-    WV = words_per_tile_column(L)
+    WV = words_per_tile_column(Lv or L)
     ng = D // G
     return {"k": (tiles, WK, TILE), "v": (tiles, WV, D), "kz": (tiles, ng, TILE), "vz": (tiles, ng, TILE)}
 
 
-def _alloc_unit(D, G, L_hi, L_lo, tiles_hi, tiles_lo):
-    hi = {n: np.zeros(s, np.uint32) for n, s in segment_shapes(D, G, L_hi, tiles_hi).items()}
-    lo = {n: np.zeros(s, np.uint32) for n, s in segment_shapes(D, G, L_lo, tiles_lo).items()}
+def _alloc_unit(D, G, L_hi, L_lo, tiles_hi, tiles_lo, L_hi_v=None, L_lo_v=None):
+    hi = {n: np.zeros(s, np.uint32) for n, s in segment_shapes(D, G, L_hi, tiles_hi, L_hi_v).items()}
+    lo = {n: np.zeros(s, np.uint32) for n, s in segment_shapes(D, G, L_lo, tiles_lo, L_lo_v).items()}
     return hi, lo
 
 
@@ -196,29 +197,33 @@ def _seg_args(hi, lo):
 
 
 def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi: int, tiles_lo: int,
-                       clip: float = 1.0):
-    """Quantize and place one unit. K16, V16: [T][D] uint16. Returns (hi, lo, status)."""
+                       clip: float = 1.0, L_hi_v: int | None = None, L_lo_v: int | None = None):
+    """Quantize and place one unit. K16, V16: [T][D] uint16.  L_hi_v, L_lo_v: V level counts of the
+    two segments (default: the K ones). Returns (hi, lo, status)."""
     K16 = np.ascontiguousarray(K16, dtype=np.uint16)
     V16 = np.ascontiguousarray(V16, dtype=np.uint16)
     T, D = K16.shape
-    hi, lo = _alloc_unit(D, G, L_hi, L_lo, tiles_hi, tiles_lo)
+    L_hi_v, L_lo_v = L_hi_v or L_hi, L_lo_v or L_lo
+    hi, lo = _alloc_unit(D, G, L_hi, L_lo, tiles_hi, tiles_lo, L_hi_v, L_lo_v)
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
     n = min(len(bitmap), len(bm))
     bm[:n] = bitmap[:n]
-    st = lib().oracle_quantize_pack_unit(K16.ravel(), V16.ravel(), T, D, G, L_hi, L_lo, float(clip), bm, tiles_hi,
-                                         tiles_lo,
+    st = lib().oracle_quantize_pack_unit(K16.ravel(), V16.ravel(), T, D, G, L_hi, L_lo, L_hi_v, L_lo_v, float(clip),
+                                         bm, tiles_hi, tiles_lo,
                                          *_seg_args(hi, lo))
     return hi, lo, st
 
 
-def dequantize_unit(T: int, D: int, G: int, L_hi: int, L_lo: int, bitmap, hi, lo):
+def dequantize_unit(T: int, D: int, G: int, L_hi: int, L_lo: int, bitmap, hi, lo, L_hi_v: int | None = None,
+                    L_lo_v: int | None = None):
     """Dequantize one unit back to original token order. Returns (Khat, Vhat) fp32 [T][D]."""
     Kh = np.zeros((max(T, 1), D), np.float32)
     Vh = np.zeros((max(T, 1), D), np.float32)
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
     n = min(len(bitmap), len(bm))
     bm[:n] = bitmap[:n]
-    lib().oracle_dequantize_unit(T, D, G, L_hi, L_lo, bm, *_seg_args(hi, lo), Kh.ravel(), Vh.ravel())
+    lib().oracle_dequantize_unit(T, D, G, L_hi, L_lo, L_hi_v or L_hi, L_lo_v or L_lo, bm, *_seg_args(hi, lo),
+                                 Kh.ravel(), Vh.ravel())
     return Kh[:T], Vh[:T]
 
 
@@ -239,15 +244,17 @@ class UnitState:
         self.lo = lo
 
 
-def append_unit(state: UnitState, k16, v16, score: float, G: int, L_hi: int, L_lo: int, clip: float = 1.0) -> int:
-    """Append one token to a unit in place (clip: as in quantize_group). Returns status bits."""
+def append_unit(state: UnitState, k16, v16, score: float, G: int, L_hi: int, L_lo: int, clip: float = 1.0,
+                L_hi_v: int | None = None, L_lo_v: int | None = None) -> int:
+    """Append one token to a unit in place (clip, V level counts: as in quantize_pack_unit).
+    Returns status bits."""
     k16 = np.ascontiguousarray(k16, dtype=np.uint16)
     v16 = np.ascontiguousarray(v16, dtype=np.uint16)
     D = k16.shape[0]
     nh = _c.c_int32(state.n_hi)
     nl = _c.c_int32(state.n_lo)
-    st = lib().oracle_append_unit(k16, v16, float(score), float(state.tau), D, G, L_hi, L_lo, float(clip),
-                                  state.T_cap,
+    st = lib().oracle_append_unit(k16, v16, float(score), float(state.tau), D, G, L_hi, L_lo, L_hi_v or L_hi,
+                                  L_lo_v or L_lo, float(clip), state.T_cap,
                                   state.bitmap, state.rank, _c.byref(nh), _c.byref(nl),
                                   state.hi["k"].shape[0], state.lo["k"].shape[0], *_seg_args(state.hi, state.lo))
     state.n_hi = nh.value
@@ -281,18 +288,19 @@ def running_is_hi(scores_prev, score_new: float, p: float) -> bool:
 
 
 def append_unit_running(state: UnitState, k16, v16, score: float, p: float, scores_prev, G: int, L_hi: int,
-                        L_lo: int, clip: float = 1.0) -> int:
+                        L_lo: int, clip: float = 1.0, L_hi_v: int | None = None, L_lo_v: int | None = None) -> int:
     """append_unit with the running top-p rule: the grid comes from running_is_hi (the fixed tau
     of the state is left as it was)."""
     tau = state.tau
     state.tau = np.float32(-np.inf) if running_is_hi(scores_prev, score, p) else np.float32(np.inf)
     try:
-        return append_unit(state, k16, v16, score, G, L_hi, L_lo, clip)
+        return append_unit(state, k16, v16, score, G, L_hi, L_lo, clip, L_hi_v, L_lo_v)
     finally:
         state.tau = tau
 
 
-def p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float, iters: int = 200):
+def p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float, iters: int = 200, L_hi_v: int | None = None,
+                L_lo_v: int | None = None):
     """Largest fraction p in [0, 1] of tokens on the L_hi grid whose storage reduction against
     fp16 (16 bits / storage_bits_per_value) is still at least `ratio`; None if even p = 0 misses
     it.  SemKV page, Abstract: the recipe is to measure the quality cliff and then interpolate
@@ -300,7 +308,7 @@ def p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float, iters: int =
     on the buffer-derived storage above (no closed-form inversion)."""
     if not ratio > 0.0:
         return None
-    ok = lambda p: 16.0 / storage_bits_per_value(D, G, L_hi, L_lo, p) >= ratio  # noqa: E731
+    ok = lambda p: 16.0 / storage_bits_per_value(D, G, L_hi, L_lo, p, L_hi_v, L_lo_v) >= ratio  # noqa: E731
     if ok(1.0):
         return 1.0
     if not ok(0.0):
@@ -317,15 +325,19 @@ def p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float, iters: int =
     return lo
 
 
-def storage_bits_per_value(D: int, G: int, L_hi: int, L_lo: int, p_real: float) -> float:
-    """Physical bits per cached value (K or V), from the oracle's own buffer sizes per full tile.
+def storage_bits_per_value(D: int, G: int, L_hi: int, L_lo: int, p_real: float, L_hi_v: int | None = None,
+                           L_lo_v: int | None = None) -> float:
+    """Physical bits per cached value (K and V averaged), from the oracle's own buffer sizes per
+    full tile.
 
-    Counts the packed code words, the fp16 scale + fp16 zero per group and the one-bit precision
-    bitmap (shared by K and V, so half a bit per token per channel pair / D).
+    Counts the packed code words of K and of V (each with its own level count), the fp16 scale +
+    fp16 zero per group and the one-bit precision bitmap (shared by K and V, so half a bit per
+    token per channel pair / D).
     """
-    def seg_bits(L):
-        sh = segment_shapes(D, G, L, 1)
+    def seg_bits(L, Lv):
+        sh = segment_shapes(D, G, L, 1, Lv)
         words_k = int(np.prod(sh["k"]))     # one tile of K rows: 128 tokens x D channels
-        words_sz = int(np.prod(sh["kz"]))
-        return (words_k + words_sz) * 32 / (TILE * D)
-    return p_real * seg_bits(L_hi) + (1 - p_real) * seg_bits(L_lo) + 1.0 / (2 * D)
+        words_v = int(np.prod(sh["v"]))     # one tile of V columns: the same 128 x D values
+        words_sz = int(np.prod(sh["kz"]))   # per tensor
+        return ((words_k + words_v) / 2 + words_sz) * 32 / (TILE * D)
+    return p_real * seg_bits(L_hi, L_hi_v or L_hi) + (1 - p_real) * seg_bits(L_lo, L_lo_v or L_lo) + 1.0 / (2 * D)

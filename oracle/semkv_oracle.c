@@ -38,11 +38,13 @@
  *               quantization at generation time too) is hi iff its score > tau of its unit
  *               (strict) [reading]; it is quantized alone and placed at the next slot.
  *   dequantize  x^ = fmaf((float)c, s, z).
- *   variants    two quantizer variants of prior art that the pages summarise (the SKVQ abstract):
- *               a clip ratio that shrinks each group's range before the grid is fitted, and a
- *               window of the most recent tokens forced onto the finer grid at selection.  Both
- *               are off by default; the formulas are readings, given at oracle_quantize_group_clip
- *               and oracle_select.
+ *   variants    three quantizer variants of prior art that the pages summarise (the SKVQ abstract):
+ *               a clip ratio that shrinks each group's range before the grid is fitted; a window
+ *               of the most recent tokens forced onto the finer grid at selection; and level
+ *               counts of their own for V (keys and values at different bit widths): each segment
+ *               has a K level count and a V level count, and each tensor's codes, scale and radix
+ *               words use its own.  All are off by default; the formulas are readings, given at
+ *               oracle_quantize_group_clip and oracle_select.
  *   attention   fp64: o = sum_t softmax_t(sigma * q.k^_t) v^_t over all tokens of the unit, for
  *               each of the g query heads that share the kv head (GQA); no mask.
  *
@@ -321,28 +323,29 @@ static size_t sz_index(int tile, int grp, int t, int NG)
     return ((size_t)tile * NG + grp) * OR_TILE + t;
 }
 
-/* Pack one segment from its per-slot codes (zero codes past n_seg) into the tile layout. */
-static void pack_segment(const uint8_t* ck, const uint8_t* cv, int tiles, int D, int L, uint32_t* kw,
+/* Pack one segment from its per-slot codes (zero codes past n_seg) into the tile layout: K words
+ * in base Lk, V words in base Lv. */
+static void pack_segment(const uint8_t* ck, const uint8_t* cv, int tiles, int D, int Lk, int Lv, uint32_t* kw,
                          uint32_t* vw)
 {
-    int k = oracle_radix_digits(L);
-    int WK = ceil_div(D, k), WV = ceil_div(OR_TILE, k);
-    uint8_t* buf = (uint8_t*)malloc((size_t)k);
+    int kk = oracle_radix_digits(Lk), kv = oracle_radix_digits(Lv);
+    int WK = ceil_div(D, kk), WV = ceil_div(OR_TILE, kv);
+    uint8_t* buf = (uint8_t*)malloc((size_t)(kk > kv ? kk : kv));
     for (int tile = 0; tile < tiles; tile++) {
         for (int t = 0; t < OR_TILE; t++) {
             const uint8_t* row = ck + ((size_t)tile * OR_TILE + t) * D;
             for (int j = 0; j < WK; j++) {
-                for (int i = 0; i < k; i++) buf[i] = (j * k + i < D) ? row[j * k + i] : 0;
-                kw[k_word_index(tile, j, t, WK)] = oracle_pack_word(buf, k, L);
+                for (int i = 0; i < kk; i++) buf[i] = (j * kk + i < D) ? row[j * kk + i] : 0;
+                kw[k_word_index(tile, j, t, WK)] = oracle_pack_word(buf, kk, Lk);
             }
         }
         for (int d = 0; d < D; d++) {
             for (int w = 0; w < WV; w++) {
-                for (int i = 0; i < k; i++) {
-                    int slot = w * k + i;
+                for (int i = 0; i < kv; i++) {
+                    int slot = w * kv + i;
                     buf[i] = slot < OR_TILE ? cv[((size_t)tile * OR_TILE + slot) * D + d] : 0;
                 }
-                vw[v_word_index(tile, w, d, WV, D)] = oracle_pack_word(buf, k, L);
+                vw[v_word_index(tile, w, d, WV, D)] = oracle_pack_word(buf, kv, Lv);
             }
         }
     }
@@ -354,16 +357,18 @@ static void pack_segment(const uint8_t* ck, const uint8_t* cv, int tiles, int D,
  * Segment buffers must hold tiles_hi (tiles_lo) tiles; slots past n_seg are written as zeros.
  */
 int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, int D, int G, int L_hi,
-                              int L_lo, float clip, const uint32_t* bitmap, int tiles_hi, int tiles_lo,
+                              int L_lo, int L_hi_v, int L_lo_v, float clip, const uint32_t* bitmap, int tiles_hi,
+                              int tiles_lo,
                               uint32_t* k_hi, uint32_t* v_hi, uint32_t* kz_hi, uint32_t* vz_hi,
                               uint32_t* k_lo, uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo)
 {
     if (D <= 0 || G <= 0 || D % G != 0 || L_hi < 2 || L_lo < 2 || L_hi > 256 || L_lo > 256 ||
-        !(clip > 0.0f && clip <= 1.0f))
+        L_hi_v < 2 || L_lo_v < 2 || L_hi_v > 256 || L_lo_v > 256 || !(clip > 0.0f && clip <= 1.0f))
         return OR_BAD_ARG;
     int status = 0, NG = D / G;
     int tiles[2] = {tiles_hi, tiles_lo};
     int Ls[2] = {L_hi, L_lo};
+    int Lvs[2] = {L_hi_v, L_lo_v};
     uint32_t* kw[2] = {k_hi, k_lo};
     uint32_t* vw[2] = {v_hi, v_lo};
     uint32_t* kz[2] = {kz_hi, kz_lo};
@@ -391,13 +396,13 @@ int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, i
             status |= oracle_quantize_group_clip(K + (size_t)t * D + grp * G, G, Ls[seg], clip,
                                                  ck[seg] + (size_t)slot * D + grp * G, &s16, &z16);
             kz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
-            status |= oracle_quantize_group_clip(V + (size_t)t * D + grp * G, G, Ls[seg], clip,
+            status |= oracle_quantize_group_clip(V + (size_t)t * D + grp * G, G, Lvs[seg], clip,
                                                  cv[seg] + (size_t)slot * D + grp * G, &s16, &z16);
             vz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
         }
     }
     for (int s = 0; s < 2; s++) {
-        pack_segment(ck[s], cv[s], tiles[s], D, Ls[s], kw[s], vw[s]);
+        pack_segment(ck[s], cv[s], tiles[s], D, Ls[s], Lvs[s], kw[s], vw[s]);
         free(ck[s]);
         free(cv[s]);
     }
@@ -407,26 +412,27 @@ int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, i
 /* ------------------------------------------------------------------ dequantize */
 
 /* code of (slot, channel d) of a segment, read back from its packed words */
-static void segment_codes(const uint32_t* kw, const uint32_t* vw, int D, int L, int32_t slot, uint8_t* kc,
+static void segment_codes(const uint32_t* kw, const uint32_t* vw, int D, int Lk, int Lv, int32_t slot, uint8_t* kc,
                           uint8_t* vc)
 {
-    int k = oracle_radix_digits(L);
-    int WK = ceil_div(D, k), WV = ceil_div(OR_TILE, k);
+    int kk = oracle_radix_digits(Lk), kv = oracle_radix_digits(Lv);
+    int WK = ceil_div(D, kk), WV = ceil_div(OR_TILE, kv);
     int tile = slot / OR_TILE, tt = slot % OR_TILE;
-    uint8_t* buf = (uint8_t*)malloc((size_t)k);
+    uint8_t* buf = (uint8_t*)malloc((size_t)(kk > kv ? kk : kv));
     for (int j = 0; j < WK; j++) {
-        oracle_unpack_word(kw[k_word_index(tile, j, tt, WK)], k, L, buf);
-        for (int i = 0; i < k && j * k + i < D; i++) kc[j * k + i] = buf[i];
+        oracle_unpack_word(kw[k_word_index(tile, j, tt, WK)], kk, Lk, buf);
+        for (int i = 0; i < kk && j * kk + i < D; i++) kc[j * kk + i] = buf[i];
     }
     for (int d = 0; d < D; d++) {
-        oracle_unpack_word(vw[v_word_index(tile, tt / k, d, WV, D)], k, L, buf);
-        vc[d] = buf[tt % k];
+        oracle_unpack_word(vw[v_word_index(tile, tt / kv, d, WV, D)], kv, Lv, buf);
+        vc[d] = buf[tt % kv];
     }
     free(buf);
 }
 
 /* x^ = fmaf(c, s, z) for every token of a unit, in original token order.  Khat, Vhat: [T][D]. */
-void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, const uint32_t* bitmap,
+void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, int L_hi_v, int L_lo_v,
+                            const uint32_t* bitmap,
                             const uint32_t* k_hi, const uint32_t* v_hi, const uint32_t* kz_hi,
                             const uint32_t* vz_hi, const uint32_t* k_lo, const uint32_t* v_lo,
                             const uint32_t* kz_lo, const uint32_t* vz_lo, float* Khat, float* Vhat)
@@ -437,6 +443,7 @@ void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, const u
     const uint32_t* kz[2] = {kz_hi, kz_lo};
     const uint32_t* vz[2] = {vz_hi, vz_lo};
     int Ls[2] = {L_hi, L_lo};
+    int Lvs[2] = {L_hi_v, L_lo_v};
     uint8_t* kc = (uint8_t*)malloc((size_t)D);
     uint8_t* vc = (uint8_t*)malloc((size_t)D);
     int32_t next[2] = {0, 0};
@@ -444,7 +451,7 @@ void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, const u
         int seg = ((bitmap[t / 32] >> (t % 32)) & 1u) ? 0 : 1;
         int32_t slot = next[seg]++;
         int tile = slot / OR_TILE, tt = slot % OR_TILE;
-        segment_codes(kw[seg], vw[seg], D, Ls[seg], slot, kc, vc);
+        segment_codes(kw[seg], vw[seg], D, Ls[seg], Lvs[seg], slot, kc, vc);
         for (int d = 0; d < D; d++) {
             int grp = d / G;
             uint32_t kzv = kz[seg][sz_index(tile, grp, tt, NG)];
@@ -471,7 +478,7 @@ void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, const u
  * State (bitmap, rank, n_hi, n_lo) is updated in place.  Returns status bits.
  */
 int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float tau, int D, int G,
-                       int L_hi, int L_lo, float clip, int32_t T_cap, uint32_t* bitmap, uint32_t* rank,
+                       int L_hi, int L_lo, int L_hi_v, int L_lo_v, float clip, int32_t T_cap, uint32_t* bitmap, uint32_t* rank,
                        int32_t* n_hi, int32_t* n_lo, int tiles_hi, int tiles_lo, uint32_t* k_hi,
                        uint32_t* v_hi, uint32_t* kz_hi, uint32_t* vz_hi, uint32_t* k_lo,
                        uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo)
@@ -484,10 +491,10 @@ int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float 
     int32_t slot = hi ? *n_hi : *n_lo;
     int tiles = hi ? tiles_hi : tiles_lo;
     if (slot >= tiles * OR_TILE || T >= T_cap) return status | OR_OVERFLOW;
-    int L = hi ? L_hi : L_lo;
+    int L = hi ? L_hi : L_lo, Lv = hi ? L_hi_v : L_lo_v;
     int NG = D / G;
-    int kdig = oracle_radix_digits(L);
-    int WK = ceil_div(D, kdig), WV = ceil_div(OR_TILE, kdig);
+    int kdig = oracle_radix_digits(L), vdig = oracle_radix_digits(Lv);
+    int WK = ceil_div(D, kdig), WV = ceil_div(OR_TILE, vdig);
     uint32_t* kw = hi ? k_hi : k_lo;
     uint32_t* vw = hi ? v_hi : v_lo;
     uint32_t* kz = hi ? kz_hi : kz_lo;
@@ -495,23 +502,23 @@ int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float 
     (void)seg;
     uint8_t* kc = (uint8_t*)calloc((size_t)WK * kdig, 1);
     uint8_t* vc = (uint8_t*)calloc((size_t)D, 1);
-    uint8_t* buf = (uint8_t*)malloc((size_t)kdig);
+    uint8_t* buf = (uint8_t*)malloc((size_t)vdig);
     int tile = slot / OR_TILE, tt = slot % OR_TILE;
     for (int grp = 0; grp < NG; grp++) {
         uint16_t s16, z16;
         status |= oracle_quantize_group_clip(k + grp * G, G, L, clip, kc + grp * G, &s16, &z16);
         kz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
-        status |= oracle_quantize_group_clip(v + grp * G, G, L, clip, vc + grp * G, &s16, &z16);
+        status |= oracle_quantize_group_clip(v + grp * G, G, Lv, clip, vc + grp * G, &s16, &z16);
         vz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
     }
     for (int j = 0; j < WK; j++) kw[k_word_index(tile, j, tt, WK)] = oracle_pack_word(kc + j * kdig, kdig, L);
     for (int d = 0; d < D; d++) {
         /* rewrite the word that holds this slot with its digit set; other digits unchanged */
-        size_t idx = v_word_index(tile, tt / kdig, d, WV, D);
-        if (tt % kdig == 0) memset(buf, 0, (size_t)kdig); /* first slot of a word: fresh word */
-        else oracle_unpack_word(vw[idx], kdig, L, buf);
-        buf[tt % kdig] = vc[d];
-        vw[idx] = oracle_pack_word(buf, kdig, L);
+        size_t idx = v_word_index(tile, tt / vdig, d, WV, D);
+        if (tt % vdig == 0) memset(buf, 0, (size_t)vdig); /* first slot of a word: fresh word */
+        else oracle_unpack_word(vw[idx], vdig, Lv, buf);
+        buf[tt % vdig] = vc[d];
+        vw[idx] = oracle_pack_word(buf, vdig, Lv);
     }
     if (T % 32 == 0) {
         bitmap[T / 32] = 0;

@@ -146,3 +146,83 @@ def test_clipped_unit_matches_its_groups():
             z = np.uint16(z16).view(np.float16).astype(np.float32)
             ref = (c.astype(np.float32) * s).astype(np.float32) + z
             assert np.allclose(Kh[t, g * G:(g + 1) * G], ref, rtol=0, atol=1e-6 * (1 + abs(float(z))))
+
+
+# ---------------------------------------------------------------- separate V level counts
+
+
+def _digits(w, L, k):
+    out = []
+    for _ in range(k):
+        w, d = divmod(int(w), L)
+        out.append(d)
+    return out
+
+
+def test_separate_v_levels_words_decode_by_hand():
+    """K words in base L_k, V words in base L_v: decoded here with divmod, the codes are those
+    of each token's groups quantized on the tensor's own level count."""
+    r = np.random.default_rng(12)
+    T, D, G, Lh, Ll, Lhv, Llv = 70, 128, 32, 8, 5, 3, 2
+    K = r.standard_normal((T, D)).astype(np.float16).view(np.uint16)
+    V = r.standard_normal((T, D)).astype(np.float16).view(np.uint16)
+    bm, _, nh, _, _ = oracle.select(r.standard_normal(T).astype(np.float32), 0.4)
+    hi, lo, st = oracle.quantize_pack_unit(K, V, bm, G, Lh, Ll, 1, 1, L_hi_v=Lhv, L_lo_v=Llv)
+    assert st == 0
+    assert hi["v"].shape == (1, -(-128 // 20), D) and lo["v"].shape == (1, 4, D)  # k(3) = 20, k(2) = 32
+    slots = {0: 0, 1: 0}
+    for t in range(T):
+        is_hi = (int(bm[t // 32]) >> (t % 32)) & 1
+        seg, Lk, Lv = (hi, Lh, Lhv) if is_hi else (lo, Ll, Llv)
+        slot = slots[is_hi]
+        slots[is_hi] += 1
+        kk, kv = oracle.radix_digits(Lk), oracle.radix_digits(Lv)
+        kc = sum((_digits(seg["k"][0, j, slot], Lk, kk) for j in range(seg["k"].shape[1])), [])[:D]
+        vc = [_digits(seg["v"][0, slot // kv, d], Lv, kv)[slot % kv] for d in range(D)]
+        for g in range(D // G):
+            ck = oracle.quantize_group(K[t, g * G:(g + 1) * G], Lk)[0]
+            cv = oracle.quantize_group(V[t, g * G:(g + 1) * G], Lv)[0]
+            assert kc[g * G:(g + 1) * G] == ck.tolist()
+            assert vc[g * G:(g + 1) * G] == cv.tolist()
+
+
+def test_separate_v_levels_equal_counts_are_the_default():
+    r = np.random.default_rng(13)
+    K = r.standard_normal((150, 128)).astype(np.float16).view(np.uint16)
+    V = r.standard_normal((150, 128)).astype(np.float16).view(np.uint16)
+    bm, _, _, _, _ = oracle.select(r.standard_normal(150).astype(np.float32), 0.3)
+    a = oracle.quantize_pack_unit(K, V, bm, 64, 8, 5, 1, 1)
+    b = oracle.quantize_pack_unit(K, V, bm, 64, 8, 5, 1, 1, L_hi_v=8, L_lo_v=5)
+    for seg in (0, 1):
+        for n in a[seg]:
+            assert np.array_equal(a[seg][n], b[seg][n])
+
+
+def test_separate_v_levels_storage_by_hand():
+    # D 128, G 64.  hi: K L=8 (10 digits/word -> 13 words per row), V L=3 (20 -> 7 words per
+    # 128-slot column); lo: K L=5 (13 -> 10), V L=2 (32 -> 4).  Per value, K and V averaged, plus
+    # 32 bits of scale/zero per group of 64: hi (13 + 7)/2 * 32/128 + 0.5 = 3.0; lo (10 + 4)/2 *
+    # 32/128 + 0.5 = 2.25.  p = 0.25, and the bitmap's 1/256: 0.75 + 1.6875 + 0.00390625.
+    assert oracle.storage_bits_per_value(128, 64, 8, 5, 0.25, 3, 2) == pytest.approx(2.44140625, abs=1e-12)
+    assert oracle.storage_bits_per_value(128, 64, 8, 5, 0.25, 8, 5) == oracle.storage_bits_per_value(128, 64, 8, 5,
+                                                                                                    0.25)
+
+
+def test_separate_v_levels_appends_equal_a_prefill():
+    """Appending tokens one at a time leaves the same buffers as packing them all at once with the
+    same assignment (both with the separate V levels and a clip)."""
+    r = np.random.default_rng(14)
+    T0, T, D, G, Lh, Ll, Lhv, Llv, clip = 100, 180, 128, 64, 6, 4, 3, 2, 0.8
+    K = r.standard_normal((T, D)).astype(np.float16).view(np.uint16)
+    V = r.standard_normal((T, D)).astype(np.float16).view(np.uint16)
+    S = r.standard_normal(T).astype(np.float32)
+    bm, rk, nh, tau, _ = oracle.select(S[:T0], 0.3)
+    hi, lo, _ = oracle.quantize_pack_unit(K[:T0], V[:T0], bm, G, Lh, Ll, 2, 2, clip=clip, L_hi_v=Lhv, L_lo_v=Llv)
+    st = oracle.UnitState(256, bm, rk, nh, T0 - nh, tau, hi, lo)
+    for t in range(T0, T):
+        assert oracle.append_unit(st, K[t], V[t], S[t], G, Lh, Ll, clip, Lhv, Llv) == 0
+    hi2, lo2, _ = oracle.quantize_pack_unit(K, V, st.bitmap[:(T + 31) // 32], G, Lh, Ll, 2, 2, clip=clip,
+                                            L_hi_v=Lhv, L_lo_v=Llv)
+    for a, b in ((st.hi, hi2), (st.lo, lo2)):
+        for n in a:
+            assert np.array_equal(a[n], b[n]), n
