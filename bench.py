@@ -60,21 +60,25 @@ def radix_words(L: int, n: int = 128) -> int:
 # this library's kernel launches in one step: select 1, quantize 1, append+decode 3 (the hi and lo
 # segments, then the merge); the committed ncu launch list of the step shows the same kernels
 LAUNCHES_PER_STEP = 5
-# the quantizer variants timed beside the step (recent window of the selection; clipped range)
-WINDOW, CLIP = 128, 0.9
+# the quantizer variants timed beside the step (recent window of the selection; clipped range; V
+# level counts of their own for the hi and lo segments)
+WINDOW, CLIP, V_LEVELS = 128, 0.9, (5, 3)
 
 
-def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False) -> dict:
+def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False, v_levels=None) -> dict:
     """Algorithmic bytes of one layer, per hot-path step (measurement).  With
     `appended`, one generated token per unit follows the prefill (`new_hi` of them on the L_hi grid)
-    and the decode reads the cache including it."""
+    and the decode reads the cache including it.  v_levels: the V level counts of the two segments,
+    when they differ from the K ones."""
     units = w.B * w.H
     ng = w.D // w.G
-    rec = lambda L: 2 * (4 * radix_words(L, w.D) + 4 * ng)  # noqa: E731  K + V record of one token
-    cache = units * (n_hi * rec(w.L_hi) + (T - n_hi) * rec(w.L_lo))
+    lv_hi, lv_lo = v_levels or (w.L_hi, w.L_lo)
+    # K + V record of one token: K words of its row, its share of the V column words, scale/zero
+    rec = lambda L, Lv: 4 * radix_words(L, w.D) + 4 * radix_words(Lv) * w.D // 128 + 2 * 4 * ng  # noqa: E731
+    cache = units * (n_hi * rec(w.L_hi, lv_hi) + (T - n_hi) * rec(w.L_lo, lv_lo))
     bitmap_rank = units * 2 * 4 * ((T + 31) // 32)
     q = w.B * w.Hq * w.D * 2
-    new = new_hi * rec(w.L_hi) + (units - new_hi) * rec(w.L_lo) if appended else 0
+    new = new_hi * rec(w.L_hi, lv_hi) + (units - new_hi) * rec(w.L_lo, lv_lo) if appended else 0
     return {
         "select": units * 4 * T + bitmap_rank,
         "quantize": units * T * w.D * 2 * 2 + bitmap_rank + cache,
@@ -424,6 +428,23 @@ def run_semkv(args):
 
     t_win = timed(win_graph)
     t_clip = timed(clip_graph, before=(graphs[0],))
+    # V level counts of their own: quantize (generic kernel) and decode (CUDA-core decode)
+    cache.struct.L_hi_v, cache.struct.L_lo_v = V_LEVELS
+    calls[0]()
+    calls[1]()
+    kvq_graph, kvd_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(kvq_graph, capture_error_mode="relaxed"):
+        calls[1]()
+    out_v = torch.empty_like(out)
+    kv_decode = lambda: semkv_decode_attention(cache, q, scale, out_v, ws)  # noqa: E731
+    kv_decode()
+    with torch.cuda.graph(kvd_graph, capture_error_mode="relaxed"):
+        kv_decode()
+    cache.struct.L_hi_v, cache.struct.L_lo_v = 0, 0
+    torch.cuda.synchronize()
+    t_kvq = timed(kvq_graph, before=(graphs[0],))
+    t_kvd = timed(kvd_graph, before=(graphs[0], kvq_graph))
+    nb_kv = alg_bytes(w, T, n_hi0, v_levels=V_LEVELS)
     assert cache.status() == 0, f"device status {cache.status()}"
     assert torch.equal(out, out_s), "append+decode in one pass differs from append then decode"
     # leave the cache as a timed step leaves it (prefill + the fixed-threshold append)
@@ -460,6 +481,8 @@ def run_semkv(args):
         "append_decode": {"ms": t_fused, "gbs": (nb["append"] + nb["decode"]) / (t_fused * 1e-3) / 1e9},
         f"select_window{WINDOW}": {"ms": t_win, "gbs": nb["select"] / (t_win * 1e-3) / 1e9},
         f"quantize_clip{CLIP}": {"ms": t_clip, "gbs": nb["quantize"] / (t_clip * 1e-3) / 1e9},
+        "quantize_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvq, "gbs": nb_kv["quantize"] / (t_kvq * 1e-3) / 1e9},
+        "decode_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvd, "gbs": nb_kv["decode"] / (t_kvd * 1e-3) / 1e9},
     })
     dom = max(("select", "quantize", "append_decode"), key=lambda k: per_kernel[k]["ms"])
     dom_name = {"select": "semkv_assign_precision (k_select_cluster)",

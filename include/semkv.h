@@ -101,9 +101,14 @@ typedef struct semkv_cache {
      *           scaled by clip in fp32 (clipped range), the zero is the nearest binary16 of the
      *           scaled min (-0 stored as +0), the scale is fp16 rounded up of
      *           (clip*max - zero)/(L - 1) (at least 0); values outside take the end codes.  Used by
-     *           semkv_quantize_pack and every append.  Other values: SEMKV_ERR_INVALID_ARG. */
+     *           semkv_quantize_pack and every append.  Other values: SEMKV_ERR_INVALID_ARG.
+     *   L_hi_v, L_lo_v: level counts of the V codes of each segment (keys and values at different
+     *           bit widths); 0 = the K level count (L_hi, L_lo), else in [2, 256].  The V words of a
+     *           segment then hold k(L_v) codes each.  The tensor-core decode serves equal K and V
+     *           counts; other segments run on the CUDA-core decode. */
     int32_t window;
     float clip;
+    int32_t L_hi_v, L_lo_v;
     uint32_t *k_hi, *v_hi, *kz_hi, *vz_hi;
     uint32_t *k_lo, *v_lo, *kz_lo, *vz_lo;
     uint32_t *bitmap, *rank;
@@ -227,15 +232,19 @@ SEMKV_API const char* semkv_status_string(int code);
 SEMKV_API int32_t semkv_radix_digits(int32_t L);
 
 /* Fraction of tokens the finer grid can take under a storage budget (SemKV page, Abstract: measure
- * the quality cliff, then interpolate above it).  Physical bits per cached value are
- *   bits(p) = [p*32*W(L_hi) + (1-p)*32*W(L_lo)]/D + 32/G + 1/(2D)
- * (code words, fp16 scale + zero per group, the precision bitmap shared by K and V), with
- * W(L) = ceil(D/k(L)) words per row.  *p receives the largest p in [0,1] with 16/bits(p) >= ratio,
+ * the quality cliff, then interpolate above it).  Physical bits per cached value (K and V
+ * averaged) are
+ *   bits(p) = p*B(L_hi, L_hi_v) + (1-p)*B(L_lo, L_lo_v) + 32/G + 1/(2D),
+ *   B(Lk, Lv) = 16*ceil(D/k(Lk))/D + 16*ceil(128/k(Lv))/128
+ * (K code words per row, V code words per 128-slot column, fp16 scale + zero per group, the
+ * precision bitmap shared by K and V).  semkv_p_for_ratio uses L_hi_v = L_hi, L_lo_v = L_lo.  *p receives the largest p in [0,1] with 16/bits(p) >= ratio,
  * to be passed to semkv_assign_precision (which puts floor(p*T) tokens on the finer grid, never
  * more).  Pure host function.  Returns SEMKV_ERR_INVALID_ARG (null p, ratio not > 0, D or G not
  * positive, G not dividing D), SEMKV_ERR_UNSUPPORTED (L outside [2, 256]) or SEMKV_ERR_CAPACITY
  * (even p = 0 gives a smaller reduction than `ratio`). */
 SEMKV_API int semkv_p_for_ratio(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, double ratio, double* p);
+SEMKV_API int semkv_p_for_ratio_kv(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, int32_t L_hi_v, int32_t L_lo_v,
+                                   double ratio, double* p);
 
 #ifdef __cplusplus
 }

@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     semkv_dequantize,
     semkv_quantize_pack,
     semkv_p_for_ratio,
+    semkv_p_for_ratio_kv,
     semkv_radix_digits,
     semkv_workspace_bytes,
     status_string,

@@ -31,13 +31,14 @@ BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
             "semkv_append_token", "semkv_append_token_running", "semkv_append_decode", "semkv_decode_attention",
             "semkv_decode_attention_noalloc", "semkv_dequantize", "semkv_status_string", "semkv_radix_digits",
-            "semkv_p_for_ratio")
+            "semkv_p_for_ratio", "semkv_p_for_ratio_kv")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
 class CacheStruct(ctypes.Structure):
-    """Mirror of semkv_cache_t (window, clip: the quantizer variants; 0 = off)."""
-    _fields_ = [(n, ctypes.c_int32) for n in SHAPE_FIELDS] + [("window", ctypes.c_int32), ("clip", ctypes.c_float)] + \
+    """Mirror of semkv_cache_t (window, clip, L_hi_v, L_lo_v: the quantizer variants; 0 = off)."""
+    _fields_ = [(n, ctypes.c_int32) for n in SHAPE_FIELDS] + \
+        [("window", ctypes.c_int32), ("clip", ctypes.c_float), ("L_hi_v", ctypes.c_int32), ("L_lo_v", ctypes.c_int32)] + \
         [(n, ctypes.c_void_p) for n in BUF_NAMES]
 
 
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.semkv_radix_digits.argtypes = [i32]
         L.semkv_radix_digits.restype = i32
         L.semkv_p_for_ratio.argtypes = [i32, i32, i32, i32, ctypes.c_double, ctypes.POINTER(ctypes.c_double)]
+        L.semkv_p_for_ratio_kv.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_double,
+                                           ctypes.POINTER(ctypes.c_double)]
         for n in EXPORTED:
             if n not in ("semkv_status_string", "semkv_radix_digits"):
                 getattr(L, n).restype = ctypes.c_int
@@ -116,6 +119,14 @@ def semkv_p_for_ratio(D: int, G: int, L_hi: int, L_lo: int, ratio: float) -> flo
     p = ctypes.c_double()
     _check("semkv_p_for_ratio", lib().semkv_p_for_ratio(int(D), int(G), int(L_hi), int(L_lo), float(ratio),
                                                        ctypes.byref(p)))
+    return p.value
+
+
+def semkv_p_for_ratio_kv(D: int, G: int, L_hi: int, L_lo: int, L_hi_v: int, L_lo_v: int, ratio: float) -> float:
+    """semkv_p_for_ratio with V level counts of their own."""
+    p = ctypes.c_double()
+    _check("semkv_p_for_ratio_kv", lib().semkv_p_for_ratio_kv(int(D), int(G), int(L_hi), int(L_lo), int(L_hi_v),
+                                                             int(L_lo_v), float(ratio), ctypes.byref(p)))
     return p.value
 
 

@@ -25,6 +25,7 @@ int validate_shape(const semkv_cache_t* c)
     if (c->G != 8 && c->G != 16 && c->G != 32 && c->G != 64 && c->G != 128) return SEMKV_ERR_UNSUPPORTED;
     if (c->Hq / c->H > 8) return SEMKV_ERR_UNSUPPORTED;
     if (c->window < 0 || !(c->clip == 0.0f || (c->clip > 0.0f && c->clip <= 1.0f))) return SEMKV_ERR_INVALID_ARG;
+    if ((c->L_hi_v && !level_ok(c->L_hi_v)) || (c->L_lo_v && !level_ok(c->L_lo_v))) return SEMKV_ERR_UNSUPPORTED;
     return SEMKV_OK;
 }
 
@@ -93,6 +94,7 @@ SegView seg_view(const semkv_cache_t* c, bool hi)
     s.vz = hi ? c->vz_hi : c->vz_lo;
     s.n = hi ? c->n_hi : c->n_lo;
     s.L = hi ? c->L_hi : c->L_lo;
+    s.Lv = level_v(*c, hi);
     s.tiles_cap = (hi ? c->cap_hi : c->cap_lo) / TILE;
     s.is_hi = hi ? 1 : 0;
     return s;
@@ -128,7 +130,7 @@ static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_
         const SegView sv = seg_view(c, hi != 0);
         const int ns = hi ? nh : nl, off = hi ? 0 : nh;
         if (ns == 0) continue;
-        if (decode_tc_supported(sv.L, c->G, g)) {
+        if (sv.L == sv.Lv && decode_tc_supported(sv.L, c->G, g)) {
             launch_decode_tc(sv, q, units, c->H, g, c->G, scale_log2, ns, off, nh + nl, ws, c->status, dependent, app,
                              st);
         } else {
@@ -148,11 +150,20 @@ int32_t semkv_radix_digits(int32_t L) { return level_ok(L) ? radix_k(L) : 0; }
 
 int semkv_p_for_ratio(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, double ratio, double* p)
 {
+    return semkv_p_for_ratio_kv(D, G, L_hi, L_lo, L_hi, L_lo, ratio, p);
+}
+
+int semkv_p_for_ratio_kv(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, int32_t L_hi_v, int32_t L_lo_v,
+                         double ratio, double* p)
+{
     if (!p || !(ratio > 0.0) || !std::isfinite(ratio) || D < 1 || G < 1 || D % G) return SEMKV_ERR_INVALID_ARG;
-    if (!level_ok(L_hi) || !level_ok(L_lo)) return SEMKV_ERR_UNSUPPORTED;
+    if (!level_ok(L_hi) || !level_ok(L_lo) || !level_ok(L_hi_v) || !level_ok(L_lo_v)) return SEMKV_ERR_UNSUPPORTED;
     // bits(p) = a + b p, linear in p; the budget is 16 / ratio bits per value
-    const double w_hi = ceil_div(D, radix_k(L_hi)), w_lo = ceil_div(D, radix_k(L_lo));
-    const double a = 32.0 * w_lo / D + 32.0 / G + 1.0 / (2.0 * D), b = 32.0 * (w_hi - w_lo) / D;
+    auto seg_bits = [&](int Lk, int Lv) {  // K words per row and V words per 128-slot column, averaged
+        return 16.0 * ceil_div(D, radix_k(Lk)) / D + 16.0 * ceil_div(TILE, radix_k(Lv)) / TILE;
+    };
+    const double b_hi = seg_bits(L_hi, L_hi_v), b_lo = seg_bits(L_lo, L_lo_v);
+    const double a = b_lo + 32.0 / G + 1.0 / (2.0 * D), b = b_hi - b_lo;
     const double budget = 16.0 / ratio;
     if (a + b <= budget) {  // p = 1 fits (also every b <= 0 case that fits at all)
         *p = 1.0;
@@ -172,11 +183,11 @@ int semkv_cache_bytes(const semkv_cache_t* c, size_t sizes[SEMKV_NBUF])
     const size_t units = (size_t)c->B * c->H, ng = (size_t)(c->D / c->G);
     const size_t th = (size_t)c->cap_hi / TILE, tl = (size_t)c->cap_lo / TILE;
     sizes[SEMKV_BUF_K_HI] = units * th * words_row(c->L_hi) * TILE * 4;
-    sizes[SEMKV_BUF_V_HI] = units * th * words_col(c->L_hi) * c->D * 4;
+    sizes[SEMKV_BUF_V_HI] = units * th * words_col(level_v(*c, true)) * c->D * 4;
     sizes[SEMKV_BUF_KZ_HI] = units * th * ng * TILE * 4;
     sizes[SEMKV_BUF_VZ_HI] = sizes[SEMKV_BUF_KZ_HI];
     sizes[SEMKV_BUF_K_LO] = units * tl * words_row(c->L_lo) * TILE * 4;
-    sizes[SEMKV_BUF_V_LO] = units * tl * words_col(c->L_lo) * c->D * 4;
+    sizes[SEMKV_BUF_V_LO] = units * tl * words_col(level_v(*c, false)) * c->D * 4;
     sizes[SEMKV_BUF_KZ_LO] = units * tl * ng * TILE * 4;
     sizes[SEMKV_BUF_VZ_LO] = sizes[SEMKV_BUF_KZ_LO];
     sizes[SEMKV_BUF_BITMAP] = units * (size_t)(c->T_cap / 32) * 4;
@@ -262,7 +273,8 @@ int semkv_append_decode(const semkv_cache_t* c, const uint16_t* k, const uint16_
     if (r != SEMKV_OK) return r;
     if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
     const int g = c->Hq / c->H;
-    if (!decode_tc_supported(c->L_hi, c->G, g) || !decode_tc_supported(c->L_lo, c->G, g)) {
+    if (level_v(*c, true) != c->L_hi || level_v(*c, false) != c->L_lo || !decode_tc_supported(c->L_hi, c->G, g) ||
+        !decode_tc_supported(c->L_lo, c->G, g)) {
         // shapes the fused path does not cover: the two calls, in order
         launch_append(*c, k, v, score, -1.0f, (cudaStream_t)stream);
         r = launch_status();

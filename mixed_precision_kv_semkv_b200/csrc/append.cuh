@@ -26,9 +26,9 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
     __shared__ int kc[D + 32];
     __shared__ float gmn[2][4], gmx[2][4];  // per-warp partial extrema of groups wider than a warp
     const int slot = hi ? nh : nl;
-    const int L = hi ? c.L_hi : c.L_lo;
-    const int k = radix_k(L);
-    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
+    const int L = hi ? c.L_hi : c.L_lo, Lv = level_v(c, hi);
+    const int k = radix_k(L), kv = radix_k(Lv);
+    const int WK = ceil_div(D, k), WV = ceil_div(TILE, kv);
     const int tile = slot / TILE, tt = slot % TILE;
     const int tiles_cap = (hi ? c.cap_hi : c.cap_lo) / TILE;
     const size_t tb = (size_t)u * tiles_cap + tile;
@@ -66,14 +66,14 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
     const float clip = clip_ratio(c);
     uint16_t ks16, kz16, vs16, vz16;
     group_scale_zero(kmn, kmx, L, clip, ks16, kz16);
-    group_scale_zero(vmn, vmx, L, clip, vs16, vz16);
+    group_scale_zero(vmn, vmx, Lv, clip, vs16, vz16);
     const int grp = d / G;
     if (d % G == 0) {
         kz[grp * TILE + tt] = (uint32_t)ks16 | ((uint32_t)kz16 << 16);
         vz[grp * TILE + tt] = (uint32_t)vs16 | ((uint32_t)vz16 << 16);
     }
     kc[d] = quant_code(kx, h2f(kz16), h2f(ks16), L);
-    const uint32_t cv = (uint32_t)quant_code(vx, h2f(vz16), h2f(vs16), L);
+    const uint32_t cv = (uint32_t)quant_code(vx, h2f(vz16), h2f(vs16), Lv);
     const bool bad = !isfinite(kx) || !isfinite(vx);
     __syncthreads();
 
@@ -85,13 +85,13 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
     {
         // V channel d: a fresh word at the first slot of a word; otherwise the digit is added in
         // place (it was zero), with a reduction that needs no read
-        const int pos = tt % k;
-        uint32_t* p = vw + (size_t)(tt / k) * D + d;
+        const int pos = tt % kv;
+        uint32_t* p = vw + (size_t)(tt / kv) * D + d;
         if (pos == 0) {
             *p = cv;
         } else {
             uint32_t pw = 1u;
-            for (int i = 0; i < pos; ++i) pw *= (uint32_t)L;
+            for (int i = 0; i < pos; ++i) pw *= (uint32_t)Lv;
             atomicAdd(p, cv * pw);
         }
     }

@@ -43,14 +43,14 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
                                                        float* __restrict__ ws)
 {
     constexpr int D = 128;
-    const int L = LC ? LC : seg.L;
-    const int k = LC ? radix_k(LC) : radix_k(seg.L);
-    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
+    const int L = LC ? LC : seg.L, Lv = LC ? LC : seg.Lv;  // LC > 0 only when K and V share it
+    const int k = LC ? radix_k(LC) : radix_k(seg.L), kv = LC ? radix_k(LC) : radix_k(seg.Lv);
+    const int WK = ceil_div(D, k), WV = ceil_div(TILE, kv);
     const int NG = D / G, NGg = NG * g;
     const int split = blockIdx.x, u = blockIdx.y;
     const int b = u / H, hk = u % H, Hq = H * g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float mid = 0.5f * (float)(L - 1);
+    const float mid = 0.5f * (float)(L - 1), mid_v = 0.5f * (float)(Lv - 1);
 
     extern __shared__ __align__(16) float dsm[];
     float* qs = dsm;                 // [D][GMAX]
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
         for (int grp = 0; grp < NG; ++grp) {
             const uint32_t zz = vz[grp * TILE + tid];
             const float s = h2f((uint16_t)(zz & 0xffffu));
-            const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(zz >> 16)));
+            const float zc = __fmaf_rn(mid_v, s, h2f((uint16_t)(zz >> 16)));
             for (int h = 0; h < g; ++h) {  // slots past n may hold stale scale/zero bits: write zeros
                 Pv[tid * NGg + grp * g + h] = valid ? p[h] * s : 0.f;
                 part[tid * NGg + grp * g + h] = valid ? p[h] * zc : 0.f;
@@ -173,13 +173,13 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
         for (int h = 0; h < GMAX; ++h) acc[h] *= alpha[h];
         for (int w = 0; w < WV; ++w) {
             int dg[32];
-            digits_of<LC>(vw[w * D + tid], L, k, dg);
+            digits_of<LC>(vw[w * D + tid], Lv, kv, dg);
 #pragma unroll
             for (int i = 0; i < (LC ? Radix<(LC ? LC : 2)>::k : 32); ++i) {
-                if (i >= k) break;
-                const int t = w * k + i;
+                if (i >= kv) break;
+                const int t = w * kv + i;
                 if (t >= TILE) break;
-                const float cf = (float)dg[i] - mid;
+                const float cf = (float)dg[i] - mid_v;
                 const float* pv = Pv + t * NGg + grp_d * g;
 #pragma unroll
                 for (int h = 0; h < GMAX; ++h)
@@ -303,6 +303,10 @@ void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H
 {
     (void)D;
     if (nsplit == 0 || units == 0) return;
+    if (seg.Lv != seg.L) {  // V level count of its own: both radixes at run time
+        launch_ds<0>(seg, q, units, H, g, G, scale_log2, nsplit, split_off, nsplit_total, ws, st);
+        return;
+    }
     switch (seg.L) {
 #define SEMKV_D(LL) \
     case LL: launch_ds<LL>(seg, q, units, H, g, G, scale_log2, nsplit, split_off, nsplit_total, ws, st); break;

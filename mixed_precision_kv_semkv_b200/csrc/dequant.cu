@@ -28,9 +28,9 @@ __global__ void __launch_bounds__(128) k_dequantize(semkv_cache_t c, int T, floa
     const bool hi = (word >> (t % 32)) & 1u;
     const int below = (int)r + __popc(word & ((1u << (t % 32)) - 1u));
     const int slot = hi ? below : t - below;
-    const int L = hi ? c.L_hi : c.L_lo;
-    const int k = radix_k(L);
-    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
+    const int L = hi ? c.L_hi : c.L_lo, Lv = level_v(c, hi);
+    const int k = radix_k(L), kv = radix_k(Lv);
+    const int WK = ceil_div(D, k), WV = ceil_div(TILE, kv);
     const int tiles_cap = (hi ? c.cap_hi : c.cap_lo) / TILE;
     if (slot >= tiles_cap * TILE) {  // state inconsistent with the capacity: leave the row
         atomicOr(c.status, SEMKV_STATUS_LENGTH_MISMATCH);
@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(128) k_dequantize(semkv_cache_t c, int T, floa
     for (int d = 0; d < D; ++d) {
         const uint32_t kzv = kz[(d / G) * TILE + tt], vzv = vz[(d / G) * TILE + tt];
         const int ck = digit_rt(kw[(d / k) * TILE + tt], L, d % k);
-        const int cv = digit_rt(vw[(tt / k) * D + d], L, tt % k);
+        const int cv = digit_rt(vw[(tt / kv) * D + d], Lv, tt % kv);
         ko[d] = __fmaf_rn((float)ck, h2f((uint16_t)(kzv & 0xffffu)), h2f((uint16_t)(kzv >> 16)));
         vo[d] = __fmaf_rn((float)cv, h2f((uint16_t)(vzv & 0xffffu)), h2f((uint16_t)(vzv >> 16)));
     }

@@ -8,6 +8,12 @@
 
 namespace semkv {
 
+// The V level count of a segment: 0 (unset) means the K level count.
+__host__ __device__ __forceinline__ int level_v(const semkv_cache_t& c, bool hi)
+{
+    return hi ? (c.L_hi_v ? c.L_hi_v : c.L_hi) : (c.L_lo_v ? c.L_lo_v : c.L_lo);
+}
+
 // The clip ratio a cache asks for: 0 (unset) means 1, the plain min/max grid.
 __host__ __device__ __forceinline__ float clip_ratio(const semkv_cache_t& c) { return c.clip == 0.0f ? 1.0f : c.clip; }
 
@@ -18,7 +24,8 @@ struct SegView {
     uint32_t* kz;   // [units][tiles_cap][NG][128]
     uint32_t* vz;   // [units][tiles_cap][NG][128]
     int32_t* n;     // [units] tokens in the segment
-    int L;          // levels
+    int L;          // levels of the K codes
+    int Lv;         // levels of the V codes
     int tiles_cap;  // capacity in tiles of 128 slots
     int is_hi;      // 1: L_hi segment (bitmap bit 1), 0: L_lo segment
 };

@@ -35,6 +35,7 @@ struct QuantSeg {
     const int32_t* map;  // slot -> token of unit 0; unit u at + u * map_stride
     int map_stride;
     int L, k_digits, tiles_cap, is_hi;
+    int Lv, kv_digits;  // V codes: level count and codes per word
 };
 
 __device__ __forceinline__ void half8(const uint16_t* p, float (&f)[8])
@@ -120,8 +121,8 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     const bool is_hi = tile < hi.tiles_cap;
     const QuantSeg& seg = is_hi ? hi : lo;
     if (!is_hi) tile -= hi.tiles_cap;
-    const int L = seg.L, k = seg.k_digits;
-    const int WK = ceil_div(D, k), WV = ceil_div(TILE, k);
+    const int L = seg.L, k = seg.k_digits, Lv = seg.Lv, kv = seg.kv_digits;
+    const int WK = ceil_div(D, k), WV = ceil_div(TILE, kv);
     const int NG = D / G;
     const int tid = threadIdx.x;
     const int n = seg.n[u];
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     uint32_t* vw = seg.v + tile_base * WV * D;
     uint32_t* kz = seg.kz + tile_base * NG * TILE;
     uint32_t* vz = seg.vz + tile_base * NG * TILE;
-    const float top = (float)(L - 1);
+    const float top = (float)(L - 1), top_v = (float)(Lv - 1);
     bool bad = false;
 
     // ---- K row `tid`: groups and channels from the top, Horner into words
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
                 }
             }
             uint32_t packed;
-            const Grid g = make_grid(mn, mx, L, clip, &packed);
+            const Grid g = make_grid(mn, mx, Lv, clip, &packed);
             vgrid[tid * NG + grp] = make_float4(g.s, g.r, g.z, 0.0f);
             vz[grp * TILE + tid] = packed;
         }
@@ -210,16 +211,16 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     {
         const int d = tid, grp = d / G;
         uint32_t w = 0u;
-        int widx = (TILE - 1) / k, dig = (TILE - 1) % k;
+        int widx = (TILE - 1) / kv, dig = (TILE - 1) % kv;
         for (int t = TILE - 1; t >= 0; --t) {
             const float4 gg = vgrid[t * NG + grp];
             const Grid g = {gg.x, gg.y, gg.z};
-            w = w * (uint32_t)L + code_of(h2f(Vs[t * QROW + d]), g, top);
+            w = w * (uint32_t)Lv + code_of(h2f(Vs[t * QROW + d]), g, top_v);
             if (dig == 0) {
                 vw[widx * D + d] = w;
                 w = 0u;
                 --widx;
-                dig = k - 1;
+                dig = kv - 1;
             } else {
                 --dig;
             }
@@ -478,6 +479,8 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
         q.n = s.n;
         q.L = s.L;
         q.k_digits = radix_k(s.L);
+        q.Lv = s.Lv;
+        q.kv_digits = radix_k(s.Lv);
         q.tiles_cap = s.tiles_cap;
         q.is_hi = s.is_hi;
         q.map = map;
@@ -487,9 +490,10 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     const unsigned grid = (unsigned)units * per_unit;
     const QuantSeg qh = conv(shi, slot_token), ql = conv(slo, slot_token + shi.tiles_cap * TILE);
     // compile-time level pairs and group sizes of the common configurations
-    // (the clipped-range variant needs codes clamped from below, which only the generic kernel does)
+    // (the clipped-range variant needs codes clamped from below, and V level counts of their own
+    // need a second radix: both only in the generic kernel)
 #define SEMKV_QF(LH, LL, GG)                                                                                  \
-    if (clip == 1.0f && shi.L == LH && slo.L == LL && G == GG) {                                                              \
+    if (clip == 1.0f && shi.Lv == shi.L && slo.Lv == slo.L && shi.L == LH && slo.L == LL && G == GG) {                                                              \
         const size_t sm = (size_t)TILE * QROW * 2;                                                            \
         cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
         k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, status);                      \

@@ -26,9 +26,10 @@ def unit_views(cache: SemkvCache, bufs: dict, u: int):
     B, H, G, D = cache.B, cache.H, cache.G, cache.D
     units = B * H
     out = {}
-    for seg, L, cap in (("hi", cache.L_hi, cache.cap_hi), ("lo", cache.L_lo, cache.cap_lo)):
+    for seg, L, Lv, cap in (("hi", cache.L_hi, cache.L_hi_v, cache.cap_hi), ("lo", cache.L_lo, cache.L_lo_v,
+                                                                             cache.cap_lo)):
         tiles = cap // 128
-        sh = oracle.segment_shapes(D, G, L, tiles)
+        sh = oracle.segment_shapes(D, G, L, tiles, Lv)
         d = {}
         for name in ("k", "v", "kz", "vz"):
             arr = bufs[f"{name}_{seg}"].view(np.uint32)
@@ -54,12 +55,13 @@ def fetch(cache: SemkvCache) -> dict:
     return {n: t.cpu().numpy() for n, t in cache.bufs.items()}
 
 
-def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0):
+def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0, L_hi_v=0, L_lo_v=0):
     import torch
 
     B, H, T, D = K.shape
     Hq = q.shape[1]
-    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra, window=window, clip=clip).poison()
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra, window=window, clip=clip,
+                                   L_hi_v=L_hi_v, L_lo_v=L_lo_v).poison()
     dK, dV, dS, dq = to_dev(K), to_dev(V), to_dev(S), to_dev(q)
     semkv_assign_precision(cache, dS, T, p)
     semkv_quantize_pack(cache, dK, dV, T)
@@ -74,14 +76,14 @@ def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0):
     return res
 
 
-def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo, window=0, clip=0.0):
-    """Oracle results of one unit. K, V [T][D] fp16; S [T]; q [g][D] fp16.  window, clip: the
-    quantizer variants as the cache fields state them (clip 0 = 1 = off)."""
+def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo, window=0, clip=0.0, L_hi_v=0, L_lo_v=0):
+    """Oracle results of one unit. K, V [T][D] fp16; S [T]; q [g][D] fp16.  window, clip, L_hi_v,
+    L_lo_v: the quantizer variants as the cache fields state them (0 = off)."""
     bm, rk, nh, tau, st = oracle.select(S, p, window=window)
     hi, lo, st2 = oracle.quantize_pack_unit(K.view(np.uint16), V.view(np.uint16), bm, G, L_hi, L_lo, tiles_hi,
-                                            tiles_lo, clip=clip or 1.0)
+                                            tiles_lo, clip=clip or 1.0, L_hi_v=L_hi_v or None, L_lo_v=L_lo_v or None)
     T = K.shape[0]
-    Kh, Vh = oracle.dequantize_unit(T, K.shape[1], G, L_hi, L_lo, bm, hi, lo)
+    Kh, Vh = oracle.dequantize_unit(T, K.shape[1], G, L_hi, L_lo, bm, hi, lo, L_hi_v or None, L_lo_v or None)
     o = oracle.attention_fp64(q.view(np.uint16), Kh, Vh, scale)
     return {"bitmap": bm, "rank": rk, "n_hi": nh, "tau": tau, "hi": hi, "lo": lo, "Kh": Kh, "Vh": Vh, "out": o,
             "status": st | st2}
@@ -94,7 +96,8 @@ def _words_equal(a, b, what):
                              f"gpu={a[tuple(bad[0])]:#x} oracle={b[tuple(bad[0])]:#x}")
 
 
-def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = "", strict_tail: bool = True):
+def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = "", strict_tail: bool = True,
+                  L_hi_v: int = 0, L_lo_v: int = 0):
     """Bit-exact comparison of one unit's state.  strict_tail: the last tile's slots past n must be
     zero as well (true after a prefill; after appends into a new tile they are unspecified, except
     that V words holding a live slot have zero digits past n)."""
@@ -108,7 +111,7 @@ def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = "
         tokens = np.arange(T)
         assert np.array_equal(g["slot_hi"][: o["n_hi"]], tokens[bits]), f"slot map hi {where}"
         assert np.array_equal(g["slot_lo"][: T - o["n_hi"]], tokens[~bits]), f"slot map lo {where}"
-    for seg, n, L in (("hi", o["n_hi"], L_hi), ("lo", T - o["n_hi"], L_lo)):
+    for seg, n, L in (("hi", o["n_hi"], L_hi_v or L_hi), ("lo", T - o["n_hi"], L_lo_v or L_lo)):  # L: V's
         if strict_tail:
             nt = -(-n // 128)
             for name in ("k", "v", "kz", "vz"):
@@ -134,11 +137,11 @@ def attention_errors(got, ref):
     return max_abs, rel
 
 
-def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0.0):
+def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0.0, L_hi_v=0, L_lo_v=0):
     """Run the GPU path on a whole case and compare the chosen units (default: all) with the oracle."""
     B, H, T, D = K.shape
     g = q.shape[1] // H
-    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, window=window, clip=clip)
+    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, window=window, clip=clip, L_hi_v=L_hi_v, L_lo_v=L_lo_v)
     cache = res["cache"]
     assert res["status"] == 0, f"status {res['status']}"
     units = range(B * H) if units is None else units
@@ -146,9 +149,10 @@ def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0
     for u in units:
         b, h = divmod(u, H)
         o = oracle_unit(K[b, h], V[b, h], S[b, h], q[b, h * g:(h + 1) * g], p, G, L_hi, L_lo, scale,
-                        cache.cap_hi // 128, cache.cap_lo // 128, window=window, clip=clip)
+                        cache.cap_hi // 128, cache.cap_lo // 128, window=window, clip=clip, L_hi_v=L_hi_v,
+                        L_lo_v=L_lo_v)
         gu = unit_views(cache, res["bufs"], u)
-        compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}")
+        compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}", L_hi_v=L_hi_v, L_lo_v=L_lo_v)
         assert np.array_equal(res["Kh"][b, h].view(np.uint32), o["Kh"].view(np.uint32)), f"Khat unit {u}"
         assert np.array_equal(res["Vh"][b, h].view(np.uint32), o["Vh"].view(np.uint32)), f"Vhat unit {u}"
         ma, rl = attention_errors(res["out"][b, h * g:(h + 1) * g], o["out"])

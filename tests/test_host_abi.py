@@ -65,6 +65,7 @@ def test_cache_bytes_match_oracle_layout(semkv, orc, L_hi, L_lo, G):
     (dict(Hq=30), 1), (dict(G=48), 1), (dict(cap_hi=100), 1), (dict(T_cap=1000), 1), (dict(B=0), 1),
     (dict(D=64, G=64), 2), (dict(L_hi=257), 2), (dict(L_lo=1), 2), (dict(G=4), 2), (dict(Hq=8 * 16), 2),
     (dict(window=-1), 1), (dict(clip=1.5), 1), (dict(clip=-0.25), 1), (dict(clip=float("nan")), 1),
+    (dict(L_hi_v=1), 2), (dict(L_lo_v=257), 2), (dict(L_hi_v=-3), 2),
 ])
 def test_bad_shapes_are_rejected(semkv, bad, code):
     with pytest.raises(semkv.SemkvError) as e:
@@ -105,6 +106,19 @@ def test_calls_fail_before_any_launch(semkv):
     assert L.semkv_decode_attention(ref, one, ctypes.c_float(0.1), one, one, 0, nul) == 1  # workspace too small
     assert L.semkv_dequantize(ref, one, nul, 10, nul) == 1
     assert semkv.status_string(3) == "SEMKV_ERR_CAPACITY"
+
+
+@pytest.mark.parametrize("L_hi,L_lo,L_hi_v,L_lo_v", [(8, 5, 3, 2), (16, 8, 5, 4), (6, 4, 256, 17)])
+def test_cache_bytes_with_v_levels_match_oracle_layout(semkv, orc, L_hi, L_lo, L_hi_v, L_lo_v):
+    s = _shape(L_hi=L_hi, L_lo=L_lo, L_hi_v=L_hi_v, L_lo_v=L_lo_v)
+    sizes = dict(zip(semkv._lib.BUF_NAMES, semkv.semkv_cache_bytes(s)))
+    for seg, L, Lv, cap in (("hi", L_hi, L_hi_v, 256), ("lo", L_lo, L_lo_v, 768)):
+        sh = orc.segment_shapes(128, 64, L, cap // 128, Lv)
+        for name in ("k", "v", "kz", "vz"):
+            n = 1
+            for x in sh[name]:
+                n *= x
+            assert sizes[f"{name}_{seg}"] == 16 * n * 4, (seg, name)
 
 
 def test_variant_fields_accept_their_ranges(semkv):

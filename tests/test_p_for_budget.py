@@ -77,3 +77,21 @@ def test_bad_arguments(semkv):
     with pytest.raises(E) as e:
         semkv.semkv_p_for_ratio(128, 64, 257, 5, 5.0)
     assert e.value.code == semkv._lib.SEMKV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("L_hi,L_lo,L_hi_v,L_lo_v", [(8, 5, 3, 2), (6, 5, 6, 3), (16, 8, 5, 4), (5, 4, 8, 6)])
+def test_library_matches_oracle_bisection_with_v_levels(semkv, orc, L_hi, L_lo, L_hi_v, L_lo_v):
+    G = 64
+    r1 = 16.0 / orc.storage_bits_per_value(128, G, L_hi, L_lo, 1.0, L_hi_v, L_lo_v)
+    r0 = 16.0 / orc.storage_bits_per_value(128, G, L_hi, L_lo, 0.0, L_hi_v, L_lo_v)
+    a, b = min(r0, r1), max(r0, r1)
+    for ratio in np.linspace(a * 0.9, b * 1.001, 19):
+        want = orc.p_for_ratio(128, G, L_hi, L_lo, float(ratio), L_hi_v=L_hi_v, L_lo_v=L_lo_v)
+        if want is None:
+            with pytest.raises(semkv.SemkvError):
+                semkv.semkv_p_for_ratio_kv(128, G, L_hi, L_lo, L_hi_v, L_lo_v, float(ratio))
+            continue
+        got = semkv.semkv_p_for_ratio_kv(128, G, L_hi, L_lo, L_hi_v, L_lo_v, float(ratio))
+        assert abs(got - want) < 1e-9, (ratio, got, want)
+    # equal counts: the plain helper
+    assert semkv.semkv_p_for_ratio_kv(128, G, 8, 5, 8, 5, 4.8) == semkv.semkv_p_for_ratio(128, G, 8, 5, 4.8)

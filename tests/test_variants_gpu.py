@@ -154,3 +154,80 @@ def test_clip_and_window_appends_in_lockstep(mode):
         ref = oracle.attention_fp64(Q[-1, b, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, sm_scale())
         ma, rl = attention_errors(out.cpu().numpy()[b, h * g:(h + 1) * g], ref)
         assert ma <= ATOL and rl <= RTOL_L2, (ma, rl)
+
+
+# ---------------------------------------------------------------- V level counts of their own
+
+
+@pytest.mark.parametrize("B,H,Hq,T,G,L_hi,L_lo,L_hi_v,L_lo_v,p", [
+    (1, 2, 8, 600, 64, 8, 5, 3, 2, 0.25),    # 2-bit-class keys, 1.5-bit-class values
+    (2, 1, 4, 333, 32, 16, 8, 5, 4, 0.5),
+    (1, 1, 8, 700, 128, 6, 4, 4, 3, 0.1),
+    (1, 2, 8, 500, 64, 8, 5, 8, 3, 0.3),     # hi segment equal (tensor-core decode), lo on its own
+    (1, 1, 4, 260, 32, 5, 4, 256, 17, 0.4),  # V finer than K
+])
+def test_v_levels_full_path(B, H, Hq, T, G, L_hi, L_lo, L_hi_v, L_lo_v, p):
+    K, V, S, q = _case(B, H, Hq, T, T + L_hi_v * 7 + L_lo_v)
+    check_case(K, V, S, q, p, G, L_hi, L_lo, sm_scale(), L_hi_v=L_hi_v, L_lo_v=L_lo_v)
+
+
+@pytest.mark.parametrize("mode", ["append", "append_decode", "running"])
+def test_v_levels_appends_in_lockstep(mode):
+    import torch
+
+    import oracle
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, semkv_append_decode, semkv_append_token,
+                                               semkv_append_token_running, semkv_assign_precision,
+                                               semkv_decode_attention, semkv_quantize_pack)
+
+    B, H, Hq, T0, steps, G, L_hi, L_lo, Lhv, Llv, p = 1, 2, 8, 250, 80, 64, 8, 5, 3, 2, 0.3
+    r = np.random.default_rng(78)
+    K = r.standard_normal((B, H, T0 + steps, 128)).astype(np.float16)
+    V = r.standard_normal((B, H, T0 + steps, 128)).astype(np.float16)
+    S = r.standard_normal((B, H, T0 + steps)).astype(np.float32)
+    Q = r.standard_normal((steps, B, Hq, 128)).astype(np.float16)
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T0, p, extra=steps, L_hi_v=Lhv, L_lo_v=Llv).poison()
+    semkv_assign_precision(cache, to_dev(S[:, :, :T0].copy()), T0, p)
+    semkv_quantize_pack(cache, to_dev(K[:, :, :T0].copy()), to_dev(V[:, :, :T0].copy()), T0)
+    ws = cache.workspace()
+    states = []
+    for u in range(B * H):
+        b, h = divmod(u, H)
+        bm, rk, nh, tau, _ = oracle.select(S[b, h, :T0], p)
+        hi, lo, _ = oracle.quantize_pack_unit(K[b, h, :T0].view(np.uint16), V[b, h, :T0].view(np.uint16), bm, G,
+                                              L_hi, L_lo, cache.cap_hi // 128, cache.cap_lo // 128, L_hi_v=Lhv,
+                                              L_lo_v=Llv)
+        states.append(oracle.UnitState(cache.T_cap, bm, rk, nh, T0 - nh, tau, hi, lo))
+    g = Hq // H
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device="cuda")
+    for s in range(steps):
+        t = T0 + s
+        k, v, sc, q = (to_dev(x) for x in (K[:, :, t].copy(), V[:, :, t].copy(), S[:, :, t].copy(), Q[s]))
+        if mode == "append":
+            semkv_append_token(cache, k, v, sc)
+        elif mode == "append_decode":
+            semkv_append_decode(cache, k, v, sc, q, sm_scale(), out, ws)
+        else:
+            semkv_append_token_running(cache, k, v, sc, p)
+        for u in range(B * H):
+            b, h = divmod(u, H)
+            kk, vv = K[b, h, t].view(np.uint16), V[b, h, t].view(np.uint16)
+            if mode == "running":
+                oracle.append_unit_running(states[u], kk, vv, S[b, h, t], p, S[b, h, :t], G, L_hi, L_lo, 1.0, Lhv,
+                                           Llv)
+            else:
+                oracle.append_unit(states[u], kk, vv, S[b, h, t], G, L_hi, L_lo, 1.0, Lhv, Llv)
+    if mode != "append_decode":
+        semkv_decode_attention(cache, to_dev(Q[-1]), sm_scale(), out, ws)
+    bufs = fetch(cache)
+    assert cache.status() == 0
+    T = T0 + steps
+    for u, st in enumerate(states):
+        compare_state(unit_views(cache, bufs, u), {"bitmap": st.bitmap, "rank": st.rank, "n_hi": st.n_hi,
+                                                   "tau": st.tau, "hi": st.hi, "lo": st.lo},
+                      T, L_hi, L_lo, where=f"unit {u}", strict_tail=False, L_hi_v=Lhv, L_lo_v=Llv)
+        b, h = divmod(u, H)
+        Kh, Vh = oracle.dequantize_unit(T, 128, G, L_hi, L_lo, st.bitmap, st.hi, st.lo, Lhv, Llv)
+        ref = oracle.attention_fp64(Q[-1, b, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, sm_scale())
+        ma, rl = attention_errors(out.cpu().numpy()[b, h * g:(h + 1) * g], ref)
+        assert ma <= ATOL and rl <= RTOL_L2, (ma, rl)
