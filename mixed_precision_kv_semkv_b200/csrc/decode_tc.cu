@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
             for (int gg = 0; gg < NG; ++gg)
                 acc += sk[gg] * __uint_as_float(dk[gg * GQ + h]) + zk[gg] * qsum[gg * GQ + h];
             lg[h] = valid ? acc * scale_log2 : NEG_INF;
-            const float mx = warp_max(lg[h]);
+            const float mx = warp_max_redux(lg[h]);
             if (lane == 0) red[warp * 32 + h] = mx;
         }
         __syncthreads();
@@ -324,10 +324,10 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         for (int h = 0; h < GQ; ++h) {
             const float mt = fmaxf(fmaxf(red[h], red[32 + h]), fmaxf(red[64 + h], red[96 + h]));
             const float mn = fmaxf(m[h], mt);
-            alpha[h] = exp2f(m[h] - mn);
+            alpha[h] = ex2_approx(m[h] - mn);
             m[h] = mn;
             // slots past n may hold stale words (after appends): exact zeros, never a product
-            p[h] = valid ? exp2f(lg[h] - mn) : 0.f;
+            p[h] = valid ? ex2_approx(lg[h] - mn) : 0.f;
             lacc[h] = lacc[h] * alpha[h] + p[h];
 #pragma unroll
             for (int gg = 0; gg < NG; ++gg) zacc[gg][h] = zacc[gg][h] * alpha[h] + (valid ? p[h] * zv[gg] : 0.f);

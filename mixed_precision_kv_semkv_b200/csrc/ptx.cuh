@@ -206,4 +206,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
         : "memory");
 }
 
+// maximum of v over the 32 lanes of a warp (one redux instruction; NaN inputs are skipped)
+__device__ __forceinline__ float warp_max_redux(float v)
+{
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22; 2^-inf = 0, subnormal results
+// flushed to zero)
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 }  // namespace semkv
