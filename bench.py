@@ -62,7 +62,7 @@ def radix_words(L: int, n: int = 128) -> int:
 LAUNCHES_PER_STEP = 5
 # the quantizer variants timed beside the step (recent window of the selection; clipped range; V
 # level counts of their own for the hi and lo segments)
-WINDOW, CLIP, V_LEVELS = 128, 0.9, (5, 3)
+WINDOW, CLIP, V_LEVELS = 128, 0.9, (4, 2)
 
 
 def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False, v_levels=None) -> dict:
@@ -428,7 +428,7 @@ def run_semkv(args):
 
     t_win = timed(win_graph)
     t_clip = timed(clip_graph, before=(graphs[0],))
-    # V level counts of their own: quantize (generic kernel) and decode (CUDA-core decode)
+    # V level counts of their own: quantize (runtime-L kernel) and decode (tensor cores, own V radix)
     cache.struct.L_hi_v, cache.struct.L_lo_v = V_LEVELS
     calls[0]()
     calls[1]()

@@ -33,10 +33,11 @@
 
 namespace semkv {
 
-template <int L, int GQ, int NG>
-struct Tc {
+// One tensor's codes in TMEM: words per row (K) or per 128-slot column (V), digit pairs per word
+// (TMEM columns), and the MMA K-steps of 16 fp16 elements that cover them.
+template <int L>
+struct TcRadix {
     using R = Radix<L>;
-    static constexpr int D = 128;
     static constexpr int k = R::k;
     static constexpr int W = ceil_div(128, k);     // words per slot row (K) = per channel per tile (V)
     static constexpr int NPAIR = (k + 1) / 2;      // digit pairs (TMEM columns) per word
@@ -44,19 +45,29 @@ struct Tc {
     static constexpr int KCP = (KC + 7) / 8 * 8;   // padded to whole MMA K-steps (16 fp16)
     static constexpr int KSTEPS = KCP / 8;
     static constexpr int KSLOTS = 2 * KCP;         // fp16 elements along K
+    static constexpr bool ok = (R::pow2 || R::frac_ok) && KCP <= 80;
+    static constexpr uint32_t LUT_BYTES = (uint32_t)L * L * 32 * 4;
+};
+
+// LK, LV: level counts of the K and the V codes of the segment (equal unless V has its own)
+template <int LK, int LV, int GQ, int NG>
+struct Tc {
+    using RK = TcRadix<LK>;
+    using RV = TcRadix<LV>;
+    static constexpr int D = 128;
     static constexpr int G = D / NG;
     static constexpr int NK = (NG * GQ + 15) / 16 * 16;  // N of q.k
     static constexpr int GSTR = 2 * GQ <= 8 ? 8 : 16;    // D_V columns per group: limb-major, head-minor
     static constexpr int NV = NG * GSTR < 16 ? 16 : NG * GSTR;
     static constexpr uint32_t COL_A = 0, COL_DK = 80, COL_DV = 96, TMEM_COLS = 128;
-    static constexpr bool ok = (R::pow2 || R::frac_ok) && KCP <= 80 && NK <= 16 && NV <= 32 && G >= 32;
+    static constexpr bool ok = RK::ok && RV::ok && NK <= 16 && NV <= 32 && G >= 32;
     // shared memory
-    static constexpr uint32_t LBO_Q = 128, SBO_Q = (KSLOTS / 8) * 128;
-    static constexpr uint32_t LBO_P = 144, SBO_P = (KSLOTS / 8) * 144;  // 144: conflict-free slot writes
-    static constexpr uint32_t STAGE_K = 0, STAGE_V = W * 512, STAGE_KZ = 2 * W * 512,
+    static constexpr uint32_t LBO_Q = 128, SBO_Q = (RK::KSLOTS / 8) * 128;
+    static constexpr uint32_t LBO_P = 144, SBO_P = (RV::KSLOTS / 8) * 144;  // 144: conflict-free slot writes
+    static constexpr uint32_t STAGE_K = 0, STAGE_V = RK::W * 512, STAGE_KZ = STAGE_V + RV::W * 512,
                               STAGE_VZ = STAGE_KZ + NG * 512, STAGE_BYTES = STAGE_VZ + NG * 512;
-    static constexpr uint32_t LUT = 0, LUT_BYTES = (uint32_t)L * L * 32 * 4;
-    static constexpr uint32_t STAGES = (LUT_BYTES + 127) / 128 * 128;
+    static constexpr uint32_t LUT_K = 0, LUT_V = LK == LV ? 0u : (RK::LUT_BYTES + 127) / 128 * 128;
+    static constexpr uint32_t STAGES = (LUT_V + (LK == LV ? RK::LUT_BYTES : RV::LUT_BYTES) + 127) / 128 * 128;
     static constexpr uint32_t BQ = STAGES + 2 * STAGE_BYTES;
     static constexpr uint32_t BP = BQ + (NK / 8) * SBO_Q;
     static constexpr uint32_t QSUM = BP + (NV / 8) * SBO_P;
@@ -84,7 +95,43 @@ __host__ __device__ constexpr uint32_t core_off(int n, int ks, uint32_t lbo, uin
     return (uint32_t)(n >> 3) * sbo + (uint32_t)(ks >> 3) * lbo + (uint32_t)(n & 7) * 16u + (uint32_t)(ks & 7) * 2u;
 }
 
-template <int L, int GQ, int NG, bool APP>
+// One thread's row of codes -> TMEM: the tensor's W words (shared address `words` + 4 tid, stride
+// 512 B) become KCP columns of fp16 code pairs at `taddr` (this thread's lane), through the code
+// table whose lane copy starts at `lut_lane` (entry P at + 128 P bytes).
+template <int L>
+__device__ __forceinline__ void unpack_to_tmem(uint32_t words, uint32_t lut_lane, uint32_t taddr, int tid)
+{
+    using RC = TcRadix<L>;
+    constexpr int W = RC::W, NPAIR = RC::NPAIR, KC = RC::KC;
+    uint32_t wv[W];
+#pragma unroll
+    for (int j = 0; j < W; ++j) wv[j] = lds_u32_after_wait(words + (uint32_t)(j * 512 + 4 * tid));
+    uint32_t chunk[8];
+    int ci = 0;
+    uint32_t cbase = 0;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+        uint32_t f = to_fraction<L>(wv[j]);
+#pragma unroll
+        for (int pp = 0; pp < NPAIR; ++pp) {
+            const unsigned long long t = (unsigned long long)f * (unsigned long long)(L * L);
+            f = (uint32_t)t;
+            chunk[ci++] = lds_u32(lut_lane + ((uint32_t)(t >> 32) << 7));
+            if (ci == 8) {
+                tmem_st8(taddr + cbase, chunk);
+                cbase += 8;
+                ci = 0;
+            }
+        }
+    }
+    if (KC % 8) {
+#pragma unroll
+        for (int i = KC % 8; i < 8; ++i) chunk[i] = 0u;
+        tmem_st8(taddr + cbase, chunk);
+    }
+}
+
+template <int LK, int LV, int GQ, int NG, bool APP>
 __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_t* __restrict__ q, int H,
                                                        float scale_log2, int nsplit, int split_off, int nsplit_total,
                                                        float* __restrict__ ws, int32_t* __restrict__ status,
@@ -93,10 +140,11 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
                                                        const uint16_t* __restrict__ vnew,
                                                        const float* __restrict__ snew)
 {
-    using C = Tc<L, GQ, NG>;
-    constexpr int D = 128, W = C::W, NPAIR = C::NPAIR, KC = C::KC, KSTEPS = C::KSTEPS, KSLOTS = C::KSLOTS;
-    constexpr int k = C::k, G = C::G, NK = C::NK, NV = C::NV, GSTR = C::GSTR;
-    constexpr float MID = 0.5f * (float)(L - 1);
+    using C = Tc<LK, LV, GQ, NG>;
+    using RK = typename C::RK;
+    using RV = typename C::RV;
+    constexpr int D = 128, G = C::G, NK = C::NK, NV = C::NV, GSTR = C::GSTR;
+    constexpr float MID_K = 0.5f * (float)(LK - 1), MID_V = 0.5f * (float)(LV - 1);
     constexpr float NEG_INF = -__builtin_huge_valf();
 
     // a dependent launch (the other segment) may start on free SMs right away
@@ -106,7 +154,8 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     extern __shared__ __align__(1024) unsigned char smem[];
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::LUT);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::LUT_K);
+    uint32_t* lut_v = reinterpret_cast<uint32_t*>(smem + C::LUT_V);
     unsigned char* stage0 = smem + C::STAGES;
     unsigned char* bq = smem + C::BQ;
     unsigned char* bp = smem + C::BP;
@@ -144,8 +193,8 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         unsigned char* dst = stage0 + stg * C::STAGE_BYTES;
         const size_t tb = (size_t)u * seg.tiles_cap + tile;
         mbar_arrive_expect_tx(&mbar[2 + stg], C::STAGE_BYTES);
-        bulk_g2s(dst + C::STAGE_K, seg.k + tb * W * TILE, W * 512, &mbar[2 + stg]);
-        bulk_g2s(dst + C::STAGE_V, seg.v + tb * W * D, W * 512, &mbar[2 + stg]);
+        bulk_g2s(dst + C::STAGE_K, seg.k + tb * RK::W * TILE, RK::W * 512, &mbar[2 + stg]);
+        bulk_g2s(dst + C::STAGE_V, seg.v + tb * RV::W * D, RV::W * 512, &mbar[2 + stg]);
         bulk_g2s(dst + C::STAGE_KZ, seg.kz + tb * NG * TILE, NG * 512, &mbar[2 + stg]);
         bulk_g2s(dst + C::STAGE_VZ, seg.vz + tb * NG * TILE, NG * 512, &mbar[2 + stg]);
     };
@@ -173,19 +222,26 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         for (int e = 0; e < (QV + 127) / 128; ++e)
             if (tid + 128 * e < QV) qv[e] = __ldg(qu + tid + 128 * e);
     }
-    for (int i = tid; i < L * L * 32; i += 128) {
+    for (int i = tid; i < LK * LK * 32; i += 128) {
         const int P = i >> 5;
-        const __half2 pr = __floats2half2_rn((float)(P / L) - MID, (float)(P % L) - MID);  // exact: |x| <= 7.5
+        const __half2 pr = __floats2half2_rn((float)(P / LK) - MID_K, (float)(P % LK) - MID_K);  // exact: |x| <= 7.5
         lut[i] = *reinterpret_cast<const uint32_t*>(&pr);
+    }
+    if constexpr (LV != LK) {
+        for (int i = tid; i < LV * LV * 32; i += 128) {
+            const int P = i >> 5;
+            const __half2 pr = __floats2half2_rn((float)(P / LV) - MID_V, (float)(P % LV) - MID_V);
+            lut_v[i] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
     }
 #pragma unroll
     for (int e = 0; e < (QV + 127) / 128; ++e)
         if (tid + 128 * e < QV) reinterpret_cast<uint4*>(qs)[tid + 128 * e] = qv[e];
     __syncthreads();
-    for (int ks = tid; ks < KSLOTS; ks += 128) {
-        const int col = ks >> 1, h2 = ks & 1, j = col / NPAIR, pp = col % NPAIR;
-        const int pos = pair_digit(k, pp, h2);
-        const int dim = (col < KC && pos >= 0) ? j * k + pos : D;
+    for (int ks = tid; ks < RK::KSLOTS; ks += 128) {
+        const int col = ks >> 1, h2 = ks & 1, j = col / RK::NPAIR, pp = col % RK::NPAIR;
+        const int pos = pair_digit(RK::k, pp, h2);
+        const int dim = (col < RK::KC && pos >= 0) ? j * RK::k + pos : D;
         const int dgrp = dim < D ? dim / G : -1;
 #pragma unroll
         for (int nrow = 0; nrow < NK; ++nrow) {
@@ -223,8 +279,8 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     const uint32_t bq_addr = smem_u32(bq), bp_addr = smem_u32(bp);
 
     // my slot's row of B_P (slot tid -> K index along the unpacked V words)
-    const int vrank = k - 1 - (tid % k);
-    const int my_ks = 2 * ((tid / k) * NPAIR + (vrank >> 1)) + (vrank & 1);
+    const int vrank = RV::k - 1 - (tid % RV::k);
+    const int my_ks = 2 * ((tid / RV::k) * RV::NPAIR + (vrank >> 1)) + (vrank & 1);
     unsigned char* bp_my = bp + (uint32_t)(my_ks >> 3) * C::LBO_P + (uint32_t)(my_ks & 7) * 2u;
     const int grp_d = tid / G;  // my channel's group (uniform over a warp: G >= 32)
 
@@ -239,36 +295,9 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     uint32_t ph_k = 0, ph_v = 0;
     bool timeout = false;
 
-    const uint32_t lut_lane = smem_u32(lut + lane);  // this lane's copy: entry P at + 128 P bytes
-    // W words (shared address `words` + 4 tid, stride 512 B) -> KCP TMEM columns of this thread's lane
-    auto unpack_to_tmem = [&](uint32_t words) {
-        uint32_t wv[W];
-#pragma unroll
-        for (int j = 0; j < W; ++j) wv[j] = lds_u32_after_wait(words + (uint32_t)(j * 512 + 4 * tid));
-        uint32_t chunk[8];
-        int ci = 0;
-        uint32_t cbase = C::COL_A;
-#pragma unroll
-        for (int j = 0; j < W; ++j) {
-            uint32_t f = to_fraction<L>(wv[j]);
-#pragma unroll
-            for (int pp = 0; pp < NPAIR; ++pp) {
-                const unsigned long long t = (unsigned long long)f * (unsigned long long)(L * L);
-                f = (uint32_t)t;
-                chunk[ci++] = lds_u32(lut_lane + ((uint32_t)(t >> 32) << 7));
-                if (ci == 8) {
-                    tmem_st8(lane_base + cbase, chunk);
-                    cbase += 8;
-                    ci = 0;
-                }
-            }
-        }
-        if (KC % 8) {
-#pragma unroll
-            for (int i = KC % 8; i < 8; ++i) chunk[i] = 0u;
-            tmem_st8(lane_base + cbase, chunk);
-        }
-    };
+    // this lane's copies of the code tables: entry P at + 128 P bytes
+    const uint32_t lut_lane_k = smem_u32(lut + lane), lut_lane_v = smem_u32(lut_v + lane);
+    const uint32_t taddr_a = lane_base + C::COL_A;
 
     for (int tile = t0, it = 0; tile < t1; ++tile, ++it) {
         const int stg = it & 1;
@@ -276,14 +305,14 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         if (!mbar_wait(&mbar[2 + stg], (uint32_t)(it >> 1) & 1u)) timeout = true;
 
         // ---- K codes -> TMEM, q.k
-        unpack_to_tmem(smem_u32(sb + C::STAGE_K));
+        unpack_to_tmem<LK>(smem_u32(sb + C::STAGE_K), lut_lane_k, taddr_a, tid);
         tc_wait_st();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int s = 0; s < KSTEPS; ++s)
+            for (int s = 0; s < RK::KSTEPS; ++s)
                 mma_ts_f16(tmem + C::COL_DK, tmem + C::COL_A + 8 * s,
                            smem_desc(bq_addr + s * 2 * C::LBO_Q, C::LBO_Q, C::SBO_Q), idesc_k, s > 0);
             mma_commit(&mbar[0]);
@@ -295,9 +324,9 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
             const uint32_t kzv = reinterpret_cast<const uint32_t*>(sb + C::STAGE_KZ)[gg * 128 + tid];
             const uint32_t vzv = reinterpret_cast<const uint32_t*>(sb + C::STAGE_VZ)[gg * 128 + tid];
             sk[gg] = h2f((uint16_t)(kzv & 0xffffu));
-            zk[gg] = __fmaf_rn(MID, sk[gg], h2f((uint16_t)(kzv >> 16)));
+            zk[gg] = __fmaf_rn(MID_K, sk[gg], h2f((uint16_t)(kzv >> 16)));
             sv[gg] = h2f((uint16_t)(vzv & 0xffffu));
-            zv[gg] = __fmaf_rn(MID, sv[gg], h2f((uint16_t)(vzv >> 16)));
+            zv[gg] = __fmaf_rn(MID_V, sv[gg], h2f((uint16_t)(vzv >> 16)));
         }
         if (!mbar_wait(&mbar[0], ph_k)) timeout = true;
         ph_k ^= 1u;
@@ -346,7 +375,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
             }
         }
         // ---- V codes -> TMEM (same columns: the q.k product has completed), p.V
-        unpack_to_tmem(smem_u32(sb + C::STAGE_V));
+        unpack_to_tmem<LV>(smem_u32(sb + C::STAGE_V), lut_lane_v, taddr_a, tid);
         tc_wait_st();
         fence_async_smem();
         tc_fence_before();
@@ -354,7 +383,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int s = 0; s < KSTEPS; ++s)
+            for (int s = 0; s < RV::KSTEPS; ++s)
                 mma_ts_f16(tmem + C::COL_DV, tmem + C::COL_A + 8 * s,
                            smem_desc(bp_addr + s * 2 * C::LBO_P, C::LBO_P, C::SBO_P), idesc_v, s > 0);
             mma_commit(&mbar[1]);
@@ -419,17 +448,17 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     if (wait_for_prior) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <int L, int GQ, int NG>
+template <int LK, int LV, int GQ, int NG>
 static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, float scale_log2, int nsplit,
                       int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
                       const AppendIn& app, cudaStream_t st)
 {
-    using C = Tc<L, GQ, NG>;
+    using C = Tc<LK, LV, GQ, NG>;
     // at most four CTAs per SM: each holds 128 of the SM's 512 TMEM columns
     const size_t sm = C::TOTAL > 48u * 1024u ? C::TOTAL : 48u * 1024u;
     // the plain decode and the one that appends first are separate instantiations, so that the
     // plain one carries no append code
-    const auto kern = app.k ? k_decode_tc<L, GQ, NG, true> : k_decode_tc<L, GQ, NG, false>;
+    const auto kern = app.k ? k_decode_tc<LK, LV, GQ, NG, true> : k_decode_tc<LK, LV, GQ, NG, false>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)nsplit, (unsigned)units);
@@ -445,17 +474,21 @@ static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, f
                        status, dependent ? 1 : 0, app.cache, app.k, app.v, app.score);
 }
 
-// instantiated shapes: L in {4, 5, 6, 8, 16} x (g, groups) whose accumulators fit 128 TMEM columns
-#define SEMKV_TC_SHAPES(X, L) X(L, 2, 1) X(L, 2, 2) X(L, 2, 4) X(L, 4, 1) X(L, 4, 2) X(L, 4, 4) X(L, 8, 1) X(L, 8, 2)
-#define SEMKV_TC_LEVELS(X) SEMKV_TC_SHAPES(X, 4) SEMKV_TC_SHAPES(X, 5) SEMKV_TC_SHAPES(X, 6) SEMKV_TC_SHAPES(X, 8) \
-    SEMKV_TC_SHAPES(X, 16)
+// instantiated shapes: K and V level counts (equal: L in {4, 5, 6, 8, 16}; V with its own count:
+// six common pairs) x (g, groups) whose accumulators fit 128 TMEM columns
+#define SEMKV_TC_SHAPES(X, LK, LV) X(LK, LV, 2, 1) X(LK, LV, 2, 2) X(LK, LV, 2, 4) X(LK, LV, 4, 1) X(LK, LV, 4, 2) \
+    X(LK, LV, 4, 4) X(LK, LV, 8, 1) X(LK, LV, 8, 2)
+#define SEMKV_TC_SHAPES_KV(X, LK, LV) X(LK, LV, 2, 2) X(LK, LV, 4, 1) X(LK, LV, 4, 2) X(LK, LV, 8, 1) X(LK, LV, 8, 2)
+#define SEMKV_TC_LEVELS(X) SEMKV_TC_SHAPES(X, 4, 4) SEMKV_TC_SHAPES(X, 5, 5) SEMKV_TC_SHAPES(X, 6, 6) \
+    SEMKV_TC_SHAPES(X, 8, 8) SEMKV_TC_SHAPES(X, 16, 16) SEMKV_TC_SHAPES_KV(X, 8, 4) SEMKV_TC_SHAPES_KV(X, 5, 2) \
+    SEMKV_TC_SHAPES_KV(X, 8, 5) SEMKV_TC_SHAPES_KV(X, 6, 4) SEMKV_TC_SHAPES_KV(X, 5, 4) SEMKV_TC_SHAPES_KV(X, 16, 8)
 
-bool decode_tc_supported(int L, int G, int g)
+bool decode_tc_supported(int Lk, int Lv, int G, int g)
 {
     if (G <= 0 || 128 % G) return false;
     const int ng = 128 / G;
-#define SEMKV_TC_OK(LL, GG, NN) \
-    if (L == LL && g == GG && ng == NN) return Tc<LL, GG, NN>::ok;
+#define SEMKV_TC_OK(LK, LV, GG, NN) \
+    if (Lk == LK && Lv == LV && g == GG && ng == NN) return Tc<LK, LV, GG, NN>::ok;
     SEMKV_TC_LEVELS(SEMKV_TC_OK)
 #undef SEMKV_TC_OK
     return false;
@@ -467,11 +500,11 @@ void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, i
 {
     if (nsplit == 0 || units == 0) return;
     const int ng = 128 / G;
-#define SEMKV_TC_GO(LL, GG, NN)                                                                                   \
-    if (seg.L == LL && g == GG && ng == NN) {                                                                     \
-        launch_tc<LL, GG, NN>(seg, q, units, H, scale_log2, nsplit, split_off, nsplit_total, ws, status, dependent, \
-                              app, st);                                                                           \
-        return;                                                                                                   \
+#define SEMKV_TC_GO(LK, LV, GG, NN)                                                                                 \
+    if (seg.L == LK && seg.Lv == LV && g == GG && ng == NN) {                                                    \
+        launch_tc<LK, LV, GG, NN>(seg, q, units, H, scale_log2, nsplit, split_off, nsplit_total, ws, status,      \
+                                  dependent, app, st);                                                          \
+        return;                                                                                                 \
     }
     SEMKV_TC_LEVELS(SEMKV_TC_GO)
 #undef SEMKV_TC_GO

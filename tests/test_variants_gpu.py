@@ -160,7 +160,9 @@ def test_clip_and_window_appends_in_lockstep(mode):
 
 
 @pytest.mark.parametrize("B,H,Hq,T,G,L_hi,L_lo,L_hi_v,L_lo_v,p", [
-    (1, 2, 8, 600, 64, 8, 5, 3, 2, 0.25),    # 2-bit-class keys, 1.5-bit-class values
+    (1, 2, 8, 600, 64, 8, 5, 3, 2, 0.25),    # 2-bit-class keys, 1.5-bit-class values (lo on the tensor cores)
+    (1, 2, 8, 900, 64, 8, 5, 4, 2, 0.3),     # both segments on the tensor-core decode with their own V radix
+    (2, 2, 16, 400, 128, 8, 6, 5, 4, 0.2),   # g = 8, one group
     (2, 1, 4, 333, 32, 16, 8, 5, 4, 0.5),
     (1, 1, 8, 700, 128, 6, 4, 4, 3, 0.1),
     (1, 2, 8, 500, 64, 8, 5, 8, 3, 0.3),     # hi segment equal (tensor-core decode), lo on its own
@@ -171,8 +173,9 @@ def test_v_levels_full_path(B, H, Hq, T, G, L_hi, L_lo, L_hi_v, L_lo_v, p):
     check_case(K, V, S, q, p, G, L_hi, L_lo, sm_scale(), L_hi_v=L_hi_v, L_lo_v=L_lo_v)
 
 
+@pytest.mark.parametrize("Lhv,Llv", [(3, 2), (4, 2)])
 @pytest.mark.parametrize("mode", ["append", "append_decode", "running"])
-def test_v_levels_appends_in_lockstep(mode):
+def test_v_levels_appends_in_lockstep(mode, Lhv, Llv):
     import torch
 
     import oracle
@@ -180,7 +183,7 @@ def test_v_levels_appends_in_lockstep(mode):
                                                semkv_append_token_running, semkv_assign_precision,
                                                semkv_decode_attention, semkv_quantize_pack)
 
-    B, H, Hq, T0, steps, G, L_hi, L_lo, Lhv, Llv, p = 1, 2, 8, 250, 80, 64, 8, 5, 3, 2, 0.3
+    B, H, Hq, T0, steps, G, L_hi, L_lo, p = 1, 2, 8, 250, 80, 64, 8, 5, 0.3
     r = np.random.default_rng(78)
     K = r.standard_normal((B, H, T0 + steps, 128)).astype(np.float16)
     V = r.standard_normal((B, H, T0 + steps, 128)).astype(np.float16)
