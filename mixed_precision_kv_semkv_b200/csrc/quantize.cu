@@ -234,8 +234,10 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
 // constant powers (no serial Horner chain), codes are the low byte of the round-to-nearest-even
 // magic sum 1.5 * 2^23 + q (the offset is removed once per word), group minima and maxima use
 // packed fp16 (NaN-propagating, so a non-finite value shows up in the group's range), and the
-// quotient runs two lanes at a time in packed fp32.  For L >= 3 no clamp is needed: q <= L - 1
-// up to one rounding when the scale did not saturate, and q <= 131008/65504 = 2 when it did.
+// quotient runs two lanes at a time in packed fp32.  On the plain grid no clamp is needed for
+// L >= 3: q <= L - 1 up to one rounding when the scale did not saturate, and q <= 131008/65504 = 2
+// when it did.  The clipped grid clamps on both sides (group_codes).  The V part of a tile may
+// use its own level count.
 
 __host__ __device__ constexpr uint32_t upow(int L, int i)
 {
@@ -272,12 +274,14 @@ __device__ __forceinline__ uint64_t code2_bits(uint64_t x2, uint64_t z2, uint64_
 
 struct GroupGrid {
     uint64_t z2, r2, ns2;
+    uint32_t zh2;  // the zero as a binary16 pair (the clipped grid's lower clamp)
     uint32_t packed;
     bool finite;
 };
 
-template <int L, int G>
-__device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2])
+// CLIP: the clipped-range grid (clip < 1); otherwise the plain min/max grid
+template <int L, int G, bool CLIP>
+__device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2], float clip)
 {
     __half2 mn2 = *reinterpret_cast<const __half2*>(&h[0]), mx2 = mn2;
 #pragma unroll
@@ -290,8 +294,15 @@ __device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2])
     const float mx = __half2float(__hmax_nan(__low2half(mx2), __high2half(mx2)));
     GroupGrid g;
     g.finite = fabsf(mn) <= 65504.0f && fabsf(mx) <= 65504.0f;
-    const uint16_t s16 = scale_half_ru(__fdiv_rn(__fsub_rn(mx, mn), (float)(L - 1)));
-    const uint16_t z16 = zero_half(mn);
+    uint16_t s16, z16;
+    if constexpr (CLIP) {
+        group_scale_zero(mn, mx, L, clip, s16, z16);
+    } else {
+        (void)clip;
+        s16 = scale_half_ru(__fdiv_rn(__fsub_rn(mx, mn), (float)(L - 1)));
+        z16 = zero_half(mn);
+    }
+    g.zh2 = (uint32_t)z16 | ((uint32_t)z16 << 16);
     const float s = h2f(s16), z = h2f(z16);
     const float r = s != 0.0f ? __frcp_rn(s) : 0.0f;
     g.z2 = f2_pack(z, z);
@@ -301,15 +312,32 @@ __device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2])
     return g;
 }
 
-// codes (as magic-offset fp32 bits) of one group's G values, two at a time, handed to `sink(i, bits)`
-template <int L, int G, typename Sink>
+// codes (as magic-offset fp32 bits) of one group's G values, two at a time, handed to `sink(i, bits)`.
+// CLIP: values below the zero are raised to it first (exact: the zero is a binary16) and the
+// quotient is clamped to L - 1 before the rounding add, so codes are clamp(rint(q), 0, L - 1) and
+// the add stays in its exact range.
+template <int L, int G, bool CLIP, typename Sink>
 __device__ __forceinline__ void group_codes(const uint32_t (&h)[G / 2], const GroupGrid& g, Sink&& sink)
 {
     const uint64_t m2 = f2_pack(12582912.0f, 12582912.0f);
 #pragma unroll
     for (int i = 0; i < G / 2; ++i) {
-        const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-        uint64_t y = code2_bits(f2_pack(xf.x, xf.y), g.z2, g.r2, g.ns2, m2);
+        __half2 hv = *reinterpret_cast<const __half2*>(&h[i]);
+        if constexpr (CLIP) hv = __hmax2(hv, *reinterpret_cast<const __half2*>(&g.zh2));
+        const float2 xf = __half22float2(hv);
+        uint64_t y;
+        if constexpr (CLIP) {
+            uint64_t d, q0, e, q;
+            asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(xf.x, xf.y)), "l"(g.z2));
+            asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(d), "l"(g.r2));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e) : "l"(g.ns2), "l"(q0), "l"(d));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(e), "l"(g.r2), "l"(q0));
+            const float qa = fminf(__uint_as_float((uint32_t)q), (float)(L - 1));
+            const float qb = fminf(__uint_as_float((uint32_t)(q >> 32)), (float)(L - 1));
+            asm("add.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(f2_pack(qa, qb)), "l"(m2));
+        } else {
+            y = code2_bits(f2_pack(xf.x, xf.y), g.z2, g.r2, g.ns2, m2);
+        }
         uint32_t b0 = (uint32_t)y, b1 = (uint32_t)(y >> 32);
         if constexpr (L == 2) {  // the only level count whose codes can exceed L - 1 (saturated scale)
             b0 = min(b0, 0x4B400001u);
@@ -321,8 +349,9 @@ __device__ __forceinline__ void group_codes(const uint32_t (&h)[G / 2], const Gr
 }
 
 // K rows of a tile: thread `tid` quantizes row tid and packs it along the channels
-template <int L, int G>
-__device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw, uint32_t* kz, int tid, bool& bad)
+template <int L, int G, bool CLIP>
+__device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw, uint32_t* kz, int tid, bool& bad,
+                                                float clip)
 {
     constexpr int D = 128, k = radix_k(L), WK = ceil_div(D, k), NG = D / G;
     {
@@ -341,10 +370,10 @@ __device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw
                 h[4 * i + 2] = v.z;
                 h[4 * i + 3] = v.w;
             }
-            const GroupGrid g = group_grid<L, G>(h);
+            const GroupGrid g = group_grid<L, G, CLIP>(h, clip);
             bad |= !g.finite;
             kz[grp * TILE + tid] = g.packed;
-            group_codes<L, G>(h, g, [&](int i, uint32_t bits) {
+            group_codes<L, G, CLIP>(h, g, [&](int i, uint32_t bits) {
                 const int d = grp * G + i;
                 w[d / k] += bits * upow(L, d % k);
             });
@@ -359,8 +388,9 @@ __device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw
 
 // V rows of a tile: thread `tid` writes the grids of row tid and its codes as bytes over the first
 // half of its own row; after a barrier thread `tid` packs channel tid along the tile's slots
-template <int L, int G>
-__device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint32_t* vz, int tid, bool& bad)
+template <int L, int G, bool CLIP>
+__device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint32_t* vz, int tid, bool& bad,
+                                                float clip)
 {
     constexpr int D = 128, k = radix_k(L), WV = ceil_div(TILE, k), NG = D / G;
     {
@@ -378,11 +408,11 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
                 h[4 * i + 2] = v.z;
                 h[4 * i + 3] = v.w;
             }
-            const GroupGrid g = group_grid<L, G>(h);
+            const GroupGrid g = group_grid<L, G, CLIP>(h, clip);
             bad |= !g.finite;
             packed[grp] = g.packed;
             // the low byte of each magic sum is the code: byte i%4 of word i/4
-            group_codes<L, G>(h, g, [&](int i, uint32_t b) {
+            group_codes<L, G, CLIP>(h, g, [&](int i, uint32_t b) {
                 const int c = grp * G + i;
                 constexpr uint32_t sel[4] = {0x3214u, 0x3240u, 0x3410u, 0x4210u};
                 bytes[c / 4] = (c % 4 == 0) ? (b & 0xffu) : __byte_perm(bytes[c / 4], b, sel[c % 4]);
@@ -409,10 +439,12 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
     }
 }
 
-template <int LH, int LL, int G>
+// LH, LL: level counts of the K codes of the two segments; LHV, LLV: of the V codes; CLIP: the
+// clipped-range grid with ratio `clip`
+template <int LH, int LL, int LHV, int LLV, int G, bool CLIP>
 __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
                                                         const uint16_t* __restrict__ V,
-                                                        int T,
+                                                        int T, float clip,
                                                         int32_t* __restrict__ status)
 {
     constexpr int D = 128, NG = D / G;
@@ -440,19 +472,19 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
     gather_rows_warp(Xs, nullptr, seg, u, s0, min(TILE, n - s0), part ? V : K, nullptr, T);
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
-    const int W_hi = ceil_div(D, radix_k(LH)), W_lo = ceil_div(D, radix_k(LL));
-    const int Wd = is_hi ? W_hi : W_lo;
     bool bad = false;
     if (part == 0) {
-        uint32_t* kw = seg.k + tile_base * Wd * TILE;
+        const int Wk = is_hi ? ceil_div(D, radix_k(LH)) : ceil_div(D, radix_k(LL));
+        uint32_t* kw = seg.k + tile_base * Wk * TILE;
         uint32_t* kz = seg.kz + tile_base * NG * TILE;
-        if (is_hi) quantize_k_rows<LH, G>(Xs, kw, kz, tid, bad);
-        else quantize_k_rows<LL, G>(Xs, kw, kz, tid, bad);
+        if (is_hi) quantize_k_rows<LH, G, CLIP>(Xs, kw, kz, tid, bad, clip);
+        else quantize_k_rows<LL, G, CLIP>(Xs, kw, kz, tid, bad, clip);
     } else {
-        uint32_t* vw = seg.v + tile_base * Wd * D;
+        const int Wv = is_hi ? ceil_div(TILE, radix_k(LHV)) : ceil_div(TILE, radix_k(LLV));
+        uint32_t* vw = seg.v + tile_base * Wv * D;
         uint32_t* vz = seg.vz + tile_base * NG * TILE;
-        if (is_hi) quantize_v_rows<LH, G>(Xs, vw, vz, tid, bad);
-        else quantize_v_rows<LL, G>(Xs, vw, vz, tid, bad);
+        if (is_hi) quantize_v_rows<LHV, G, CLIP>(Xs, vw, vz, tid, bad, clip);
+        else quantize_v_rows<LLV, G, CLIP>(Xs, vw, vz, tid, bad, clip);
     }
     if (bad && tid < n - s0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
 }
@@ -490,17 +522,22 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     const unsigned grid = (unsigned)units * per_unit;
     const QuantSeg qh = conv(shi, slot_token), ql = conv(slo, slot_token + shi.tiles_cap * TILE);
     // compile-time level pairs and group sizes of the common configurations
-    // (the clipped-range variant needs codes clamped from below, and V level counts of their own
-    // need a second radix: both only in the generic kernel)
-#define SEMKV_QF(LH, LL, GG)                                                                                  \
-    if (clip == 1.0f && shi.Lv == shi.L && slo.Lv == slo.L && shi.L == LH && slo.L == LL && G == GG) {                                                              \
+    // compile-time level counts and group sizes of the common configurations; the quantizer
+    // variants (a clip, V level counts of their own) for a few of them, the rest on k_quantize
+    const bool clipped = clip != 1.0f;
+#define SEMKV_QF(LH, LL, LHV, LLV, GG, CL)                                                                    \
+    if (clipped == CL && shi.L == LH && slo.L == LL && shi.Lv == LHV && slo.Lv == LLV && G == GG) {           \
         const size_t sm = (size_t)TILE * QROW * 2;                                                            \
-        cudaFuncSetAttribute(k_quantize_fast<LH, LL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
-        k_quantize_fast<LH, LL, GG><<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, status);                      \
+        const auto kern = k_quantize_fast<LH, LL, LHV, LLV, GG, CL>;                                          \
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);                    \
+        kern<<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, clip, status);                                       \
         return;                                                                                               \
     }
-#define SEMKV_QF_G(LH, LL) SEMKV_QF(LH, LL, 32) SEMKV_QF(LH, LL, 64) SEMKV_QF(LH, LL, 128)
+#define SEMKV_QF_G(LH, LL) SEMKV_QF(LH, LL, LH, LL, 32, false) SEMKV_QF(LH, LL, LH, LL, 64, false) \
+    SEMKV_QF(LH, LL, LH, LL, 128, false) SEMKV_QF(LH, LL, LH, LL, 64, true)
     SEMKV_QF_G(8, 5) SEMKV_QF_G(6, 5) SEMKV_QF_G(8, 6) SEMKV_QF_G(16, 8) SEMKV_QF_G(5, 4)
+    SEMKV_QF(8, 5, 4, 2, 64, false) SEMKV_QF(6, 5, 4, 3, 64, false) SEMKV_QF(8, 6, 4, 2, 64, false)
+    SEMKV_QF(16, 8, 8, 4, 64, false)
 #undef SEMKV_QF_G
 #undef SEMKV_QF
     const size_t sm = quantize_smem(G);
