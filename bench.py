@@ -214,6 +214,15 @@ def oracle_sample(w, seconds_target: float = 15.0, max_units: int = 8):
 # ---------------------------------------------------------------- reference arm
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` of both arms' JSON lines: the workload, named by what it is and its sizes."""
+    return {"workload": f"{w.name}: Llama-3.1-8B-shaped layer, B{w.B} H{w.H} Hq{w.Hq} T{w.T} D{w.D}, "
+                        f"G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}",
+"parallelism": f"dp{world} (independent units)",
+            "step": "assign_precision + quantize_pack + append_decode (append_token of one generated token per "
+                    "unit and decode_attention in one pass)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -221,8 +230,10 @@ def run_reference(args):
     from mixed_precision_kv_semkv_b200 import synth
 
     w = synth.WORKLOADS[args.workload]
-    steps = max(1, min(args.steps, 3))
-    warm = max(0, min(args.warmup, 1))
+    # each step is a bounded sample (one unit, ~0.5 s of the oracle on one core), so that the run
+    # ends within seconds whatever --steps asks
+    steps = max(1, min(args.steps, 10))
+    warm = max(0, min(args.warmup, 3))
     for _ in range(warm):
         oracle_sample(w, seconds_target=0.0, max_units=1)
     secs, byts = 0.0, 0.0
@@ -234,8 +245,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": steps, "warmup": warm,
             "ms_per_step": secs / steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "Hq": w.Hq, "T": w.T, "G": w.G, "L_hi": w.L_hi,
-                       "L_lo": w.L_lo, "p": w.p, "sample": "1 unit per step"},
+            "config": dict(workload_config(w, args.gpus), sample="1 unit (one batch row x kv head) per step"),
             "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": r["sample"]},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -539,14 +549,10 @@ def run_semkv(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warm,
         "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "u32-packed codes, fp32 math", "data": "synthetic",
-        "config": {"workload": f"{w.name}: Llama-3.1-8B-shaped layer, B{w.B} H{w.H} Hq{w.Hq} T{T} D{w.D}, "
-                               f"G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}",
-                   "l2": "flushed between steps (512 MB write)", "parallelism": f"dp{world} (independent units)",
-                   "timing": "step = one CUDA graph of its three calls; per_kernel = each call (and the separate "
-                             "append_token and decode_attention) replayed from a graph of its own (so each also pays "
-                             "a graph launch)",
-                   "step": "assign_precision + quantize_pack + append_decode (append_token of one generated token "
-                           "per unit and decode_attention in one pass)"},
+        "config": dict(workload_config(w, world), l2="flushed between steps (512 MB write)",
+                       timing="step = one CUDA graph of its three calls; per_kernel = each call (and the separate "
+                              "append_token and decode_attention) replayed from a graph of its own (so each also pays "
+                              "a graph launch)"),
         "per_kernel": per_kernel,
         "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                      "frac": ach / hbm_peak, "peak_kind": peak_note, "traffic": traffic,
