@@ -78,15 +78,20 @@ def lib():
         L.oracle_pack_word.argtypes = [_u8p, _c.c_int, _c.c_int]
         L.oracle_pack_word.restype = _c.c_uint32
         L.oracle_unpack_word.argtypes = [_c.c_uint32, _c.c_int, _c.c_int, _u8p]
+        _u32p_or_null = _c.c_void_p
         L.oracle_quantize_pack_unit.argtypes = [_u16p, _u16p, _c.c_int32, _c.c_int, _c.c_int, _c.c_int,
                                                 _c.c_int, _c.c_int, _c.c_int, _c.c_float, _u32p, _c.c_int,
-                                                _c.c_int] + [_u32p] * 8
+                                                _c.c_int] + [_u32p] * 8 + [_u32p_or_null]
+        L.oracle_k_channel_grid.argtypes = [_u16p, _c.c_int32, _c.c_int, _c.c_int, _c.c_int, _c.c_float, _u32p]
+        L.oracle_k_channel_grid.restype = _c.c_int
+        L.oracle_code_on_grid.argtypes = [_c.c_uint16, _c.c_uint16, _c.c_uint16, _c.c_int]
+        L.oracle_code_on_grid.restype = _c.c_int
         L.oracle_quantize_pack_unit.restype = _c.c_int
         L.oracle_dequantize_unit.argtypes = [_c.c_int32, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int,
-                                             _u32p] + [_u32p] * 8 + [_f32p, _f32p]
+                                             _u32p] + [_u32p] * 8 + [_f32p, _f32p, _c.c_void_p]
         L.oracle_append_unit.argtypes = [_u16p, _u16p, _c.c_float, _c.c_float, _c.c_int, _c.c_int, _c.c_int,
                                          _c.c_int, _c.c_int, _c.c_int, _c.c_float, _c.c_int32, _u32p, _u32p, _c.POINTER(_c.c_int32),
-                                         _c.POINTER(_c.c_int32), _c.c_int, _c.c_int] + [_u32p] * 8
+                                         _c.POINTER(_c.c_int32), _c.c_int, _c.c_int] + [_u32p] * 8 + [_c.c_void_p]
         L.oracle_append_unit.restype = _c.c_int
         L.oracle_attention_fp64.argtypes = [_u16p, _c.c_int, _f32p, _f32p, _c.c_int32, _c.c_int, _c.c_float,
                                             _f64p]
@@ -196,10 +201,29 @@ def _seg_args(hi, lo):
             lo["k"].ravel(), lo["v"].ravel(), lo["kz"].ravel(), lo["vz"].ravel()]
 
 
+def _ptr_or_null(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.uint32).ctypes.data
+
+
+def k_channel_grid(K16, L_hi: int, L_lo: int, clip: float = 1.0):
+    """Per-channel K grids of one unit: uint32 [2][D] (hi, lo; fp16 scale | fp16 zero << 16) and status."""
+    K16 = np.ascontiguousarray(K16, dtype=np.uint16)
+    T, D = K16.shape
+    kc = np.zeros((2, D), np.uint32)
+    st = lib().oracle_k_channel_grid(K16.ravel() if T else np.zeros(1, np.uint16), T, D, L_hi, L_lo, float(clip),
+                                     kc.ravel())
+    return kc, st
+
+
+def code_on_grid(x16: int, s16: int, z16: int, L: int) -> int:
+    return int(lib().oracle_code_on_grid(int(x16), int(s16), int(z16), int(L)))
+
+
 def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi: int, tiles_lo: int,
-                       clip: float = 1.0, L_hi_v: int | None = None, L_lo_v: int | None = None):
+                       clip: float = 1.0, L_hi_v: int | None = None, L_lo_v: int | None = None, kc=None):
     """Quantize and place one unit. K16, V16: [T][D] uint16.  L_hi_v, L_lo_v: V level counts of the
-    two segments (default: the K ones). Returns (hi, lo, status)."""
+    two segments (default: the K ones).  kc: per-channel K grids (k_channel_grid), or None for
+    per-token K groups. Returns (hi, lo, status)."""
     K16 = np.ascontiguousarray(K16, dtype=np.uint16)
     V16 = np.ascontiguousarray(V16, dtype=np.uint16)
     T, D = K16.shape
@@ -208,29 +232,31 @@ def quantize_pack_unit(K16, V16, bitmap, G: int, L_hi: int, L_lo: int, tiles_hi:
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
     n = min(len(bitmap), len(bm))
     bm[:n] = bitmap[:n]
+    kc = None if kc is None else np.ascontiguousarray(kc, dtype=np.uint32)
     st = lib().oracle_quantize_pack_unit(K16.ravel(), V16.ravel(), T, D, G, L_hi, L_lo, L_hi_v, L_lo_v, float(clip),
                                          bm, tiles_hi, tiles_lo,
-                                         *_seg_args(hi, lo))
+                                         *_seg_args(hi, lo), _ptr_or_null(kc))
     return hi, lo, st
 
 
 def dequantize_unit(T: int, D: int, G: int, L_hi: int, L_lo: int, bitmap, hi, lo, L_hi_v: int | None = None,
-                    L_lo_v: int | None = None):
+                    L_lo_v: int | None = None, kc=None):
     """Dequantize one unit back to original token order. Returns (Khat, Vhat) fp32 [T][D]."""
     Kh = np.zeros((max(T, 1), D), np.float32)
     Vh = np.zeros((max(T, 1), D), np.float32)
     bm = np.zeros(max((T + 31) // 32, 1), np.uint32)
     n = min(len(bitmap), len(bm))
     bm[:n] = bitmap[:n]
+    kc = None if kc is None else np.ascontiguousarray(kc, dtype=np.uint32)
     lib().oracle_dequantize_unit(T, D, G, L_hi, L_lo, L_hi_v or L_hi, L_lo_v or L_lo, bm, *_seg_args(hi, lo),
-                                 Kh.ravel(), Vh.ravel())
+                                 Kh.ravel(), Vh.ravel(), _ptr_or_null(kc))
     return Kh[:T], Vh[:T]
 
 
 class UnitState:
     """Mutable state of one unit for the append path (bitmap, rank, counts, segments)."""
 
-    def __init__(self, T_cap, bitmap, rank, n_hi, n_lo, tau, hi, lo):
+    def __init__(self, T_cap, bitmap, rank, n_hi, n_lo, tau, hi, lo, kc=None):
         nw = (T_cap + 31) // 32
         self.T_cap = T_cap
         self.bitmap = np.zeros(nw, np.uint32)
@@ -242,6 +268,7 @@ class UnitState:
         self.tau = np.float32(tau)
         self.hi = hi
         self.lo = lo
+        self.kc = None if kc is None else np.ascontiguousarray(kc, dtype=np.uint32)  # per-channel K grids
 
 
 def append_unit(state: UnitState, k16, v16, score: float, G: int, L_hi: int, L_lo: int, clip: float = 1.0,
@@ -256,7 +283,8 @@ def append_unit(state: UnitState, k16, v16, score: float, G: int, L_hi: int, L_l
     st = lib().oracle_append_unit(k16, v16, float(score), float(state.tau), D, G, L_hi, L_lo, L_hi_v or L_hi,
                                   L_lo_v or L_lo, float(clip), state.T_cap,
                                   state.bitmap, state.rank, _c.byref(nh), _c.byref(nl),
-                                  state.hi["k"].shape[0], state.lo["k"].shape[0], *_seg_args(state.hi, state.lo))
+                                  state.hi["k"].shape[0], state.lo["k"].shape[0], *_seg_args(state.hi, state.lo),
+                                  _ptr_or_null(state.kc))
     state.n_hi = nh.value
     state.n_lo = nl.value
     return st

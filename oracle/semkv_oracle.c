@@ -43,8 +43,11 @@
  *               of the most recent tokens forced onto the finer grid at selection; and level
  *               counts of their own for V (keys and values at different bit widths): each segment
  *               has a K level count and a V level count, and each tensor's codes, scale and radix
- *               words use its own.  All are off by default; the formulas are readings, given at
- *               oracle_quantize_group_clip and oracle_select.
+ *               words use its own; and per-channel K grouping (the KVQuant blog page: keys quantized
+ *               per channel): each channel of a unit's K gets one grid, fitted over all prefill
+ *               tokens, and every token of the unit (appended ones too) is coded on it.  All are off
+ *               by default; the formulas are readings, given at oracle_quantize_group_clip,
+ *               oracle_select and oracle_k_channel_grid.
  *   attention   fp64: o = sum_t softmax_t(sigma * q.k^_t) v^_t over all tokens of the unit, for
  *               each of the g query heads that share the kv head (GQA); no mask.
  *
@@ -229,6 +232,19 @@ int oracle_select(const float* score, int32_t T, float p, int32_t window, uint32
 
 /* ------------------------------------------------------------------ quantize and pack */
 
+/* code of one fp16 value on the grid (s16, z16) with L levels: clamp(rint((x - z)/s), 0, L - 1) in
+ * binary32 (RN subtract and divide, ties to even); 0 when s = 0 */
+int oracle_code_on_grid(uint16_t x, uint16_t s16, uint16_t z16, int L)
+{
+    float v = oracle_half_to_float(x), s = oracle_half_to_float(s16), z = oracle_half_to_float(z16);
+    if (s == 0.0f) return 0;
+    float q = (v - z) / s;
+    float r = rintf(q); /* round half to even in the default rounding mode */
+    if (!(r >= 0.0f)) r = 0.0f;
+    if (r > (float)(L - 1)) r = (float)(L - 1);
+    return (int)r;
+}
+
 /*
  * Affine quantization of one group of G fp16 values to L levels (SemKV page, Abstract: a uniform
  * affine grid whose level count need not be a power of two).  Writes G codes, the fp16 scale and
@@ -268,18 +284,9 @@ int oracle_quantize_group_clip(const uint16_t* x, int G, int L, float clip, uint
     }
     float s = oracle_half_to_float(s16);
     float z = oracle_half_to_float(z16);
-    for (int i = 0; i < G; i++) {
-        float v = oracle_half_to_float(x[i]);
-        int c = 0;
-        if (s != 0.0f) {
-            float q = (v - z) / s;
-            float r = rintf(q); /* round half to even in the default rounding mode */
-            if (!(r >= 0.0f)) r = 0.0f;
-            if (r > (float)(L - 1)) r = (float)(L - 1);
-            c = (int)r;
-        }
-        code[i] = (uint8_t)c;
-    }
+    for (int i = 0; i < G; i++) code[i] = (uint8_t)oracle_code_on_grid(x[i], s16, z16, L);
+    (void)s;
+    (void)z;
     *scale_out = s16;
     *zero_out = z16;
     return status;
@@ -289,6 +296,31 @@ int oracle_quantize_group(const uint16_t* x, int G, int L, uint8_t* code, uint16
                           uint16_t* zero_out)
 {
     return oracle_quantize_group_clip(x, G, L, 1.0f, code, scale_out, zero_out);
+}
+
+/*
+ * Per-channel K grids of one unit (prior-art variant; the KVQuant blog page on the same pages names
+ * per-channel key quantization) [reading]: channel d's T prefill values form one group, fitted as
+ * in oracle_quantize_group_clip (same clip) once with L_hi and once with L_lo levels.
+ * kc[d] = hi grid, kc[D + d] = lo grid, each fp16 scale | fp16 zero << 16.  Tokens appended later
+ * are coded on the same grids (clamped), since the pages give no rule for refitting them.
+ */
+int oracle_k_channel_grid(const uint16_t* K, int32_t T, int D, int L_hi, int L_lo, float clip, uint32_t* kc)
+{
+    int status = 0;
+    uint16_t* col = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(T > 0 ? T : 1));
+    uint8_t* codes = (uint8_t*)malloc((size_t)(T > 0 ? T : 1));
+    for (int d = 0; d < D; d++) {
+        for (int32_t t = 0; t < T; t++) col[t] = K[(size_t)t * D + d];
+        uint16_t s16 = 0, z16 = 0;
+        if (T > 0) status |= oracle_quantize_group_clip(col, T, L_hi, clip, codes, &s16, &z16);
+        kc[d] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+        if (T > 0) status |= oracle_quantize_group_clip(col, T, L_lo, clip, codes, &s16, &z16);
+        kc[D + d] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+    }
+    free(col);
+    free(codes);
+    return status;
 }
 
 /* word = sum_i c_i L^i over k codes (base-L positional notation, lowest index least significant) */
@@ -360,8 +392,9 @@ int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, i
                               int L_lo, int L_hi_v, int L_lo_v, float clip, const uint32_t* bitmap, int tiles_hi,
                               int tiles_lo,
                               uint32_t* k_hi, uint32_t* v_hi, uint32_t* kz_hi, uint32_t* vz_hi,
-                              uint32_t* k_lo, uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo)
+                              uint32_t* k_lo, uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo, const uint32_t* kc)
 {
+    /* kc: per-channel K grids (oracle_k_channel_grid), or NULL for per-token K groups */
     if (D <= 0 || G <= 0 || D % G != 0 || L_hi < 2 || L_lo < 2 || L_hi > 256 || L_lo > 256 ||
         L_hi_v < 2 || L_lo_v < 2 || L_hi_v > 256 || L_lo_v > 256 || !(clip > 0.0f && clip <= 1.0f))
         return OR_BAD_ARG;
@@ -393,9 +426,20 @@ int oracle_quantize_pack_unit(const uint16_t* K, const uint16_t* V, int32_t T, i
         int tile = slot / OR_TILE, tt = slot % OR_TILE;
         for (int grp = 0; grp < NG; grp++) {
             uint16_t s16, z16;
-            status |= oracle_quantize_group_clip(K + (size_t)t * D + grp * G, G, Ls[seg], clip,
-                                                 ck[seg] + (size_t)slot * D + grp * G, &s16, &z16);
-            kz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+            if (kc) { /* K on its channels' grids; the per-token K scale/zero stay 0 */
+                for (int d = grp * G; d < (grp + 1) * G; d++) {
+                    uint32_t g = kc[(size_t)seg * D + d];
+                    uint16_t x = K[(size_t)t * D + d];
+                    if (!isfinite(oracle_half_to_float(x))) status |= OR_NONFINITE_KV;
+                    ck[seg][(size_t)slot * D + d] =
+                        (uint8_t)oracle_code_on_grid(x, (uint16_t)(g & 0xFFFF), (uint16_t)(g >> 16), Ls[seg]);
+                }
+                kz[seg][sz_index(tile, grp, tt, NG)] = 0;
+            } else {
+                status |= oracle_quantize_group_clip(K + (size_t)t * D + grp * G, G, Ls[seg], clip,
+                                                     ck[seg] + (size_t)slot * D + grp * G, &s16, &z16);
+                kz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+            }
             status |= oracle_quantize_group_clip(V + (size_t)t * D + grp * G, G, Lvs[seg], clip,
                                                  cv[seg] + (size_t)slot * D + grp * G, &s16, &z16);
             vz[seg][sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
@@ -435,7 +479,8 @@ void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, int L_h
                             const uint32_t* bitmap,
                             const uint32_t* k_hi, const uint32_t* v_hi, const uint32_t* kz_hi,
                             const uint32_t* vz_hi, const uint32_t* k_lo, const uint32_t* v_lo,
-                            const uint32_t* kz_lo, const uint32_t* vz_lo, float* Khat, float* Vhat)
+                            const uint32_t* kz_lo, const uint32_t* vz_lo, float* Khat, float* Vhat,
+                            const uint32_t* kgrid)
 {
     int NG = D / G;
     const uint32_t* kw[2] = {k_hi, k_lo};
@@ -454,7 +499,7 @@ void oracle_dequantize_unit(int32_t T, int D, int G, int L_hi, int L_lo, int L_h
         segment_codes(kw[seg], vw[seg], D, Ls[seg], Lvs[seg], slot, kc, vc);
         for (int d = 0; d < D; d++) {
             int grp = d / G;
-            uint32_t kzv = kz[seg][sz_index(tile, grp, tt, NG)];
+            uint32_t kzv = kgrid ? kgrid[(size_t)seg * D + d] : kz[seg][sz_index(tile, grp, tt, NG)];
             uint32_t vzv = vz[seg][sz_index(tile, grp, tt, NG)];
             float ks = oracle_half_to_float((uint16_t)(kzv & 0xFFFF));
             float kz0 = oracle_half_to_float((uint16_t)(kzv >> 16));
@@ -481,7 +526,8 @@ int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float 
                        int L_hi, int L_lo, int L_hi_v, int L_lo_v, float clip, int32_t T_cap, uint32_t* bitmap, uint32_t* rank,
                        int32_t* n_hi, int32_t* n_lo, int tiles_hi, int tiles_lo, uint32_t* k_hi,
                        uint32_t* v_hi, uint32_t* kz_hi, uint32_t* vz_hi, uint32_t* k_lo,
-                       uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo)
+                       uint32_t* v_lo, uint32_t* kz_lo, uint32_t* vz_lo,
+                       const uint32_t* kgrid)
 {
     int status = 0;
     if (isnan(score)) status |= OR_NAN_SCORE;
@@ -506,8 +552,17 @@ int oracle_append_unit(const uint16_t* k, const uint16_t* v, float score, float 
     int tile = slot / OR_TILE, tt = slot % OR_TILE;
     for (int grp = 0; grp < NG; grp++) {
         uint16_t s16, z16;
-        status |= oracle_quantize_group_clip(k + grp * G, G, L, clip, kc + grp * G, &s16, &z16);
-        kz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+        if (kgrid) { /* per-channel K grids fitted at prefill (clamped) */
+            for (int d = grp * G; d < (grp + 1) * G; d++) {
+                uint32_t g = kgrid[(size_t)seg * D + d];
+                if (!isfinite(oracle_half_to_float(k[d]))) status |= OR_NONFINITE_KV;
+                kc[d] = (uint8_t)oracle_code_on_grid(k[d], (uint16_t)(g & 0xFFFF), (uint16_t)(g >> 16), L);
+            }
+            kz[sz_index(tile, grp, tt, NG)] = 0;
+        } else {
+            status |= oracle_quantize_group_clip(k + grp * G, G, L, clip, kc + grp * G, &s16, &z16);
+            kz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
+        }
         status |= oracle_quantize_group_clip(v + grp * G, G, Lv, clip, vc + grp * G, &s16, &z16);
         vz[sz_index(tile, grp, tt, NG)] = (uint32_t)s16 | ((uint32_t)z16 << 16);
     }

@@ -226,3 +226,66 @@ def test_separate_v_levels_appends_equal_a_prefill():
     for a, b in ((st.hi, hi2), (st.lo, lo2)):
         for n in a:
             assert np.array_equal(a[n], b[n]), n
+
+
+# ---------------------------------------------------------------- per-channel K grids
+
+
+def test_k_channel_grid_worked_by_hand():
+    """Channel 0 holds -1, 0, 1, 2 over four tokens (the other channels 0).  Its hi grid (L 5) is
+    s = 3/4 = 0.75 (exact), z = -1; its lo grid (L 3) s = 1.5, z = -1.  Tokens 0, 2 on hi and 1, 3
+    on lo: codes 0 ((-1+1)/0.75), 1 ((0+1)/1.5 = 0.67), 3 ((1+1)/0.75 = 2.67), 2 ((2+1)/1.5)
+    -> dequantized -1, 0.5, 1.25, 2.  Constant channels get s = 0, z = 0."""
+    T, D = 4, 128
+    K = np.zeros((T, D), np.float16)
+    K[:, 0] = [-1, 0, 1, 2]
+    K16 = K.view(np.uint16)
+    kc, st = oracle.k_channel_grid(K16, 5, 3)
+    assert st == 0
+    assert kc[0, 0] == (0x3A00 | (0xBC00 << 16))  # 0.75 | -1.0
+    assert kc[1, 0] == (0x3E00 | (0xBC00 << 16))  # 1.5 | -1.0
+    assert (kc[:, 1:] == 0).all()
+    bm = np.array([0b0101], np.uint32)
+    V = np.zeros((T, D), np.float16).view(np.uint16)
+    hi, lo, st = oracle.quantize_pack_unit(K16, V, bm, 64, 5, 3, 1, 1, kc=kc)
+    assert st == 0
+    assert not hi["kz"].any() and not lo["kz"].any()  # no per-token K grids in this mode
+    Kh, _ = oracle.dequantize_unit(T, D, 64, 5, 3, bm, hi, lo, kc=kc)
+    assert Kh[:, 0].tolist() == [-1.0, 0.5, 1.25, 2.0]
+    assert not Kh[:, 1:].any()
+
+
+def test_k_channel_grid_appends_clamp_to_the_prefill_grid():
+    T, D = 4, 128
+    K = np.zeros((T, D), np.float16)
+    K[:, 0] = [-1, 0, 1, 2]
+    kc, _ = oracle.k_channel_grid(K.view(np.uint16), 5, 3)
+    bm, rk, nh, tau, _ = oracle.select(np.float32([3, 0, 2, 1]), 0.5)  # tokens 0, 2 hi; tau = 2
+    hi, lo, _ = oracle.quantize_pack_unit(K.view(np.uint16), np.zeros((T, D), np.uint16), bm, 64, 5, 3, 1, 1, kc=kc)
+    st = oracle.UnitState(32, bm, rk, nh, T - nh, tau, hi, lo, kc=kc)
+    for x, score in ((5.0, 9.0), (-3.0, 9.0), (0.4, -9.0)):  # hi, hi, lo
+        k = np.zeros(D, np.float16)
+        k[0] = x
+        assert oracle.append_unit(st, k.view(np.uint16), np.zeros(D, np.uint16), score, 64, 5, 3) == 0
+    Kh, _ = oracle.dequantize_unit(T + 3, D, 64, 5, 3, st.bitmap, st.hi, st.lo, kc=kc)
+    # 5 -> top hi code 4 -> 2.0; -3 -> code 0 -> -1.0; 0.4 on lo: (0.4+1)/1.5 = 0.93 -> 1 -> 0.5
+    assert Kh[T:, 0].tolist() == [2.0, -1.0, 0.5]
+
+
+def test_k_channel_grid_error_bound_and_v_untouched():
+    r = np.random.default_rng(15)
+    T, D, G = 300, 128, 64
+    K = (r.standard_normal((T, D)) * r.uniform(0.1, 8, D)).astype(np.float16)
+    V = r.standard_normal((T, D)).astype(np.float16).view(np.uint16)
+    bm, _, _, _, _ = oracle.select(r.standard_normal(T).astype(np.float32), 0.3)
+    kc, _ = oracle.k_channel_grid(K.view(np.uint16), 8, 5)
+    hi, lo, _ = oracle.quantize_pack_unit(K.view(np.uint16), V, bm, G, 8, 5, 3, 3, kc=kc)
+    hi0, lo0, _ = oracle.quantize_pack_unit(K.view(np.uint16), V, bm, G, 8, 5, 3, 3)
+    for a, b in ((hi, hi0), (lo, lo0)):
+        assert np.array_equal(a["v"], b["v"]) and np.array_equal(a["vz"], b["vz"])
+    Kh, _ = oracle.dequantize_unit(T, D, G, 8, 5, bm, hi, lo, kc=kc)
+    is_hi = np.unpackbits(bm.view(np.uint8), bitorder="little")[:T].astype(bool)
+    s = np.where(is_hi[:, None], (kc[0] & 0xFFFF).astype(np.uint16).view(np.float16)[None, :],
+                 (kc[1] & 0xFFFF).astype(np.uint16).view(np.float16)[None, :]).astype(np.float64)
+    err = np.abs(Kh.astype(np.float64) - K.astype(np.float64))
+    assert (err <= s / 2 + 1e-6 * (1 + np.abs(K.astype(np.float64)))).all()
