@@ -455,6 +455,21 @@ def run_semkv(args):
     t_kvq = timed(kvq_graph, before=(graphs[0],))
     t_kvd = timed(kvd_graph, before=(graphs[0], kvq_graph))
     nb_kv = alg_bytes(w, T, n_hi0, v_levels=V_LEVELS)
+    # per-channel K grids: quantize (grid pass over K, then the runtime-L kernel) and decode (CUDA cores)
+    cache.struct.k_per_channel = 1
+    calls[0]()
+    calls[1]()
+    kpq_graph, kpd_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(kpq_graph, capture_error_mode="relaxed"):
+        calls[1]()
+    kv_decode()
+    with torch.cuda.graph(kpd_graph, capture_error_mode="relaxed"):
+        kv_decode()
+    cache.struct.k_per_channel = 0
+    torch.cuda.synchronize()
+    t_kpq = timed(kpq_graph, before=(graphs[0],))
+    t_kpd = timed(kpd_graph, before=(graphs[0], kpq_graph))
+    kpc_range_bytes = w.B * w.H * T * w.D * 2  # the grid pass reads K once more
     assert cache.status() == 0, f"device status {cache.status()}"
     assert torch.equal(out, out_s), "append+decode in one pass differs from append then decode"
     # leave the cache as a timed step leaves it (prefill + the fixed-threshold append)
@@ -493,6 +508,8 @@ def run_semkv(args):
         f"quantize_clip{CLIP}": {"ms": t_clip, "gbs": nb["quantize"] / (t_clip * 1e-3) / 1e9},
         "quantize_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvq, "gbs": nb_kv["quantize"] / (t_kvq * 1e-3) / 1e9},
         "decode_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvd, "gbs": nb_kv["decode"] / (t_kvd * 1e-3) / 1e9},
+        "quantize_k_per_channel": {"ms": t_kpq, "gbs": (nb["quantize"] + kpc_range_bytes) / (t_kpq * 1e-3) / 1e9},
+        "decode_k_per_channel": {"ms": t_kpd, "gbs": nb["decode"] / (t_kpd * 1e-3) / 1e9},
     })
     dom = max(("select", "quantize", "append_decode"), key=lambda k: per_kernel[k]["ms"])
     dom_name = {"select": "semkv_assign_precision (k_select_cluster)",

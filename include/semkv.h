@@ -105,10 +105,18 @@ typedef struct semkv_cache {
      *   L_hi_v, L_lo_v: level counts of the V codes of each segment (keys and values at different
      *           bit widths); 0 = the K level count (L_hi, L_lo), else in [2, 256].  The V words of a
      *           segment then hold k(L_v) codes each.  The tensor-core decode serves equal K and V
-     *           counts; other segments run on the CUDA-core decode. */
+     *           counts; other segments run on the CUDA-core decode.
+     *   k_per_channel: 0 = K grids per token and group of G channels (the plain method); 1 = one K
+     *           grid per channel of each unit (keys quantized per channel), fitted by
+     *           semkv_quantize_pack over all T prefill tokens (min and max of the channel, the clip
+     *           applied), once on the L_hi and once on the L_lo levels, and kept in the `kc` buffer;
+     *           every K code of the unit, appended tokens included, is coded on its channel's grid
+     *           of its segment, clamped to [0, L-1]; the per-token K scale/zero are 0.  Decoded on
+     *           the CUDA-core decode. */
     int32_t window;
     float clip;
     int32_t L_hi_v, L_lo_v;
+    int32_t k_per_channel;
     uint32_t *k_hi, *v_hi, *kz_hi, *vz_hi;
     uint32_t *k_lo, *v_lo, *kz_lo, *vz_lo;
     uint32_t *bitmap, *rank;
@@ -117,13 +125,14 @@ typedef struct semkv_cache {
     int32_t *status;
     int32_t *slot_token;  /* [B*H][cap_hi + cap_lo], see the layout above */
     uint32_t *score_keys; /* [B*H][T_cap], see the layout above */
+    uint32_t *kc;         /* [B*H][2][D] per-channel K grids (hi, lo): fp16 scale | fp16 zero << 16 */
 } semkv_cache_t;
 
 enum {
     SEMKV_BUF_K_HI = 0, SEMKV_BUF_V_HI, SEMKV_BUF_KZ_HI, SEMKV_BUF_VZ_HI,
     SEMKV_BUF_K_LO, SEMKV_BUF_V_LO, SEMKV_BUF_KZ_LO, SEMKV_BUF_VZ_LO,
     SEMKV_BUF_BITMAP, SEMKV_BUF_RANK, SEMKV_BUF_N_HI, SEMKV_BUF_N_LO, SEMKV_BUF_TAU, SEMKV_BUF_STATUS,
-    SEMKV_BUF_SLOT_TOKEN, SEMKV_BUF_SCORE_KEYS, SEMKV_NBUF
+    SEMKV_BUF_SLOT_TOKEN, SEMKV_BUF_SCORE_KEYS, SEMKV_BUF_KC, SEMKV_NBUF
 };
 
 /* Byte size of each of the SEMKV_NBUF buffers of a cache with the shape fields of `shape`

@@ -27,7 +27,7 @@ STATUS_TIMEOUT = 16
 
 SHAPE_FIELDS = ("B", "H", "Hq", "D", "G", "L_hi", "L_lo", "cap_hi", "cap_lo", "T_cap")
 BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
-             "bitmap", "rank", "n_hi", "n_lo", "tau", "status", "slot_token", "score_keys")
+             "bitmap", "rank", "n_hi", "n_lo", "tau", "status", "slot_token", "score_keys", "kc")
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
             "semkv_append_token", "semkv_append_token_running", "semkv_append_decode", "semkv_decode_attention",
             "semkv_decode_attention_noalloc", "semkv_dequantize", "semkv_status_string", "semkv_radix_digits",
@@ -36,9 +36,11 @@ NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
 class CacheStruct(ctypes.Structure):
-    """Mirror of semkv_cache_t (window, clip, L_hi_v, L_lo_v: the quantizer variants; 0 = off)."""
+    """Mirror of semkv_cache_t (window, clip, L_hi_v, L_lo_v, k_per_channel: the quantizer variants;
+    0 = off)."""
     _fields_ = [(n, ctypes.c_int32) for n in SHAPE_FIELDS] + \
-        [("window", ctypes.c_int32), ("clip", ctypes.c_float), ("L_hi_v", ctypes.c_int32), ("L_lo_v", ctypes.c_int32)] + \
+        [("window", ctypes.c_int32), ("clip", ctypes.c_float), ("L_hi_v", ctypes.c_int32), ("L_lo_v", ctypes.c_int32),
+         ("k_per_channel", ctypes.c_int32)] + \
         [(n, ctypes.c_void_p) for n in BUF_NAMES]
 
 

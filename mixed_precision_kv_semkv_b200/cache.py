@@ -29,18 +29,19 @@ def capacities(T: int, p: float, extra: int = 0, window: int = 0):
 
 
 class SemkvCache:
-    """One layer's cache: device buffers + the semkv_cache_t descriptor.  window, clip, L_hi_v and
-    L_lo_v select the quantizer variants (recent tokens forced onto the finer grid; clipped group
-    range; V level counts of their own); 0 is the plain method."""
+    """One layer's cache: device buffers + the semkv_cache_t descriptor.  window, clip, L_hi_v,
+    L_lo_v and k_per_channel select the quantizer variants (recent tokens forced onto the finer
+    grid; clipped group range; V level counts of their own; per-channel K grids); 0 is the plain
+    method."""
 
     def __init__(self, B: int, H: int, Hq: int, G: int, L_hi: int, L_lo: int, cap_hi: int, cap_lo: int,
                  T_cap: int, D: int = 128, device="cuda", window: int = 0, clip: float = 0.0, L_hi_v: int = 0,
-                 L_lo_v: int = 0):
+                 L_lo_v: int = 0, k_per_channel: int = 0):
         import torch
 
         self.struct = _lib.CacheStruct(B=B, H=H, Hq=Hq, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=cap_hi,
                                        cap_lo=cap_lo, T_cap=T_cap, window=window, clip=clip, L_hi_v=L_hi_v,
-                                       L_lo_v=L_lo_v)
+                                       L_lo_v=L_lo_v, k_per_channel=int(k_per_channel))
         sizes = _lib.semkv_cache_bytes(self.struct)
         self.sizes = dict(zip(_lib.BUF_NAMES, sizes))
         self.bufs = {}
@@ -51,14 +52,15 @@ class SemkvCache:
             setattr(self.struct, name, int(t.data_ptr()))
         self.bufs["status"].zero_()
         self.shape = dict(B=B, H=H, Hq=Hq, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=cap_hi, cap_lo=cap_lo,
-                          T_cap=T_cap, window=window, clip=clip, L_hi_v=L_hi_v or L_hi, L_lo_v=L_lo_v or L_lo)
+                          T_cap=T_cap, window=window, clip=clip, L_hi_v=L_hi_v or L_hi, L_lo_v=L_lo_v or L_lo,
+                          k_per_channel=int(k_per_channel))
 
     @classmethod
     def for_prefill(cls, B, H, Hq, G, L_hi, L_lo, T, p, extra=0, device="cuda", window=0, clip=0.0, L_hi_v=0,
-                    L_lo_v=0):
+                    L_lo_v=0, k_per_channel=0):
         ch, cl, tc = capacities(T, p, extra, window)
         return cls(B, H, Hq, G, L_hi, L_lo, ch, cl, tc, device=device, window=window, clip=clip, L_hi_v=L_hi_v,
-                   L_lo_v=L_lo_v)
+                   L_lo_v=L_lo_v, k_per_channel=k_per_channel)
 
     def __getattr__(self, name):
         shape = self.__dict__.get("shape", {})

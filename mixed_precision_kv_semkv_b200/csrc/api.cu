@@ -26,6 +26,7 @@ int validate_shape(const semkv_cache_t* c)
     if (c->Hq / c->H > 8) return SEMKV_ERR_UNSUPPORTED;
     if (c->window < 0 || !(c->clip == 0.0f || (c->clip > 0.0f && c->clip <= 1.0f))) return SEMKV_ERR_INVALID_ARG;
     if ((c->L_hi_v && !level_ok(c->L_hi_v)) || (c->L_lo_v && !level_ok(c->L_lo_v))) return SEMKV_ERR_UNSUPPORTED;
+    if (c->k_per_channel != 0 && c->k_per_channel != 1) return SEMKV_ERR_INVALID_ARG;
     return SEMKV_OK;
 }
 
@@ -33,7 +34,7 @@ int validate_ptrs(const semkv_cache_t* c)
 {
     const void* p[] = {c->k_hi, c->v_hi, c->kz_hi, c->vz_hi, c->k_lo, c->v_lo, c->kz_lo, c->vz_lo,
                        c->bitmap, c->rank, c->n_hi, c->n_lo, c->tau, c->status, c->slot_token,
-                       c->score_keys};
+                       c->score_keys, c->kc};
     for (const void* x : p)
         if (!x) return SEMKV_ERR_INVALID_ARG;
     return SEMKV_OK;
@@ -97,6 +98,7 @@ SegView seg_view(const semkv_cache_t* c, bool hi)
     s.Lv = level_v(*c, hi);
     s.tiles_cap = (hi ? c->cap_hi : c->cap_lo) / TILE;
     s.is_hi = hi ? 1 : 0;
+    s.kc = c->k_per_channel ? c->kc + (hi ? 0 : 128) : nullptr;
     return s;
 }
 
@@ -130,7 +132,7 @@ static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_
         const SegView sv = seg_view(c, hi != 0);
         const int ns = hi ? nh : nl, off = hi ? 0 : nh;
         if (ns == 0) continue;
-        if (decode_tc_supported(sv.L, sv.Lv, c->G, g)) {
+        if (!c->k_per_channel && decode_tc_supported(sv.L, sv.Lv, c->G, g)) {
             launch_decode_tc(sv, q, units, c->H, g, c->G, scale_log2, ns, off, nh + nl, ws, c->status, dependent, app,
                              st);
         } else {
@@ -198,6 +200,7 @@ int semkv_cache_bytes(const semkv_cache_t* c, size_t sizes[SEMKV_NBUF])
     sizes[SEMKV_BUF_STATUS] = 4;
     sizes[SEMKV_BUF_SLOT_TOKEN] = units * (size_t)(c->cap_hi + c->cap_lo) * 4;
     sizes[SEMKV_BUF_SCORE_KEYS] = units * (size_t)c->T_cap * 4;
+    sizes[SEMKV_BUF_KC] = units * 2 * (size_t)c->D * 4;
     return SEMKV_OK;
 }
 
@@ -230,10 +233,14 @@ int semkv_quantize_pack(const semkv_cache_t* c, const uint16_t* K, const uint16_
     int r = validate(c);
     if (r != SEMKV_OK) return r;
     if (T < 0 || T > c->T_cap || ((!K || !V) && T > 0)) return SEMKV_ERR_INVALID_ARG;
-    if (T == 0) return SEMKV_OK;
+    if (T == 0) {  // nothing to place; per-channel K grids of an empty prefill are zero
+        if (c->k_per_channel) launch_kc_grids(*c, K, 0, (cudaStream_t)stream);
+        return launch_status();
+    }
     if ((((uintptr_t)K) | ((uintptr_t)V)) & 15u) return SEMKV_ERR_INVALID_ARG;  // rows are fetched by bulk copies
+    if (c->k_per_channel) launch_kc_grids(*c, K, T, (cudaStream_t)stream);  // grids first: the codes use them
     launch_quantize(seg_view(c, true), seg_view(c, false), K, V, c->slot_token, c->B * c->H, T, c->D, c->G,
-                    clip_ratio(*c), c->status, (cudaStream_t)stream);
+                    clip_ratio(*c), c->k_per_channel ? c->kc : nullptr, c->status, (cudaStream_t)stream);
     return launch_status();
 }
 
@@ -273,7 +280,7 @@ int semkv_append_decode(const semkv_cache_t* c, const uint16_t* k, const uint16_
     if (r != SEMKV_OK) return r;
     if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
     const int g = c->Hq / c->H;
-    if (!decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g) ||
+    if (c->k_per_channel || !decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g) ||
         !decode_tc_supported(c->L_lo, level_v(*c, false), c->G, g)) {
         // shapes the fused path does not cover: the two calls, in order
         launch_append(*c, k, v, score, -1.0f, (cudaStream_t)stream);

@@ -69,10 +69,16 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
     group_scale_zero(vmn, vmx, Lv, clip, vs16, vz16);
     const int grp = d / G;
     if (d % G == 0) {
-        kz[grp * TILE + tt] = (uint32_t)ks16 | ((uint32_t)kz16 << 16);
+        // per-channel K grids: no per-token K grid
+        kz[grp * TILE + tt] = c.k_per_channel ? 0u : (uint32_t)ks16 | ((uint32_t)kz16 << 16);
         vz[grp * TILE + tt] = (uint32_t)vs16 | ((uint32_t)vz16 << 16);
     }
-    kc[d] = quant_code(kx, h2f(kz16), h2f(ks16), L);
+    if (c.k_per_channel) {  // the channel's grid of this segment, fitted at prefill (clamped)
+        const uint32_t gk = c.kc[(size_t)u * 2 * D + (hi ? 0 : D) + d];
+        kc[d] = quant_code(kx, h2f((uint16_t)(gk >> 16)), h2f((uint16_t)(gk & 0xffffu)), L);
+    } else {
+        kc[d] = quant_code(kx, h2f(kz16), h2f(ks16), L);
+    }
     const uint32_t cv = (uint32_t)quant_code(vx, h2f(vz16), h2f(vs16), Lv);
     const bool bad = !isfinite(kx) || !isfinite(vx);
     __syncthreads();

@@ -74,6 +74,31 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
         qsum[grp * GMAX + h] = s;
     }
     __syncthreads();
+    // per-channel K grids: q_hd s_d replaces q_hd (the scale folds into the query) and the zero
+    // terms sum_d q_hd (z_d + m s_d) become one constant per head
+    __shared__ float kzt[GMAX];
+    if (seg.kc) {
+        float v[GMAX];
+        {
+            const uint32_t gk = seg.kc[(size_t)u * 256 + tid];  // thread = channel (128 threads)
+            const float s = h2f((uint16_t)(gk & 0xffffu));
+            const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(gk >> 16)));
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) {
+                v[h] = h < g ? qs[tid * GMAX + h] * zc : 0.f;
+                if (h < g) qs[tid * GMAX + h] *= s;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v[h] += __shfl_xor_sync(0xffffffffu, v[h], o);
+            if (lane == 0) red[warp * GMAX + h] = v[h];
+        }
+        __syncthreads();
+        if (tid < GMAX) kzt[tid] = red[tid] + red[GMAX + tid] + red[2 * GMAX + tid] + red[3 * GMAX + tid];
+        __syncthreads();
+    }
 
     const int n = seg.n[u];
     const int tiles = min(ceil_div(n, TILE), seg.tiles_cap);  // never past the segment's capacity
@@ -99,15 +124,24 @@ __global__ void __launch_bounds__(128) k_decode_split(SegView seg, const uint16_
         // ---- K side: thread = slot
         float logit[GMAX], a[GMAX];
 #pragma unroll
-        for (int h = 0; h < GMAX; ++h) logit[h] = a[h] = 0.f;
+        for (int h = 0; h < GMAX; ++h) {
+            logit[h] = seg.kc ? kzt[h] : 0.f;
+            a[h] = 0.f;
+        }
         int cur = 0;
         auto flush = [&](int grp) {
-            const uint32_t zz = kz[grp * TILE + tid];
-            const float s = h2f((uint16_t)(zz & 0xffffu));
-            const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(zz >> 16)));
+            if (seg.kc) {  // the channel scales are in qs
 #pragma unroll
-            for (int h = 0; h < GMAX; ++h)
-                if (h < g) logit[h] += s * a[h] + zc * qsum[grp * GMAX + h];
+                for (int h = 0; h < GMAX; ++h)
+                    if (h < g) logit[h] += a[h];
+            } else {
+                const uint32_t zz = kz[grp * TILE + tid];
+                const float s = h2f((uint16_t)(zz & 0xffffu));
+                const float zc = __fmaf_rn(mid, s, h2f((uint16_t)(zz >> 16)));
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h)
+                    if (h < g) logit[h] += s * a[h] + zc * qsum[grp * GMAX + h];
+            }
 #pragma unroll
             for (int h = 0; h < GMAX; ++h) a[h] = 0.f;
         };

@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(128) k_dequantize(semkv_cache_t c, int T, floa
     float* ko = Kout + ((size_t)u * T + t) * D;
     float* vo = Vout + ((size_t)u * T + t) * D;
     for (int d = 0; d < D; ++d) {
-        const uint32_t kzv = kz[(d / G) * TILE + tt], vzv = vz[(d / G) * TILE + tt];
+        const uint32_t kzv = c.k_per_channel ? c.kc[(size_t)u * 2 * D + (hi ? 0 : D) + d] : kz[(d / G) * TILE + tt];
+        const uint32_t vzv = vz[(d / G) * TILE + tt];
         const int ck = digit_rt(kw[(d / k) * TILE + tt], L, d % k);
         const int cv = digit_rt(vw[(tt / kv) * D + d], Lv, tt % kv);
         ko[d] = __fmaf_rn((float)ck, h2f((uint16_t)(kzv & 0xffffu)), h2f((uint16_t)(kzv >> 16)));

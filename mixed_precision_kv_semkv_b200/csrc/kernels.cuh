@@ -28,6 +28,7 @@ struct SegView {
     int Lv;         // levels of the V codes
     int tiles_cap;  // capacity in tiles of 128 slots
     int is_hi;      // 1: L_hi segment (bitmap bit 1), 0: L_lo segment
+    const uint32_t* kc;  // per-channel K grids of this segment (unit u at + u * 256), or null
 };
 
 // A generated token to append while decoding (k == nullptr: none); the fixed-threshold rule.
@@ -46,8 +47,11 @@ void launch_select(const float* scores, int units, int T, int n_sel, int window,
 
 // reads the slot map (slot_token) that launch_select wrote
 void launch_quantize(const SegView& hi, const SegView& lo, const uint16_t* K, const uint16_t* V,
-                     const int32_t* slot_token, int units, int T, int D, int G, float clip, int32_t* status,
-                     cudaStream_t st);
+                     const int32_t* slot_token, int units, int T, int D, int G, float clip, const uint32_t* kc,
+                     int32_t* status, cudaStream_t st);
+
+// per-channel K grids of every unit from the prefill's K (kchannel.cu)
+void launch_kc_grids(const semkv_cache_t& c, const uint16_t* K, int T, cudaStream_t st);
 
 // p < 0: the fixed threshold rule (score > tau); p in [0, 1]: the running top-p rule
 void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, float p,

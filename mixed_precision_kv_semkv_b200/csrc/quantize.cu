@@ -36,6 +36,7 @@ struct QuantSeg {
     int map_stride;
     int L, k_digits, tiles_cap, is_hi;
     int Lv, kv_digits;  // V codes: level count and codes per word
+    const uint32_t* kc;  // per-channel K grids of this segment (unit u at + u * 256), or null
 };
 
 __device__ __forceinline__ void half8(const uint16_t* p, float (&f)[8])
@@ -134,7 +135,14 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
     uint16_t* Ks = reinterpret_cast<uint16_t*>(smem);
     uint16_t* Vs = Ks + TILE * QROW;
     float4* vgrid = reinterpret_cast<float4*>(Vs + TILE * QROW);  // [TILE][NG] (s, r, z, -)
+    float4* cgrid = vgrid + TILE * NG;                             // [128] per-channel K grids
+    if (seg.kc) {
+        const uint32_t gk = seg.kc[(size_t)u * 256 + tid];
+        const float s = h2f((uint16_t)(gk & 0xffffu)), z = h2f((uint16_t)(gk >> 16));
+        cgrid[tid] = make_float4(s, s != 0.0f ? __frcp_rn(s) : 0.0f, z, 0.0f);
+    }
     gather_rows_warp(Ks, Vs, seg, u, s0, nv, K, V, T);
+    __syncthreads();  // the channel grids (the rows are per warp)
 
     const size_t tile_base = (size_t)u * seg.tiles_cap + tile;
     uint32_t* kw = seg.k + tile_base * WK * TILE;
@@ -163,13 +171,20 @@ __global__ void __launch_bounds__(128) k_quantize(QuantSeg hi, QuantSeg lo, cons
             }
             uint32_t packed;
             const Grid g = make_grid(mn, mx, L, clip, &packed);
-            kz[grp * TILE + tid] = packed;
+            kz[grp * TILE + tid] = seg.kc ? 0u : packed;  // per-channel K grids: no per-token grid
             for (int i = G - 8; i >= 0; i -= 8) {
                 float f[8];
                 half8(row + grp * G + i, f);
 #pragma unroll
                 for (int j = 7; j >= 0; --j) {
-                    w = w * (uint32_t)L + code_of(f[j], g, top);
+                    uint32_t code;
+                    if (seg.kc) {  // slots past the segment's end hold zero codes, as on the plain grids
+                        const float4 cg = cgrid[grp * G + i + j];
+                        code = tid < nv ? code_of(f[j], Grid{cg.x, cg.y, cg.z}, top) : 0u;
+                    } else {
+                        code = code_of(f[j], g, top);
+                    }
+                    w = w * (uint32_t)L + code;
                     if (dig == 0) {
                         kw[widx * TILE + tid] = w;
                         w = 0u;
@@ -491,12 +506,12 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
 
 static size_t quantize_smem(int G)
 {
-    return (size_t)2 * TILE * QROW * 2 + (size_t)TILE * (128 / G) * 16;
+    return (size_t)2 * TILE * QROW * 2 + (size_t)TILE * (128 / G) * 16 + 128 * 16;
 }
 
 void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, const uint16_t* V,
                      const int32_t* slot_token, int units, int T, int D, int G, float clip,
-                     int32_t* status, cudaStream_t st)
+                     const uint32_t* kc, int32_t* status, cudaStream_t st)
 {
     (void)D;
     const int per_unit = shi.tiles_cap + slo.tiles_cap;
@@ -513,6 +528,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
         q.k_digits = radix_k(s.L);
         q.Lv = s.Lv;
         q.kv_digits = radix_k(s.Lv);
+        q.kc = kc ? kc + (s.is_hi ? 0 : 128) : nullptr;
         q.tiles_cap = s.tiles_cap;
         q.is_hi = s.is_hi;
         q.map = map;
@@ -525,6 +541,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     // compile-time level counts and group sizes of the common configurations; the quantizer
     // variants (a clip, V level counts of their own) for a few of them, the rest on k_quantize
     const bool clipped = clip != 1.0f;
+    if (!kc) {
 #define SEMKV_QF(LH, LL, LHV, LLV, GG, CL)                                                                    \
     if (clipped == CL && shi.L == LH && slo.L == LL && shi.Lv == LHV && slo.Lv == LLV && G == GG) {           \
         const size_t sm = (size_t)TILE * QROW * 2;                                                            \
@@ -540,6 +557,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     SEMKV_QF(16, 8, 8, 4, 64, false)
 #undef SEMKV_QF_G
 #undef SEMKV_QF
+    }  // per-channel K grids: the runtime-L kernel below
     const size_t sm = quantize_smem(G);
     cudaFuncSetAttribute(k_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     k_quantize<<<grid, 128, sm, st>>>(qh, ql, K, V, T, G, clip, status);

@@ -45,6 +45,7 @@ def unit_views(cache: SemkvCache, bufs: dict, u: int):
     caps = cache.cap_hi + cache.cap_lo
     st = bufs["slot_token"].view(np.int32)[: units * caps].reshape(units, caps)[u]
     out["slot_hi"], out["slot_lo"] = st[: cache.cap_hi], st[cache.cap_hi:]
+    out["kc"] = bufs["kc"].view(np.uint32)[: units * 2 * D].reshape(units, 2, D)[u]
     return out
 
 
@@ -55,13 +56,13 @@ def fetch(cache: SemkvCache) -> dict:
     return {n: t.cpu().numpy() for n, t in cache.bufs.items()}
 
 
-def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0, L_hi_v=0, L_lo_v=0):
+def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0, L_hi_v=0, L_lo_v=0, k_per_channel=0):
     import torch
 
     B, H, T, D = K.shape
     Hq = q.shape[1]
     cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T, p, extra=extra, window=window, clip=clip,
-                                   L_hi_v=L_hi_v, L_lo_v=L_lo_v).poison()
+                                   L_hi_v=L_hi_v, L_lo_v=L_lo_v, k_per_channel=k_per_channel).poison()
     dK, dV, dS, dq = to_dev(K), to_dev(V), to_dev(S), to_dev(q)
     semkv_assign_precision(cache, dS, T, p)
     semkv_quantize_pack(cache, dK, dV, T)
@@ -76,17 +77,23 @@ def run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, extra=0, window=0, clip=0.0, L_
     return res
 
 
-def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo, window=0, clip=0.0, L_hi_v=0, L_lo_v=0):
+def oracle_unit(K, V, S, q, p, G, L_hi, L_lo, scale, tiles_hi, tiles_lo, window=0, clip=0.0, L_hi_v=0, L_lo_v=0,
+                k_per_channel=0):
     """Oracle results of one unit. K, V [T][D] fp16; S [T]; q [g][D] fp16.  window, clip, L_hi_v,
-    L_lo_v: the quantizer variants as the cache fields state them (0 = off)."""
+    L_lo_v, k_per_channel: the quantizer variants as the cache fields state them (0 = off)."""
     bm, rk, nh, tau, st = oracle.select(S, p, window=window)
+    kc = oracle.k_channel_grid(K.view(np.uint16), L_hi, L_lo, clip or 1.0)[0] if k_per_channel else None
     hi, lo, st2 = oracle.quantize_pack_unit(K.view(np.uint16), V.view(np.uint16), bm, G, L_hi, L_lo, tiles_hi,
-                                            tiles_lo, clip=clip or 1.0, L_hi_v=L_hi_v or None, L_lo_v=L_lo_v or None)
+                                            tiles_lo, clip=clip or 1.0, L_hi_v=L_hi_v or None, L_lo_v=L_lo_v or None,
+                                            kc=kc)
     T = K.shape[0]
-    Kh, Vh = oracle.dequantize_unit(T, K.shape[1], G, L_hi, L_lo, bm, hi, lo, L_hi_v or None, L_lo_v or None)
+    Kh, Vh = oracle.dequantize_unit(T, K.shape[1], G, L_hi, L_lo, bm, hi, lo, L_hi_v or None, L_lo_v or None, kc=kc)
     o = oracle.attention_fp64(q.view(np.uint16), Kh, Vh, scale)
-    return {"bitmap": bm, "rank": rk, "n_hi": nh, "tau": tau, "hi": hi, "lo": lo, "Kh": Kh, "Vh": Vh, "out": o,
-            "status": st | st2}
+    res = {"bitmap": bm, "rank": rk, "n_hi": nh, "tau": tau, "hi": hi, "lo": lo, "Kh": Kh, "Vh": Vh, "out": o,
+           "status": st | st2}
+    if kc is not None:
+        res["kc"] = kc
+    return res
 
 
 def _words_equal(a, b, what):
@@ -106,6 +113,8 @@ def compare_state(g: dict, o: dict, T: int, L_hi: int, L_lo: int, where: str = "
     assert np.array_equal(g["rank"][:nw], o["rank"][:nw]), f"rank {where}"
     assert g["n_hi"] == o["n_hi"] and g["n_lo"] == T - o["n_hi"], f"counts {where}"
     assert np.float32(g["tau"]).view(np.uint32) == np.float32(o["tau"]).view(np.uint32), f"tau {where}"
+    if o.get("kc") is not None:
+        _words_equal(g["kc"], o["kc"], f"per-channel K grids {where}")
     if strict_tail and "slot_hi" in g:  # after a prefill: the slot map is the inverse of the ranks
         bits = np.unpackbits(o["bitmap"][:nw].view(np.uint8), bitorder="little")[:T].astype(bool)
         tokens = np.arange(T)
@@ -137,11 +146,13 @@ def attention_errors(got, ref):
     return max_abs, rel
 
 
-def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0.0, L_hi_v=0, L_lo_v=0):
+def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0.0, L_hi_v=0, L_lo_v=0,
+               k_per_channel=0):
     """Run the GPU path on a whole case and compare the chosen units (default: all) with the oracle."""
     B, H, T, D = K.shape
     g = q.shape[1] // H
-    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, window=window, clip=clip, L_hi_v=L_hi_v, L_lo_v=L_lo_v)
+    res = run_gpu(K, V, S, q, p, G, L_hi, L_lo, scale, window=window, clip=clip, L_hi_v=L_hi_v, L_lo_v=L_lo_v,
+                  k_per_channel=k_per_channel)
     cache = res["cache"]
     assert res["status"] == 0, f"status {res['status']}"
     units = range(B * H) if units is None else units
@@ -150,7 +161,7 @@ def check_case(K, V, S, q, p, G, L_hi, L_lo, scale, units=None, window=0, clip=0
         b, h = divmod(u, H)
         o = oracle_unit(K[b, h], V[b, h], S[b, h], q[b, h * g:(h + 1) * g], p, G, L_hi, L_lo, scale,
                         cache.cap_hi // 128, cache.cap_lo // 128, window=window, clip=clip, L_hi_v=L_hi_v,
-                        L_lo_v=L_lo_v)
+                        L_lo_v=L_lo_v, k_per_channel=k_per_channel)
         gu = unit_views(cache, res["bufs"], u)
         compare_state(gu, o, T, L_hi, L_lo, where=f"unit {u}", L_hi_v=L_hi_v, L_lo_v=L_lo_v)
         assert np.array_equal(res["Kh"][b, h].view(np.uint32), o["Kh"].view(np.uint32)), f"Khat unit {u}"

@@ -234,3 +234,77 @@ def test_v_levels_appends_in_lockstep(mode, Lhv, Llv):
         ref = oracle.attention_fp64(Q[-1, b, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, sm_scale())
         ma, rl = attention_errors(out.cpu().numpy()[b, h * g:(h + 1) * g], ref)
         assert ma <= ATOL and rl <= RTOL_L2, (ma, rl)
+
+
+# ---------------------------------------------------------------- per-channel K grids
+
+
+@pytest.mark.parametrize("B,H,Hq,T,G,L_hi,L_lo,p,clip,dist", [
+    (1, 2, 8, 600, 64, 8, 5, 0.25, 0.0, "outlier"),   # a few large key channels
+    (2, 1, 4, 333, 32, 6, 5, 0.5, 0.7, "normal"),
+    (1, 1, 8, 1500, 128, 16, 4, 0.1, 0.0, "wide"),
+])
+def test_k_per_channel_full_path(B, H, Hq, T, G, L_hi, L_lo, p, clip, dist):
+    K, V, S, q = _case(B, H, Hq, T, T + 91, dist)
+    check_case(K, V, S, q, p, G, L_hi, L_lo, sm_scale(), clip=clip, k_per_channel=1)
+
+
+@pytest.mark.parametrize("mode", ["append", "append_decode", "running"])
+def test_k_per_channel_appends_in_lockstep(mode):
+    import torch
+
+    import oracle
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, semkv_append_decode, semkv_append_token,
+                                               semkv_append_token_running, semkv_assign_precision,
+                                               semkv_decode_attention, semkv_quantize_pack)
+
+    B, H, Hq, T0, steps, G, L_hi, L_lo, p = 1, 2, 8, 260, 70, 64, 8, 5, 0.3
+    r = np.random.default_rng(79)
+    K = (r.standard_normal((B, H, T0 + steps, 128)) * 1.3).astype(np.float16)  # appends reach past the grid
+    V = r.standard_normal((B, H, T0 + steps, 128)).astype(np.float16)
+    S = r.standard_normal((B, H, T0 + steps)).astype(np.float32)
+    Q = r.standard_normal((steps, B, Hq, 128)).astype(np.float16)
+    cache = SemkvCache.for_prefill(B, H, Hq, G, L_hi, L_lo, T0, p, extra=steps, k_per_channel=1).poison()
+    semkv_assign_precision(cache, to_dev(S[:, :, :T0].copy()), T0, p)
+    semkv_quantize_pack(cache, to_dev(K[:, :, :T0].copy()), to_dev(V[:, :, :T0].copy()), T0)
+    ws = cache.workspace()
+    states = []
+    for u in range(B * H):
+        b, h = divmod(u, H)
+        bm, rk, nh, tau, _ = oracle.select(S[b, h, :T0], p)
+        kc, _ = oracle.k_channel_grid(K[b, h, :T0].view(np.uint16), L_hi, L_lo)
+        hi, lo, _ = oracle.quantize_pack_unit(K[b, h, :T0].view(np.uint16), V[b, h, :T0].view(np.uint16), bm, G,
+                                              L_hi, L_lo, cache.cap_hi // 128, cache.cap_lo // 128, kc=kc)
+        states.append(oracle.UnitState(cache.T_cap, bm, rk, nh, T0 - nh, tau, hi, lo, kc=kc))
+    g = Hq // H
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device="cuda")
+    for s in range(steps):
+        t = T0 + s
+        k, v, sc, q = (to_dev(x) for x in (K[:, :, t].copy(), V[:, :, t].copy(), S[:, :, t].copy(), Q[s]))
+        if mode == "append":
+            semkv_append_token(cache, k, v, sc)
+        elif mode == "append_decode":
+            semkv_append_decode(cache, k, v, sc, q, sm_scale(), out, ws)
+        else:
+            semkv_append_token_running(cache, k, v, sc, p)
+        for u in range(B * H):
+            b, h = divmod(u, H)
+            kk, vv = K[b, h, t].view(np.uint16), V[b, h, t].view(np.uint16)
+            if mode == "running":
+                oracle.append_unit_running(states[u], kk, vv, S[b, h, t], p, S[b, h, :t], G, L_hi, L_lo)
+            else:
+                oracle.append_unit(states[u], kk, vv, S[b, h, t], G, L_hi, L_lo)
+    if mode != "append_decode":
+        semkv_decode_attention(cache, to_dev(Q[-1]), sm_scale(), out, ws)
+    bufs = fetch(cache)
+    assert cache.status() == 0
+    T = T0 + steps
+    for u, st in enumerate(states):
+        compare_state(unit_views(cache, bufs, u), {"bitmap": st.bitmap, "rank": st.rank, "n_hi": st.n_hi,
+                                                   "tau": st.tau, "hi": st.hi, "lo": st.lo, "kc": st.kc},
+                      T, L_hi, L_lo, where=f"unit {u}", strict_tail=False)
+        b, h = divmod(u, H)
+        Kh, Vh = oracle.dequantize_unit(T, 128, G, L_hi, L_lo, st.bitmap, st.hi, st.lo, kc=st.kc)
+        ref = oracle.attention_fp64(Q[-1, b, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, sm_scale())
+        ma, rl = attention_errors(out.cpu().numpy()[b, h * g:(h + 1) * g], ref)
+        assert ma <= ATOL and rl <= RTOL_L2, (ma, rl)
