@@ -132,7 +132,7 @@ static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_
         const SegView sv = seg_view(c, hi != 0);
         const int ns = hi ? nh : nl, off = hi ? 0 : nh;
         if (ns == 0) continue;
-        if (!c->k_per_channel && decode_tc_supported(sv.L, sv.Lv, c->G, g)) {
+        if (decode_tc_supported(sv.L, sv.Lv, c->G, g, c->k_per_channel != 0)) {
             launch_decode_tc(sv, q, units, c->H, g, c->G, scale_log2, ns, off, nh + nl, ws, c->status, dependent, app,
                              st);
         } else {
@@ -280,8 +280,8 @@ int semkv_append_decode(const semkv_cache_t* c, const uint16_t* k, const uint16_
     if (r != SEMKV_OK) return r;
     if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
     const int g = c->Hq / c->H;
-    if (c->k_per_channel || !decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g) ||
-        !decode_tc_supported(c->L_lo, level_v(*c, false), c->G, g)) {
+    if (!decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g, c->k_per_channel != 0) ||
+        !decode_tc_supported(c->L_lo, level_v(*c, false), c->G, g, c->k_per_channel != 0)) {
         // shapes the fused path does not cover: the two calls, in order
         launch_append(*c, k, v, score, -1.0f, (cudaStream_t)stream);
         r = launch_status();

@@ -131,7 +131,9 @@ __device__ __forceinline__ void unpack_to_tmem(uint32_t words, uint32_t lut_lane
     }
 }
 
-template <int LK, int LV, int GQ, int NG, bool APP>
+// KPC: per-channel K grids (seg.kc): B_Q holds q_hd s_d as two fp16 limbs per head (rows h and
+// GQ + h), and the zero terms sum_d q_hd (z_d + m s_d) are one constant per head
+template <int LK, int LV, int GQ, int NG, bool APP, bool KPC>
 __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_t* __restrict__ q, int H,
                                                        float scale_log2, int nsplit, int split_off, int nsplit_total,
                                                        float* __restrict__ ws, int32_t* __restrict__ status,
@@ -243,13 +245,45 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
         const int pos = pair_digit(RK::k, pp, h2);
         const int dim = (col < RK::KC && pos >= 0) ? j * RK::k + pos : D;
         const int dgrp = dim < D ? dim / G : -1;
+        if constexpr (KPC) {
+            static_assert(2 * GQ <= NK, "two limbs per head must fit the q.k columns");
+            const float sd = dim < D ? h2f((uint16_t)(seg.kc[(size_t)u * 256 + dim] & 0xffffu)) : 0.f;
 #pragma unroll
-        for (int nrow = 0; nrow < NK; ++nrow) {
-            const uint16_t v = (nrow < NG * GQ && nrow / GQ == dgrp) ? qs[(nrow % GQ) * D + dim] : (uint16_t)0;
-            *reinterpret_cast<uint16_t*>(bq + core_off(nrow, ks, C::LBO_Q, C::SBO_Q)) = v;
+            for (int nrow = 0; nrow < NK; ++nrow) {
+                uint16_t v = 0;
+                if (nrow < 2 * GQ && dim < D) {
+                    const float x = h2f(qs[(nrow % GQ) * D + dim]) * sd;
+                    const __half hi = __float2half_rn(x);
+                    v = __half_as_ushort(nrow < GQ ? hi : __float2half_rn(x - __half2float(hi)));
+                }
+                *reinterpret_cast<uint16_t*>(bq + core_off(nrow, ks, C::LBO_Q, C::SBO_Q)) = v;
+            }
+        } else {
+#pragma unroll
+            for (int nrow = 0; nrow < NK; ++nrow) {
+                const uint16_t v = (nrow < NG * GQ && nrow / GQ == dgrp) ? qs[(nrow % GQ) * D + dim] : (uint16_t)0;
+                *reinterpret_cast<uint16_t*>(bq + core_off(nrow, ks, C::LBO_Q, C::SBO_Q)) = v;
+            }
         }
     }
-    {
+    if constexpr (KPC) {
+        // zero term of each head: 8 threads per head, 16 channels each
+        const int h = tid >> 3, part = tid & 7;
+        float a = 0.f;
+        if (h < GQ) {
+#pragma unroll 4
+            for (int e = 0; e < 16; ++e) {
+                const int d = part * 16 + e;
+                const uint32_t gk = seg.kc[(size_t)u * 256 + d];
+                const float sd = h2f((uint16_t)(gk & 0xffffu));
+                a += h2f(qs[h * D + d]) * __fmaf_rn(MID_K, sd, h2f((uint16_t)(gk >> 16)));
+            }
+        }
+        a += __shfl_xor_sync(0xffffffffu, a, 4);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        if (h < GQ && part == 0) qsum[h] = a;
+    } else {
         // per-group query sums: 8 threads per (group, head), G/8 channels each
         const int si = tid >> 3, part = tid & 7;
         float a = 0.f;
@@ -340,9 +374,13 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
             float acc = 0.f;
+            if constexpr (KPC) {
+                acc = __uint_as_float(dk[h]) + __uint_as_float(dk[GQ + h]) + qsum[h];
+            } else {
 #pragma unroll
-            for (int gg = 0; gg < NG; ++gg)
-                acc += sk[gg] * __uint_as_float(dk[gg * GQ + h]) + zk[gg] * qsum[gg * GQ + h];
+                for (int gg = 0; gg < NG; ++gg)
+                    acc += sk[gg] * __uint_as_float(dk[gg * GQ + h]) + zk[gg] * qsum[gg * GQ + h];
+            }
             lg[h] = valid ? acc * scale_log2 : NEG_INF;
             const float mx = warp_max_redux(lg[h]);
             if (lane == 0) red[warp * 32 + h] = mx;
@@ -448,7 +486,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     if (wait_for_prior) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <int LK, int LV, int GQ, int NG>
+template <int LK, int LV, int GQ, int NG, bool KPC>
 static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, float scale_log2, int nsplit,
                       int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
                       const AppendIn& app, cudaStream_t st)
@@ -458,7 +496,7 @@ static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, f
     const size_t sm = C::TOTAL > 48u * 1024u ? C::TOTAL : 48u * 1024u;
     // the plain decode and the one that appends first are separate instantiations, so that the
     // plain one carries no append code
-    const auto kern = app.k ? k_decode_tc<LK, LV, GQ, NG, true> : k_decode_tc<LK, LV, GQ, NG, false>;
+    const auto kern = app.k ? k_decode_tc<LK, LV, GQ, NG, true, KPC> : k_decode_tc<LK, LV, GQ, NG, false, KPC>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)nsplit, (unsigned)units);
@@ -475,20 +513,23 @@ static void launch_tc(const SegView& seg, const uint16_t* q, int units, int H, f
 }
 
 // instantiated shapes: K and V level counts (equal: L in {4, 5, 6, 8, 16}; V with its own count:
-// six common pairs) x (g, groups) whose accumulators fit 128 TMEM columns
-#define SEMKV_TC_SHAPES(X, LK, LV) X(LK, LV, 2, 1) X(LK, LV, 2, 2) X(LK, LV, 2, 4) X(LK, LV, 4, 1) X(LK, LV, 4, 2) \
-    X(LK, LV, 4, 4) X(LK, LV, 8, 1) X(LK, LV, 8, 2)
-#define SEMKV_TC_SHAPES_KV(X, LK, LV) X(LK, LV, 2, 2) X(LK, LV, 4, 1) X(LK, LV, 4, 2) X(LK, LV, 8, 1) X(LK, LV, 8, 2)
+// six common pairs) x (g, groups) whose accumulators fit 128 TMEM columns; per-channel K grids for
+// the equal counts on the common shapes
+#define SEMKV_TC_SHAPES(X, LK, LV) X(LK, LV, 2, 1, false) X(LK, LV, 2, 2, false) X(LK, LV, 2, 4, false) \
+    X(LK, LV, 4, 1, false) X(LK, LV, 4, 2, false) X(LK, LV, 4, 4, false) X(LK, LV, 8, 1, false) X(LK, LV, 8, 2, false) \
+    X(LK, LV, 4, 1, true) X(LK, LV, 4, 2, true) X(LK, LV, 8, 1, true) X(LK, LV, 8, 2, true)
+#define SEMKV_TC_SHAPES_KV(X, LK, LV) X(LK, LV, 2, 2, false) X(LK, LV, 4, 1, false) X(LK, LV, 4, 2, false) \
+    X(LK, LV, 8, 1, false) X(LK, LV, 8, 2, false)
 #define SEMKV_TC_LEVELS(X) SEMKV_TC_SHAPES(X, 4, 4) SEMKV_TC_SHAPES(X, 5, 5) SEMKV_TC_SHAPES(X, 6, 6) \
     SEMKV_TC_SHAPES(X, 8, 8) SEMKV_TC_SHAPES(X, 16, 16) SEMKV_TC_SHAPES_KV(X, 8, 4) SEMKV_TC_SHAPES_KV(X, 5, 2) \
     SEMKV_TC_SHAPES_KV(X, 8, 5) SEMKV_TC_SHAPES_KV(X, 6, 4) SEMKV_TC_SHAPES_KV(X, 5, 4) SEMKV_TC_SHAPES_KV(X, 16, 8)
 
-bool decode_tc_supported(int Lk, int Lv, int G, int g)
+bool decode_tc_supported(int Lk, int Lv, int G, int g, bool kpc)
 {
     if (G <= 0 || 128 % G) return false;
     const int ng = 128 / G;
-#define SEMKV_TC_OK(LK, LV, GG, NN) \
-    if (Lk == LK && Lv == LV && g == GG && ng == NN) return Tc<LK, LV, GG, NN>::ok;
+#define SEMKV_TC_OK(LK, LV, GG, NN, KP) \
+    if (Lk == LK && Lv == LV && g == GG && ng == NN && kpc == KP) return Tc<LK, LV, GG, NN>::ok;
     SEMKV_TC_LEVELS(SEMKV_TC_OK)
 #undef SEMKV_TC_OK
     return false;
@@ -500,10 +541,11 @@ void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, i
 {
     if (nsplit == 0 || units == 0) return;
     const int ng = 128 / G;
-#define SEMKV_TC_GO(LK, LV, GG, NN)                                                                                 \
-    if (seg.L == LK && seg.Lv == LV && g == GG && ng == NN) {                                                    \
-        launch_tc<LK, LV, GG, NN>(seg, q, units, H, scale_log2, nsplit, split_off, nsplit_total, ws, status,      \
-                                  dependent, app, st);                                                          \
+    const bool kpc = seg.kc != nullptr;
+#define SEMKV_TC_GO(LK, LV, GG, NN, KP)                                                                             \
+    if (seg.L == LK && seg.Lv == LV && g == GG && ng == NN && kpc == KP) {                                       \
+        launch_tc<LK, LV, GG, NN, KP>(seg, q, units, H, scale_log2, nsplit, split_off, nsplit_total, ws, status,  \
+                                      dependent, app, st);                                                      \
         return;                                                                                                 \
     }
     SEMKV_TC_LEVELS(SEMKV_TC_GO)

@@ -65,8 +65,8 @@ void launch_decode_split(const SegView& seg, const uint16_t* q, int units, int H
 void launch_decode_merge(const float* ws, int units, int H, int g, int D, int nsplit_total, float* out,
                          const AppendIn& app, cudaStream_t st);
 
-// tcgen05 decode (decode_tc.cu): the instantiated (K levels, V levels, g, groups), G >= 32.
-bool decode_tc_supported(int Lk, int Lv, int G, int g);
+// tcgen05 decode (decode_tc.cu): the instantiated (K levels, V levels, g, groups, per-channel K), G >= 32.
+bool decode_tc_supported(int Lk, int Lv, int G, int g, bool kpc);
 // `dependent`: launched as a programmatic dependent of the previous kernel in the stream (it may
 // start while that kernel drains, and waits for it to complete before it exits).
 void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, int g, int G, float scale_log2,
