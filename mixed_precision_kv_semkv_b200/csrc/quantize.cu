@@ -401,6 +401,60 @@ __device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw
     }
 }
 
+// Per-channel K grids of a segment as channel pairs: (z, z'), (r, r'), (-s, -s') in packed fp32 and
+// the zeros as a binary16 pair
+struct KpcPair {
+    uint64_t z2, r2, ns2;
+    uint32_t zh2, pad;
+};
+
+// K rows of a tile on per-channel grids (thread `tid` = slot `tid`; slots at or past `nv` get zero
+// codes): the value is raised to its channel's zero, the quotient clamped to L - 1 before the
+// rounding add, as on the clipped grid
+template <int L>
+__device__ __forceinline__ void quantize_k_rows_kpc(const uint16_t* Ks, uint32_t* kw, uint32_t* kz, int tid, int nv,
+                                                    int NG, const KpcPair* tab, bool& bad)
+{
+    constexpr int D = 128, k = radix_k(L), WK = ceil_div(D, k);
+    const uint64_t m2 = f2_pack(12582912.0f, 12582912.0f);
+    const bool live = tid < nv;
+    uint32_t w[WK];
+#pragma unroll
+    for (int j = 0; j < WK; ++j) w[j] = 0u;
+    const uint16_t* row = Ks + tid * QROW;
+#pragma unroll
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + 8 * c8);
+        const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = 4 * c8 + e;  // channel pair (2i, 2i + 1)
+            const KpcPair p = tab[i];
+            const __half2 x2 = *reinterpret_cast<const __half2*>(&hw[e]);
+            const float2 xr = __half22float2(x2);
+            bad |= !(fabsf(xr.x) <= 65504.0f) || !(fabsf(xr.y) <= 65504.0f);
+            const float2 xf = __half22float2(__hmax2(x2, *reinterpret_cast<const __half2*>(&p.zh2)));
+            uint64_t d, q0, ee, q, y;
+            asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(xf.x, xf.y)), "l"(p.z2));
+            asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(d), "l"(p.r2));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(ee) : "l"(p.ns2), "l"(q0), "l"(d));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(ee), "l"(p.r2), "l"(q0));
+            const float qa = fminf(__uint_as_float((uint32_t)q), (float)(L - 1));
+            const float qb = fminf(__uint_as_float((uint32_t)(q >> 32)), (float)(L - 1));
+            asm("add.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(f2_pack(qa, qb)), "l"(m2));
+            const uint32_t b0 = live ? (uint32_t)y : 0x4B400000u, b1 = live ? (uint32_t)(y >> 32) : 0x4B400000u;
+            w[(2 * i) / k] += b0 * upow(L, (2 * i) % k);
+            w[(2 * i + 1) / k] += b1 * upow(L, (2 * i + 1) % k);
+        }
+    }
+    for (int grp = 0; grp < NG; ++grp) kz[grp * TILE + tid] = 0u;  // no per-token K grid
+#pragma unroll
+    for (int j = 0; j < WK; ++j) {
+        const int cnt = (j + 1) * k <= D ? k : D - j * k;
+        kw[j * TILE + tid] = w[j] - magic_sum(L, cnt);
+    }
+}
+
 // V rows of a tile: thread `tid` writes the grids of row tid and its codes as bytes over the first
 // half of its own row; after a barrier thread `tid` packs channel tid along the tile's slots
 template <int L, int G, bool CLIP>
@@ -455,8 +509,8 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
 }
 
 // LH, LL: level counts of the K codes of the two segments; LHV, LLV: of the V codes; CLIP: the
-// clipped-range grid with ratio `clip`
-template <int LH, int LL, int LHV, int LLV, int G, bool CLIP>
+// clipped-range grid with ratio `clip`; KPC: K on the per-channel grids of seg.kc
+template <int LH, int LL, int LHV, int LLV, int G, bool CLIP, bool KPC = false>
 __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
                                                         const uint16_t* __restrict__ V,
                                                         int T, float clip,
@@ -492,8 +546,30 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
         const int Wk = is_hi ? ceil_div(D, radix_k(LH)) : ceil_div(D, radix_k(LL));
         uint32_t* kw = seg.k + tile_base * Wk * TILE;
         uint32_t* kz = seg.kz + tile_base * NG * TILE;
-        if (is_hi) quantize_k_rows<LH, G, CLIP>(Xs, kw, kz, tid, bad, clip);
-        else quantize_k_rows<LL, G, CLIP>(Xs, kw, kz, tid, bad, clip);
+        if constexpr (KPC) {
+            KpcPair* tab = reinterpret_cast<KpcPair*>(smem + (size_t)TILE * QROW * 2);  // [64]
+            if (tid < 64) {
+                float z[2], r[2], sv[2];
+                uint16_t zh[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t gk = seg.kc[(size_t)u * 256 + 2 * tid + e];
+                    sv[e] = h2f((uint16_t)(gk & 0xffffu));
+                    zh[e] = (uint16_t)(gk >> 16);
+                    z[e] = h2f(zh[e]);
+                    r[e] = sv[e] != 0.0f ? __frcp_rn(sv[e]) : 0.0f;
+                }
+                tab[tid] = KpcPair{f2_pack(z[0], z[1]), f2_pack(r[0], r[1]), f2_pack(-sv[0], -sv[1]),
+                                   (uint32_t)zh[0] | ((uint32_t)zh[1] << 16), 0u};
+            }
+            __syncthreads();  // uniform: every thread of a K-part CTA
+            const int nv = min(TILE, n - s0);
+            if (is_hi) quantize_k_rows_kpc<LH>(Xs, kw, kz, tid, nv, NG, tab, bad);
+            else quantize_k_rows_kpc<LL>(Xs, kw, kz, tid, nv, NG, tab, bad);
+        } else {
+            if (is_hi) quantize_k_rows<LH, G, CLIP>(Xs, kw, kz, tid, bad, clip);
+            else quantize_k_rows<LL, G, CLIP>(Xs, kw, kz, tid, bad, clip);
+        }
     } else {
         const int Wv = is_hi ? ceil_div(TILE, radix_k(LHV)) : ceil_div(TILE, radix_k(LLV));
         uint32_t* vw = seg.v + tile_base * Wv * D;
@@ -541,6 +617,16 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
     // compile-time level counts and group sizes of the common configurations; the quantizer
     // variants (a clip, V level counts of their own) for a few of them, the rest on k_quantize
     const bool clipped = clip != 1.0f;
+#define SEMKV_QK(LH, LL, GG)                                                                                  \
+    if (kc && !clipped && shi.L == LH && slo.L == LL && shi.Lv == LH && slo.Lv == LL && G == GG) {            \
+        const size_t sm = (size_t)TILE * QROW * 2 + 64 * sizeof(KpcPair);                                     \
+        const auto kern = k_quantize_fast<LH, LL, LH, LL, GG, false, true>;                                   \
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);                    \
+        kern<<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, clip, status);                                       \
+        return;                                                                                               \
+    }
+    SEMKV_QK(8, 5, 64) SEMKV_QK(6, 5, 64) SEMKV_QK(8, 6, 64) SEMKV_QK(16, 8, 64) SEMKV_QK(5, 4, 64)
+#undef SEMKV_QK
     if (!kc) {
 #define SEMKV_QF(LH, LL, LHV, LLV, GG, CL)                                                                    \
     if (clipped == CL && shi.L == LH && slo.L == LL && shi.Lv == LHV && slo.Lv == LLV && G == GG) {           \
