@@ -59,13 +59,15 @@ def test_cache_bytes_match_oracle_layout(semkv, orc, L_hi, L_lo, G):
     assert sizes["status"] == 4
     assert sizes["slot_token"] == units * (256 + 768) * 4
     assert sizes["score_keys"] == units * 1024 * 4
+    assert sizes["kc"] == units * 2 * 128 * 4  # per-channel K grids: hi and lo per channel
 
 
 @pytest.mark.parametrize("bad,code", [
     (dict(Hq=30), 1), (dict(G=48), 1), (dict(cap_hi=100), 1), (dict(T_cap=1000), 1), (dict(B=0), 1),
     (dict(D=64, G=64), 2), (dict(L_hi=257), 2), (dict(L_lo=1), 2), (dict(G=4), 2), (dict(Hq=8 * 16), 2),
     (dict(window=-1), 1), (dict(clip=1.5), 1), (dict(clip=-0.25), 1), (dict(clip=float("nan")), 1),
-    (dict(L_hi_v=1), 2), (dict(L_lo_v=257), 2), (dict(L_hi_v=-3), 2),
+    (dict(L_hi_v=1), 2), (dict(L_lo_v=257), 2), (dict(L_hi_v=-3), 2), (dict(k_per_channel=2), 1),
+    (dict(k_per_channel=-1), 1),
 ])
 def test_bad_shapes_are_rejected(semkv, bad, code):
     with pytest.raises(semkv.SemkvError) as e:
