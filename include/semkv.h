@@ -111,8 +111,8 @@ typedef struct semkv_cache {
      *           semkv_quantize_pack over all T prefill tokens (min and max of the channel, the clip
      *           applied), once on the L_hi and once on the L_lo levels, and kept in the `kc` buffer;
      *           every K code of the unit, appended tokens included, is coded on its channel's grid
-     *           of its segment, clamped to [0, L-1]; the per-token K scale/zero are 0.  Decoded on
-     *           the CUDA-core decode. */
+     *           of its segment, clamped to [0, L-1]; the per-token K scale/zero are 0.  The decode
+     *           folds each channel's scale into the query. */
     int32_t window;
     float clip;
     int32_t L_hi_v, L_lo_v;

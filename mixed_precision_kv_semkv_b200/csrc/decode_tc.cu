@@ -18,12 +18,15 @@
 //   q.k      D_K[slot][(group,head)] = sum over the group's channels of (c - m) q_head: a chain of
 //            tcgen05.mma (M=128 slots, N = groups x heads, K = code slots), A (codes) in TMEM and
 //            B (the fp16 queries, zero outside each group) in shared memory.
+//   (per-channel K grids: B holds q_hd s_d as two fp16 limbs instead, and the zero terms are one
+//   constant per head: logit = scale * (D_K[hi limb] + D_K[lo limb] + sum_d q_hd (z_d + m s_d)))
 //   softmax  logit = scale * sum_group [ s_K D_K + (z_K + m s_K) sum_{group} q ]; online softmax
 //            in the log2 domain across tiles (warp shuffles + one shared exchange per tile).
 //   p.V      D_V[channel][(group,limb,head)] = sum_slots (c - m) P', P' = p s_V split into two
 //            fp16 limbs (P' = hi + lo, ~22 bits kept); A = V codes in the same TMEM columns (the
 //            q.k product has completed), B = P' in shared memory written by the slot threads.
 //            The zero terms sum_t p (z_V + m s_V) and the denominators stay on the CUDA cores.
+// K and V may use different level counts (a radix configuration per tensor, TcRadix).
 // Each CTA writes (max, sum, unnormalized o) per query head to the workspace; k_decode_merge
 // combines the splits.  Every mbarrier wait is bounded; a timeout sets SEMKV_STATUS_TIMEOUT.
 #include "append.cuh"
