@@ -66,7 +66,7 @@ WINDOW, CLIP, V_LEVELS = 128, 0.9, (4, 2)
 
 
 def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False, v_levels=None) -> dict:
-    """Algorithmic bytes of one layer, per hot-path step (measurement).  With
+    """Algorithmic bytes of one layer, per hot-path step (what the method must move).  With
     `appended`, one generated token per unit follows the prefill (`new_hi` of them on the L_hi grid)
     and the decode reads the cache including it.  v_levels: the V level counts of the two segments,
     when they differ from the K ones."""

@@ -15,7 +15,7 @@
  * sit above the quality cliff, the rest the lower one; each precision is a uniform affine grid
  * whose level count need not be a power of two (5 levels = 2.322 code bits per value, 4 levels =
  * 2.0 bits).  The Abstract fixes neither the quantizer's rounding, the packing, nor the tie rule;
- * every such choice below is a reading, marked [reading], and the same list is kept in the design doc.
+ * every such choice below is a reading, marked [reading].
  *
  *   select      order the tokens of one (batch, kv-head) unit by score; the n_hi = floor(p*T) with
  *               the largest scores get L_hi levels, the rest L_lo.  [reading: floor; equal scores
