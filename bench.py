@@ -552,6 +552,7 @@ def run_semkv(args):
             e1.synchronize()
             if i >= 2:
                 el += e0.elapsed_time(e1)
+        el = max_over_ranks(el, dist, "cuda")  # every rank gets here (same flags): the slowest rank's time
         h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hS, hq, hk, hv, hs))
         e2e = {"value": world * step_bytes * e2e_steps / (el * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * 4,
