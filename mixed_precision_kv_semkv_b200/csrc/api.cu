@@ -234,11 +234,11 @@ int semkv_quantize_pack(const semkv_cache_t* c, const uint16_t* K, const uint16_
     if (r != SEMKV_OK) return r;
     if (T < 0 || T > c->T_cap || ((!K || !V) && T > 0)) return SEMKV_ERR_INVALID_ARG;
     if (T == 0) {  // nothing to place; per-channel K grids of an empty prefill are zero
-        if (c->k_per_channel) launch_kc_grids(*c, K, 0, (cudaStream_t)stream);
+        if (c->k_per_channel) launch_kc_grids(*c, K, 0, sm_count(), (cudaStream_t)stream);
         return launch_status();
     }
     if ((((uintptr_t)K) | ((uintptr_t)V)) & 15u) return SEMKV_ERR_INVALID_ARG;  // rows are fetched by bulk copies
-    if (c->k_per_channel) launch_kc_grids(*c, K, T, (cudaStream_t)stream);  // grids first: the codes use them
+    if (c->k_per_channel) launch_kc_grids(*c, K, T, sm_count(), (cudaStream_t)stream);  // grids first: the codes use them
     launch_quantize(seg_view(c, true), seg_view(c, false), K, V, c->slot_token, c->B * c->H, T, c->D, c->G,
                     clip_ratio(*c), c->k_per_channel ? c->kc : nullptr, c->status, (cudaStream_t)stream);
     return launch_status();

@@ -94,13 +94,13 @@ __global__ void k_kc_finalize(uint32_t* __restrict__ kc, int units, int L_hi, in
     p[D] = glo;
 }
 
-void launch_kc_grids(const semkv_cache_t& c, const uint16_t* K, int T, cudaStream_t st)
+void launch_kc_grids(const semkv_cache_t& c, const uint16_t* K, int T, int sms, cudaStream_t st)
 {
     const int units = c.B * c.H, n = units * 2 * 128;
     k_kc_init<<<(n + 255) / 256, 256, 0, st>>>(c.kc, n);
     if (T > 0) {
         // about four CTAs per SM over all units, at least 32 tokens per slice
-        int slices = (4 * 148 + units - 1) / units;
+        int slices = (4 * sms + units - 1) / units;
         slices = min(slices, (T + 31) / 32);
         slices = max(slices, 1);
         k_kc_range<<<dim3((unsigned)slices, (unsigned)units), KC_THREADS, 0, st>>>(K, T, slices, c.kc, c.status);

@@ -51,7 +51,7 @@ void launch_quantize(const SegView& hi, const SegView& lo, const uint16_t* K, co
                      int32_t* status, cudaStream_t st);
 
 // per-channel K grids of every unit from the prefill's K (kchannel.cu)
-void launch_kc_grids(const semkv_cache_t& c, const uint16_t* K, int T, cudaStream_t st);
+void launch_kc_grids(const semkv_cache_t& c, const uint16_t* K, int T, int sms, cudaStream_t st);
 
 // p < 0: the fixed threshold rule (score > tau); p in [0, 1]: the running top-p rule
 void launch_append(const semkv_cache_t& c, const uint16_t* k, const uint16_t* v, const float* score, float p,
