@@ -31,7 +31,8 @@
  *                                          WK = ceil(D/k); channels past D are zero digits)
  *   v_seg   [B*H][cap_seg/128][WV][D]     V codes of one channel, packed along the slots of a
  *                                          tile: word w of channel d holds slots w*k .. w*k+k-1,
- *                                          value sum_i code_i * L^i  (WV = ceil(128/k))
+ *                                          value sum_i code_i * L^i  (WV = ceil(128/k); with V
+ *                                          level counts of their own, L and k are the V ones)
  *   kz_seg, vz_seg [B*H][cap_seg/128][D/G][128]   per (slot, channel group): fp16 scale in the
  *                                          low half, fp16 zero in the high half
  *   bitmap  [B*H][T_cap/32]  bit t%32 of word t/32 = 1 iff token t is on the L_hi grid
@@ -50,6 +51,9 @@
  *   score_keys [B*H][T_cap] uint32   every token's score as an order-preserving key (-0 as +0;
  *                            key order = score order), written by semkv_assign_precision and by
  *                            every append; semkv_append_token_running ranks a new token by it
+ *   kc      [B*H][2][D] uint32   per-channel K grids of the L_hi and L_lo segments (fp16 scale |
+ *                            fp16 zero << 16), written by semkv_quantize_pack when k_per_channel
+ *                            is set (then the per-token K scale/zero in kz_seg are 0)
  * Code c of value x on a group with scale s and zero z dequantizes to fmaf((float)c, s, z).
  */
 #ifndef SEMKV_H
