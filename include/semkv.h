@@ -204,8 +204,10 @@ SEMKV_API int semkv_decode_attention(const semkv_cache_t* cache, const uint16_t*
  * cache (SemKV page, Abstract: generation-time quantization): the decode CTA whose tiles hold the new
  * token's slot quantizes and writes the token before it reads that tile, and the merge then updates
  * the unit's counts, bitmap, rank and score key.  Results (cache state, out, status) are those of
- * the two calls in order.  Shapes the tensor-core decode does not cover run the two calls.  k, v:
- * device fp16 [B][H][D]; score: device fp32 [B][H]; the rest as semkv_decode_attention. */
+ * the two calls in order.  Shapes the tensor-core decode does not cover run the two calls.  Every
+ * argument (the decode's too) is checked first: an error returns before anything is enqueued, so
+ * a failed call leaves the cache as it was.  k, v: device fp16 [B][H][D]; score: device fp32
+ * [B][H]; the rest as semkv_decode_attention. */
 SEMKV_API int semkv_append_decode(const semkv_cache_t* cache, const uint16_t* k, const uint16_t* v, const float* score,
                                   const uint16_t* q, float softmax_scale, float* out, void* workspace,
                                   size_t workspace_bytes, void* stream);

@@ -111,9 +111,9 @@ int launch_status()
 
 namespace {
 
-// decode, with an appended token first when app.k is set (both segments on the tensor-core kernel)
-static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_scale, float* out, void* workspace,
-                       size_t workspace_bytes, const AppendIn& app, cudaStream_t st)
+// host checks of a decode call, before anything is launched
+static int decode_args(const semkv_cache_t* c, const uint16_t* q, float softmax_scale, const float* out,
+                       const void* workspace, size_t workspace_bytes)
 {
     int r = validate(c);
     if (r != SEMKV_OK) return r;
@@ -122,6 +122,15 @@ static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_
     size_t need = 0;
     semkv_workspace_bytes(c, &need);
     if (workspace_bytes < need || (need > 0 && !workspace)) return SEMKV_ERR_INVALID_ARG;
+    return SEMKV_OK;
+}
+
+// decode, with an appended token first when app.k is set (both segments on the tensor-core kernel)
+static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_scale, float* out, void* workspace,
+                       size_t workspace_bytes, const AppendIn& app, cudaStream_t st)
+{
+    const int r = decode_args(c, q, softmax_scale, out, workspace, workspace_bytes);
+    if (r != SEMKV_OK) return r;
     int nh, nl;
     decode_splits(c, &nh, &nl);
     const int units = c->B * c->H, g = c->Hq / c->H;
@@ -276,7 +285,8 @@ int semkv_append_decode(const semkv_cache_t* c, const uint16_t* k, const uint16_
                         const uint16_t* q, float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                         void* stream)
 {
-    int r = validate(c);
+    // every argument is checked before anything is launched, on both paths below
+    int r = decode_args(c, q, softmax_scale, out, workspace, workspace_bytes);
     if (r != SEMKV_OK) return r;
     if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
     const int g = c->Hq / c->H;

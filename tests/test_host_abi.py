@@ -107,6 +107,15 @@ def test_calls_fail_before_any_launch(semkv):
     assert L.semkv_decode_attention(ref, one, ctypes.c_float(float("inf")), one, one, 1 << 30, nul) == 1
     assert L.semkv_decode_attention(ref, one, ctypes.c_float(0.1), one, one, 0, nul) == 1  # workspace too small
     assert L.semkv_dequantize(ref, one, nul, 10, nul) == 1
+    # append_decode checks the decode's arguments before it appends (on every path)
+    sc = ctypes.c_float(0.1)
+    assert L.semkv_append_decode(ref, one, one, one, nul, sc, one, one, 1 << 30, nul) == 1   # null q
+    assert L.semkv_append_decode(ref, one, one, one, one, sc, one, one, 0, nul) == 1         # workspace too small
+    assert L.semkv_append_decode(ref, one, one, one, ctypes.c_void_p(0x1008), sc, one, one, 1 << 30, nul) == 1  # q
+    assert L.semkv_append_decode(ref, nul, one, one, one, sc, one, one, 1 << 30, nul) == 1   # null k
+    s.L_hi_v = 3  # a shape on the two-call path: the same checks come first
+    assert L.semkv_append_decode(ref, one, one, one, nul, sc, one, one, 1 << 30, nul) == 1
+    s.L_hi_v = 0
     assert semkv.status_string(3) == "SEMKV_ERR_CAPACITY"
 
 
