@@ -38,3 +38,24 @@ def test_v_level_bytes_by_hand():
     w = synth.WORKLOADS["llama8b_1L"]
     nb = bench.alg_bytes(w, 32768, 8192, v_levels=(4, 2))
     assert nb["cache"] == 8 * (8192 * 100 + 24576 * 72)
+
+
+def test_reference_arm_prints_its_contract_line():
+    """`bench.py --impl reference` (the oracle on the host, a bounded sample) prints one JSON line
+    with the keys of the contract and the same config as the GPU arm's."""
+    import json
+    import subprocess
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["config"]["workload"] == bench.workload_config(synth.WORKLOADS["llama8b_1L"], 1)["workload"]
