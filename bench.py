@@ -1,22 +1,37 @@
 #!/usr/bin/env python
 """Benchmark of the SemKV mixed-precision KV-cache hot path on B200.
 
-One step = one pass of the whole hot path over one layer of synthetic input: precision
-assignment (semkv_assign_precision), affine quantization + radix packing of the prefill
-(semkv_quantize_pack) and one GQA decode step over the packed cache (semkv_decode_attention).
-Default workload: one Llama-3.1-8B-shaped layer, batch 1, 32768 cached tokens, 8 KV heads,
-32 query heads, head_dim 128, group 64, L_hi 8 / L_lo 5, p 0.25.
+Default workload (the headline line): generation-time quantization on a Llama-3.1-8B-shaped
+model, batch 16, 32 layers, 8 KV heads, 32 query heads, head_dim 128, a 32768-token prefill per
+sequence, group 64, L_hi 8 / L_lo 5, p 0.25.  One step = one generated token per sequence in every
+layer: semkv_append_decode per layer (the token is quantized at the precision its score earns
+against the unit's threshold and appended, then GQA decode attention reads the packed cache,
+appended token included), the 32 calls captured as one CUDA graph.  The prefill that builds the
+cache (semkv_assign_precision + semkv_quantize_pack of every layer) is timed in the same run.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl semkv|reference]
+Also reported in the same run (keys of the JSON line):
+  per_kernel.prefill_*  selection and quantize/pack GB/s of the 32-layer prefill
+  per_kernel.decode_32L the 32 decode_attention calls alone, over the cache the timed steps left
+  extras.llama8b_32L    decode attention of all 32 layers per step over a 131072-token cache
+                        (B1, G128, L 6/5, p 0.5), the 32 calls as one CUDA graph
+  extras.llama8b_1L     one layer (B1, T32768, G64, L 8/5, p 0.25): select + quantize + append_decode
+                        as one graph, the per-call split and the quantizer variants
+  sweep                 the Mistral-7B-shaped cache (B8, T32768, Student-t values, Zipf(1.0) scores)
+                        at 45 points (level pair x p x G): storage ratio against fp16 from the
+                        cache's buffer sizes, and decode GB/s
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl semkv|reference] [--workload NAME]
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own data (independent
 units, no collective on the data path: weak scaling); the time is the max over ranks.
-Throughput unit: GB/s of algorithmic bytes (the bytes the method must move: fp16 K/V read once,
-packed codes + fp16 scale/zero written and read once, scores, queries, bitmap/rank).
+Throughput unit: GB/s of algorithmic bytes (what the method must move: fp16 K/V read once by the
+prefill, packed codes + fp16 scale/zero written once and read once per decode, scores, queries,
+bitmap/rank).
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import json
 import math
 import os
@@ -30,19 +45,22 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn HBM GB/s & %roofline over packed mixed-precision KV; quantize GB/s"
 L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2
+HEADLINES = ("gen", "llama8b_32L", "llama8b_1L")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["semkv", "reference"], default="semkv")
-    ap.add_argument("--workload", default="llama8b_1L")
+    ap.add_argument("--workload", choices=HEADLINES, default="gen")
+    ap.add_argument("--layers", type=int, default=0, help="layers of the multi-layer workloads (0: all)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", action="store_true", help="few steps, no clocks/e2e/cpu legs (for ncu)")
-    return ap.parse_args()
+    ap.add_argument("--no-extras", action="store_true", help="only the headline workload")
+    ap.add_argument("--profile", action="store_true", help="few steps, no clocks/e2e/cpu/extras (for ncu)")
+    return ap.parse_args(argv)
 
 
 # ---------------------------------------------------------------- algorithmic bytes
@@ -57,12 +75,19 @@ def radix_words(L: int, n: int = 128) -> int:
     return -(-n // k)
 
 
-# this library's kernel launches in one step: select 1, quantize 1, append+decode 3 (the hi and lo
-# segments, then the merge); the committed ncu launch list of the step shows the same kernels
-LAUNCHES_PER_STEP = 5
-# the quantizer variants timed beside the step (recent window of the selection; clipped range; V
-# level counts of their own for the hi and lo segments)
+def record_bytes(w, L: int, Lv: int | None = None) -> int:
+    """K + V record of one token in a segment: the K words of its row, its share of the V column
+    words, and the fp16 scale/zero pair per group of each."""
+    Lv = Lv or L
+    return 4 * radix_words(L, w.D) + 4 * radix_words(Lv) * w.D // 128 + 2 * 4 * (w.D // w.G)
+
+
+# the quantizer variants timed beside the one-layer step (recent window of the selection; clipped
+# range; V level counts of their own for the hi and lo segments)
 WINDOW, CLIP, V_LEVELS = 128, 0.9, (4, 2)
+# kernels one decode call launches when both segments hold tiles: the hi and lo decode grids, then
+# the merge (the committed ncu launch lists show the same kernels)
+DECODE_KERNELS_PER_CALL = 3
 
 
 def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False, v_levels=None) -> dict:
@@ -71,14 +96,12 @@ def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False, v_l
     and the decode reads the cache including it.  v_levels: the V level counts of the two segments,
     when they differ from the K ones."""
     units = w.B * w.H
-    ng = w.D // w.G
     lv_hi, lv_lo = v_levels or (w.L_hi, w.L_lo)
-    # K + V record of one token: K words of its row, its share of the V column words, scale/zero
-    rec = lambda L, Lv: 4 * radix_words(L, w.D) + 4 * radix_words(Lv) * w.D // 128 + 2 * 4 * ng  # noqa: E731
-    cache = units * (n_hi * rec(w.L_hi, lv_hi) + (T - n_hi) * rec(w.L_lo, lv_lo))
+    rec_hi, rec_lo = record_bytes(w, w.L_hi, lv_hi), record_bytes(w, w.L_lo, lv_lo)
+    cache = units * (n_hi * rec_hi + (T - n_hi) * rec_lo)
     bitmap_rank = units * 2 * 4 * ((T + 31) // 32)
     q = w.B * w.Hq * w.D * 2
-    new = new_hi * rec(w.L_hi, lv_hi) + (units - new_hi) * rec(w.L_lo, lv_lo) if appended else 0
+    new = new_hi * rec_hi + (units - new_hi) * rec_lo if appended else 0
     return {
         "select": units * 4 * T + bitmap_rank,
         "quantize": units * T * w.D * 2 * 2 + bitmap_rank + cache,
@@ -89,6 +112,45 @@ def alg_bytes(w, T: int, n_hi: int, new_hi: int = 0, appended: bool = False, v_l
         "decode": cache + new + q,
         "cache": cache,
     }
+
+
+def gen_steps_bytes(w, nh0, nl0, nh1, nl1, steps: int) -> dict:
+    """Algorithmic bytes of `steps` generation steps over all layers, from each layer's segment
+    counts summed over its units before (nh0, nl0) and after (nh1, nl1) them.  Per step and layer:
+    every unit's new k, v rows and score read and its record written (append), then the records of
+    every cached token, the new one included, and the fp16 queries read (decode).  The split of the
+    new tokens between the grids is taken evenly over the steps (exact in total)."""
+    units = w.B * w.H
+    rec_hi, rec_lo = record_bytes(w, w.L_hi), record_bytes(w, w.L_lo)
+    q = w.B * w.Hq * w.D * 2
+    dec = app = 0.0
+    for a, b, c, d in zip(nh0, nl0, nh1, nl1):
+        dh, dl = c - a, d - b
+        assert dh + dl == units * steps, "every unit appends one token per step"
+        # step j (1..steps) attends over a + j dh/steps hi and b + j dl/steps lo tokens
+        dec += rec_hi * (steps * a + dh * (steps + 1) / 2) + rec_lo * (steps * b + dl * (steps + 1) / 2)
+        dec += steps * q
+        app += steps * units * (w.D * 2 * 2 + 4) + dh * rec_hi + dl * rec_lo
+    return {"decode": dec, "append": app, "total": dec + app}
+
+
+def decode_bytes_now(w, nh, nl) -> float:
+    """Bytes one decode of every layer reads, from the layers' summed segment counts."""
+    q = w.B * w.Hq * w.D * 2
+    return sum(a * record_bytes(w, w.L_hi) + b * record_bytes(w, w.L_lo) + q for a, b in zip(nh, nl))
+
+
+def storage_ratio(D: int, G: int, L_hi: int, L_lo: int, p: float, T: int, B: int = 1, H: int = 1) -> float:
+    """Storage reduction against fp16 of one layer's cache (K and V at 2 bytes per value), from the
+    buffer sizes the library reports for it (semkv_cache_bytes: code words, scale/zero pairs and the
+    precision bitmap; a pure host call)."""
+    from mixed_precision_kv_semkv_b200 import _lib
+
+    _, ch, cl, tc = _lib.semkv_capacities(T, p)
+    s = _lib.CacheStruct(B=B, H=H, Hq=H, D=D, G=G, L_hi=L_hi, L_lo=L_lo, cap_hi=ch, cap_lo=cl, T_cap=tc)
+    sizes = dict(zip(_lib.BUF_NAMES, _lib.semkv_cache_bytes(s)))
+    packed = sum(sizes[n] for n in ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo", "bitmap"))
+    return B * H * T * D * 2 * 2 / packed
 
 
 # ---------------------------------------------------------------- ranks (one process per GPU)
@@ -162,53 +224,115 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ---------------------------------------------------------------- CPU oracle timing
+# ---------------------------------------------------------------- the oracle on the host cores
 
 
-_SAMPLE_INPUTS = {}
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
 
 
-def oracle_sample(w, seconds_target: float = 15.0, max_units: int = 8):
-    """Time the oracle on a bounded sample of the workload: whole units (one (b, kv-head) of one
-    layer each: select + quantize/pack + fp64 attention), as many as fit the time target.
-    Input generation is not timed."""
-    import numpy as np
+class OracleGen:
+    """Units of the generation workload on the host, run by the oracle as it stands.
 
-    import oracle
-    from mixed_precision_kv_semkv_b200 import synth
+    The units' prefill (selection + quantize/pack, one layer) is built first; each `step` then runs
+    one generation step of every unit -- the oracle's append of the unit's next generated token,
+    its dequantization of the whole cache and its attention of the g query heads -- with the units
+    spread over a pool of threads, one per host core (the oracle's C routines run without the
+    interpreter lock).  Inputs come from the seeded generator; nothing here is timed but `step`
+    and `prefill_seconds`."""
 
-    if w.name not in _SAMPLE_INPUTS:
-        d0 = synth.layer_cpu(w, 0, B=1)
-        gen = synth.gen_steps_cpu(w, d0["K"], 0, 0, 1)
-        d0.update(kn=gen["k"][0], vn=gen["v"][0], sn=gen["scores"][0])
-        _SAMPLE_INPUTS[w.name] = d0
-    d = _SAMPLE_INPUTS[w.name]
-    g = w.Hq // w.H
-    T = w.T
-    n_hi = oracle.n_hi(w.p, T)
-    tiles_hi, tiles_lo = -(-(n_hi + 1) // 128), -(-(T - n_hi + 1) // 128)
-    done, new_hi, t0 = 0, 0, time.perf_counter()
-    while done < min(max_units, w.H):
-        h = done
-        bm, rk, nh, tau, _ = oracle.select(d["scores"][0, h], w.p)
-        hi, lo, _ = oracle.quantize_pack_unit(d["K"][0, h].view(np.uint16), d["V"][0, h].view(np.uint16), bm, w.G,
-                                              w.L_hi, w.L_lo, tiles_hi, tiles_lo)
-        st = oracle.UnitState(T + 1, bm, rk, nh, T - nh, tau, hi, lo)
-        oracle.append_unit(st, d["kn"][0, h].view(np.uint16), d["vn"][0, h].view(np.uint16), float(d["sn"][0, h]),
-                           w.G, w.L_hi, w.L_lo)
-        new_hi += st.n_hi - nh
-        Kh, Vh = oracle.dequantize_unit(T + 1, w.D, w.G, w.L_hi, w.L_lo, st.bitmap, hi, lo)
-        oracle.attention_fp64(d["q"][0, h * g:(h + 1) * g].view(np.uint16), Kh, Vh, synth.sm_scale())
-        done += 1
-        if time.perf_counter() - t0 > seconds_target:
-            break
-    el = time.perf_counter() - t0
-    units_layer = w.B * w.H
-    per = alg_bytes(w, T, n_hi, new_hi * units_layer // max(done, 1), appended=True)
-    step_bytes = (per["select"] + per["quantize"] + per["append"] + per["decode"]) / units_layer * done
-    return {"seconds": el, "units": done, "bytes": step_bytes, "gbs": step_bytes / el / 1e9,
-            "sample": f"{done} unit(s) (one batch row x kv head each, T={T} + 1 appended) of workload {w.name}: "
-                      f"select + quantize/pack + append + dequantize + fp64 attention, oracle as it stands, 1 thread"}
+    def __init__(self, w, n_units: int, steps: int, threads: int, T: int | None = None):
+        import numpy as np
+
+        import oracle
+        from mixed_precision_kv_semkv_b200 import synth
+
+        self.np, self.oracle, self.synth, self.w = np, oracle, synth, w
+        self.T = w.T if T is None else T
+        B = max(1, -(-n_units // w.H))
+        self.units = [(b, h) for b in range(B) for h in range(w.H)][:n_units]
+        self.threads = threads
+        self.pool = concurrent.futures.ThreadPoolExecutor(max_workers=threads)
+        d = synth.layer_cpu(w, 0, B=B, T=self.T)
+        gen = synth.gen_steps_cpu(w, d["K"], 0, 0, steps)
+        self.d, self.gen = d, gen
+        self.g = w.Hq // w.H
+        n_hi = oracle.n_hi(w.p, self.T)
+        self.tiles = (-(-(n_hi + steps) // 128), -(-(self.T - n_hi + steps) // 128))
+        self.T_cap = -(-(self.T + steps) // 32) * 32
+        t0 = time.perf_counter()
+        self.states = list(self.pool.map(self._prefill, self.units))
+        self.prefill_seconds = time.perf_counter() - t0
+        rec_hi, rec_lo = record_bytes(w, w.L_hi), record_bytes(w, w.L_lo)
+        n = len(self.units)
+        # bytes of the timed prefill: scores and fp16 K/V read, records and bitmap/rank written
+        self.prefill_bytes = n * (4 * self.T + self.T * w.D * 2 * 2 + n_hi * rec_hi + (self.T - n_hi) * rec_lo
+                                  + 2 * 2 * 4 * ((self.T + 31) // 32))
+        self.step_i = 0
+
+    def _prefill(self, bh):
+        b, h = bh
+        o, w = self.oracle, self.w
+        bm, rk, nh, tau, _ = o.select(self.d["scores"][b, h], w.p)
+        hi, lo, _ = o.quantize_pack_unit(self.d["K"][b, h].view(self.np.uint16), self.d["V"][b, h].view(self.np.uint16),
+                                         bm, w.G, w.L_hi, w.L_lo, *self.tiles)
+        return o.UnitState(self.T_cap, bm, rk, nh, self.T - nh, tau, hi, lo)
+
+    def _unit_step(self, args):
+        (b, h), st, i, fp64 = args
+        o, w, np = self.oracle, self.w, self.np
+        nh_before = st.n_hi
+        o.append_unit(st, self.gen["k"][i, b, h].view(np.uint16), self.gen["v"][i, b, h].view(np.uint16),
+                      float(self.gen["scores"][i, b, h]), w.G, w.L_hi, w.L_lo)
+        T = st.n_hi + st.n_lo
+        Kh, Vh = o.dequantize_unit(T, w.D, w.G, w.L_hi, w.L_lo, st.bitmap, st.hi, st.lo)
+        q = self.gen["q"][i, b, h * self.g:(h + 1) * self.g].view(np.uint16)
+        (o.attention_fp64 if fp64 else o.attention_f32)(q, Kh, Vh, self.synth.sm_scale(w.D))
+        rec_hi, rec_lo = record_bytes(w, w.L_hi), record_bytes(w, w.L_lo)
+        new_rec = rec_hi if st.n_hi > nh_before else rec_lo
+        # append: k, v rows and score read, the record written; decode: every record and the queries
+        return (w.D * 2 * 2 + 4) + new_rec + st.n_hi * rec_hi + st.n_lo * rec_lo + self.g * w.D * 2
+
+    def step(self, fp64: bool = False) -> tuple[float, float]:
+        """One generation step of every unit; (seconds, algorithmic bytes)."""
+        i = self.step_i
+        self.step_i += 1
+        t0 = time.perf_counter()
+        nbytes = sum(self.pool.map(self._unit_step, [(u, st, i, fp64) for u, st in zip(self.units, self.states)]))
+        return time.perf_counter() - t0, float(nbytes)
+
+    def close(self):
+        self.pool.shutdown()
+
+
+def oracle_gen_baseline(w, seconds_target: float = 15.0, max_steps: int = 20, n_units: int | None = None):
+    """The oracle timed on the host's cores on a bounded sample of the generation workload: one
+    layer's units (one per core, up to 64), each running generation steps (append + dequantize +
+    attention of its g heads), until about `seconds_target` of wall time."""
+    cores = host_cores()
+    n = n_units or max(w.H, min(64, cores))
+    og = OracleGen(w, n, max_steps + 1, threads=min(cores, n))
+    try:
+        secs = nbytes = secs64 = nbytes64 = 0.0
+        steps = 0
+        s64, b64 = og.step(fp64=True)  # the parity variant (fp64 attention), one step
+        secs64, nbytes64 = s64, b64
+        while steps < max_steps and secs < seconds_target:
+            s, b = og.step(fp64=False)
+            secs += s
+            nbytes += b
+            steps += 1
+    finally:
+        og.close()
+    return {"gbs": nbytes / secs / 1e9, "gbs_fp64": nbytes64 / secs64 / 1e9, "seconds": secs, "steps": steps,
+            "units": n, "threads": og.threads, "prefill_gbs": og.prefill_bytes / og.prefill_seconds / 1e9,
+            "sample": f"{n} units (batch row x kv head) of one layer of workload {w.name}, T={og.T}: the prefill "
+                      f"(select + quantize/pack), then {steps} generation steps (append + dequantize + fp32-"
+                      f"accumulate attention) timed; fp64 attention (the parity variant) one step; units spread "
+                      f"over {og.threads} threads"}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -216,11 +340,19 @@ def oracle_sample(w, seconds_target: float = 15.0, max_units: int = 8):
 
 def workload_config(w, world: int) -> dict:
     """The `config` of both arms' JSON lines: the workload, named by what it is and its sizes."""
-    return {"workload": f"{w.name}: Llama-3.1-8B-shaped layer, B{w.B} H{w.H} Hq{w.Hq} T{w.T} D{w.D}, "
-                        f"G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}",
-"parallelism": f"dp{world} (independent units)",
-            "step": "assign_precision + quantize_pack + append_decode (append_token of one generated token per "
-                    "unit and decode_attention in one pass)"}
+    shape = (f"B{w.B} H{w.H} Hq{w.Hq} D{w.D}, G{w.G}, L {w.L_hi}/{w.L_lo}, p {w.p}")
+    if w.name == "gen":
+        text = (f"gen: Llama-3.1-8B-shaped generation, {w.layers} layers, {shape}, {w.T}-token prefill; "
+                f"step = one generated token per sequence in every layer")
+        step = "semkv_append_decode per layer (append-quantize at the running threshold + GQA decode), one graph"
+    elif w.name == "llama8b_32L":
+        text = f"llama8b_32L: Llama-3.1-8B-shaped cache, {w.layers} layers, {shape}, T{w.T}"
+        step = "semkv_decode_attention per layer, one graph"
+    else:
+        text = f"{w.name}: Llama-3.1-8B-shaped layer, {shape}, T{w.T}"
+        step = ("assign_precision + quantize_pack + append_decode (append_token of one generated token per unit "
+                "and decode_attention in one pass)")
+    return {"workload": text, "parallelism": f"dp{world} (independent units)", "step": step}
 
 
 def run_reference(args):
@@ -229,362 +361,615 @@ def run_reference(args):
         return 0
     from mixed_precision_kv_semkv_b200 import synth
 
-    w = synth.WORKLOADS[args.workload]
-    # each step is a bounded sample (one unit, ~0.5 s of the oracle on one core), so that the run
-    # ends within seconds whatever --steps asks
+    w = synth.WORKLOADS["gen"]
+    cores = host_cores()
     steps = max(1, min(args.steps, 10))
     warm = max(0, min(args.warmup, 3))
-    for _ in range(warm):
-        oracle_sample(w, seconds_target=0.0, max_units=1)
-    secs, byts = 0.0, 0.0
-    for _ in range(steps):
-        r = oracle_sample(w, seconds_target=0.0, max_units=1)
-        secs += r["seconds"]
-        byts += r["bytes"]
+    n = max(w.H, min(32, cores))
+    og = OracleGen(w, n, steps + warm + 1, threads=min(cores, n))
+    try:
+        for _ in range(warm):
+            og.step()
+        secs = byts = 0.0
+        for _ in range(steps):
+            s, b = og.step()
+            secs += s
+            byts += b
+    finally:
+        og.close()
     gbs = byts / secs / 1e9
+    sample = (f"{n} units (batch row x kv head) of one layer per step, T={w.T}: append + dequantize + fp32-"
+              f"accumulate attention, units over {og.threads} threads")
     line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": steps, "warmup": warm,
             "ms_per_step": secs / steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": dict(workload_config(w, args.gpus), sample="1 unit (one batch row x kv head) per step"),
-            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": r["sample"]},
+            "dtype": "f32", "data": "synthetic", "impl": "reference",
+            "config": dict(workload_config(w, args.gpus), sample=sample),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": og.threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-# ---------------------------------------------------------------- GPU arm
+# ---------------------------------------------------------------- GPU arm: shared pieces
 
 
-def run_semkv(args):
-    import torch
+class Gpu:
+    """Per-process GPU context: device, stream, L2 flush buffer, rank info."""
 
-    from mixed_precision_kv_semkv_b200 import (SemkvCache, build, semkv_append_decode, semkv_append_token,
-                                               semkv_append_token_running, semkv_assign_precision,
-                                               semkv_decode_attention, semkv_quantize_pack, synth)
+    def __init__(self, args):
+        import torch
 
-    world, rank, local = rank_env()
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
+        self.torch = torch
+        self.args = args
+        self.world, self.rank, self.local = rank_env()
+        torch.cuda.set_device(self.local)
+        self.dist = None
+        if self.world > 1:
+            import datetime
 
-        import torch.distributed as dist
+            import torch.distributed as dist
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    build.build()
-    w = synth.WORKLOADS[args.workload]
-    T = w.T
-    d = synth.layer_gpu(w, seed=rank_seed(rank))
-    K, V, S, q = d["K"], d["V"], d["scores"], d["q"]
-    # one generated token per unit: its k, v rows and score (appended after the prefill every step)
-    gen = synth.gen_steps_gpu(w, K, seed=rank_seed(rank), layer=0, steps=1)
-    kn, vn, sn = (gen[x][0].contiguous() for x in ("k", "v", "scores"))
-    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=1, window=WINDOW)
-    ws = cache.workspace()
-    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")  # the step's attention output
-    out_s = torch.empty_like(out)  # the same, from the separate append and decode calls
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.dist = dist
+        self.stream = torch.cuda.current_stream()
+        self.flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+        self.seed = rank_seed(self.rank)
+
+    def flush(self):
+        self.flush_buf.zero_()
+
+    def event(self):
+        return self.torch.cuda.Event(enable_timing=True)
+
+    def graph(self, fn):
+        fn()  # eager once: module loading and kernel attributes happen outside capture
+        self.torch.cuda.synchronize()
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g, capture_error_mode="relaxed"):
+            fn()
+        return g
+
+    def time_graph(self, g, reps: int, before=(), flush: bool = True) -> float:
+        """Average ms of one replay of g (events around it on the launching stream), each rep after
+        an optional L2 flush and the untimed graphs `before`."""
+        pairs = []
+        for _ in range(reps):
+            if flush:
+                self.flush()
+            for b in before:
+                b.replay()
+            e0, e1 = self.event(), self.event()
+            e0.record(self.stream)
+            g.replay()
+            e1.record(self.stream)
+            pairs.append((e0, e1))
+        self.torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in pairs) / reps
+
+
+def hbm_peak():
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(peaks["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+def captured_traffic(name: str, kernel_key: str):
+    """DRAM bytes per launch of a kernel from the committed ncu capture, if its sources are
+    unchanged since (profiles/traffic_<name>.json holds the sources' sha256)."""
+    try:
+        import hashlib
+
+        prof = json.load(open(os.path.join(ROOT, "profiles", f"traffic_{name}.json")))
+        m = hashlib.sha256()
+        for f in prof["sources"][kernel_key]:
+            m.update(open(os.path.join(ROOT, f), "rb").read())
+        if m.hexdigest() == prof["source_sha256"][kernel_key]:
+            return prof[kernel_key]
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+def counts(caches):
+    """Per layer: (sum of n_hi over units, sum of n_lo over units) (synchronizes)."""
+    nh = [int(c.bufs["n_hi"].sum().item()) for c in caches]
+    nl = [int(c.bufs["n_lo"].sum().item()) for c in caches]
+    return nh, nl
+
+
+def prefill_layer(gpu, w, cache, d, T):
+    """semkv_assign_precision then semkv_quantize_pack of one layer, each timed after an L2 flush;
+    returns (select ms, quantize ms)."""
+    from mixed_precision_kv_semkv_b200 import semkv_assign_precision, semkv_quantize_pack
+
+    gpu.flush()
+    e = [gpu.event() for _ in range(3)]
+    e[0].record(gpu.stream)
+    semkv_assign_precision(cache, d["scores"], T, w.p)
+    e[1].record(gpu.stream)
+    gpu.flush()  # the quantization reads the fp16 rows from HBM, not from L2
+    e[1].synchronize()
+    e1b = gpu.event()
+    e1b.record(gpu.stream)
+    semkv_quantize_pack(cache, d["K"], d["V"], T)
+    e[2].record(gpu.stream)
+    e[2].synchronize()
+    return e[0].elapsed_time(e[1]), e1b.elapsed_time(e[2])
+
+
+# ---------------------------------------------------------------- GPU arm: generation workload
+
+
+def run_gen(gpu, w, K: int, W: int, want_e2e: bool):
+    """The generation workload: prefill of every layer, then K timed generation steps (each one
+    graph of the layers' append_decode calls), plus the decode calls alone and, optionally, the
+    end-to-end steps with host buffers."""
+    torch = gpu.torch
+    from mixed_precision_kv_semkv_b200 import SemkvCache, semkv_append_decode, semkv_decode_attention, synth
+
+    layers = gpu.args.layers or w.layers
+    E = min(K, 10) if want_e2e else 0
+    S = 1 + W + K + E  # generated tokens per unit: the eager capture step, warm-up, timed, end-to-end
+    T, U = w.T, w.B * w.H
+    caches, t_sel, t_q = [], [], []
+    pool_k = torch.empty((S, layers, w.B, w.H, w.D), dtype=torch.float16, device="cuda")
+    pool_v = torch.empty_like(pool_k)
+    pool_s = torch.empty((S, layers, w.B, w.H), dtype=torch.float32, device="cuda")
+    pool_q = torch.empty((S, layers, w.B, w.Hq, w.D), dtype=torch.float16, device="cuda")
+    for layer in range(layers):
+        d = synth.layer_gpu(w, gpu.seed, layer=layer)
+        cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=S)
+        ts, tq = prefill_layer(gpu, w, cache, d, T)
+        t_sel.append(ts)
+        t_q.append(tq)
+        gen = synth.gen_steps_gpu(w, d["K"], gpu.seed, layer, S)
+        pool_k[:, layer] = gen["k"]
+        pool_v[:, layer] = gen["v"]
+        pool_s[:, layer] = gen["scores"]
+        pool_q[:, layer] = gen["q"]
+        caches.append(cache)
+        del d, gen
+    torch.cuda.synchronize()
+    assert all(c.status() == 0 for c in caches), "device status after the prefill"
+    nh_pre, nl_pre = counts(caches)
+    nb_layer = alg_bytes(w, T, nh_pre[0] // U)
+    prefill = {"select_ms": sum(t_sel), "quantize_ms": sum(t_q),
+               "select_gbs": layers * nb_layer["select"] / (sum(t_sel) * 1e-3) / 1e9,
+               "quantize_gbs": sum(alg_bytes(w, T, nh // U)["quantize"] for nh in nh_pre) / (sum(t_q) * 1e-3) / 1e9}
+    torch.cuda.empty_cache()
+
+    cur_k, cur_v, cur_s, cur_q = (torch.empty_like(x[0]) for x in (pool_k, pool_v, pool_s, pool_q))
+    out = torch.empty((layers, w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    ws = caches[0].workspace()
     scale = synth.sm_scale(w.D)
-    from mixed_precision_kv_semkv_b200.cache import n_hi_for
+    si = [0]  # next generated token of the pool
 
-    stream = torch.cuda.current_stream()
+    def stage(i):
+        cur_k.copy_(pool_k[i])
+        cur_v.copy_(pool_v[i])
+        cur_s.copy_(pool_s[i])
+        cur_q.copy_(pool_q[i])
 
-    # each C-ABI call is captured once into its own CUDA graph: replaying it costs the host a few
-    # microseconds, so the device timings below are not bounded by Python/ctypes enqueue time
-    calls = [lambda: semkv_assign_precision(cache, S, T, w.p),
-             lambda: semkv_quantize_pack(cache, K, V, T),
+    def step_calls():
+        for layer in range(layers):
+            semkv_append_decode(caches[layer], cur_k[layer], cur_v[layer], cur_s[layer], cur_q[layer], scale,
+                                out[layer], ws)
+
+    stage(0)
+    step_graph = gpu.graph(step_calls)  # the eager call appends pool token 0
+    si[0] = 1
+    for _ in range(W):
+        stage(si[0])
+        si[0] += 1
+        step_graph.replay()
+    torch.cuda.synchronize()
+    assert all(c.status() == 0 for c in caches), "device status after the warm-up"
+    nh0, nl0 = counts(caches)
+
+    clocks = Clocks(gpu.local)
+    if not gpu.args.profile:
+        clocks.start()
+        time.sleep(0.3)
+    if gpu.dist is not None:
+        gpu.dist.barrier()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(K):
+        stage(si[0])  # this step's generated tokens into the graph's input buffers (untimed)
+        si[0] += 1
+        e0, e1 = gpu.event(), gpu.event()
+        e0.record(gpu.stream)
+        step_graph.replay()
+        e1.record(gpu.stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    if gpu.dist is not None:
+        gpu.dist.barrier()
+    ck = clocks.stop() if not gpu.args.profile else {}
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(sum(step_ms), gpu.dist, "cuda")
+    nh1, nl1 = counts(caches)
+    assert all(c.status() == 0 for c in caches), "device status after the timed steps"
+    nb = gen_steps_bytes(w, nh0, nl0, nh1, nl1, K)
+
+    # the decode calls alone (graph of the layers' decode_attention), over the cache as it is now
+    def decode_calls():
+        for layer in range(layers):
+            semkv_decode_attention(caches[layer], cur_q[layer], scale, out[layer], ws)
+
+    dec_graph = gpu.graph(decode_calls)
+    dec_ms = gpu.time_graph(dec_graph, reps=min(max(K, 3), 20), flush=False)
+    dec_bytes = decode_bytes_now(w, nh1, nl1)
+
+    e2e = None
+    if E:
+        hk, hv, hs, hq = (x[si[0]:si[0] + E].cpu().pin_memory() for x in (pool_k, pool_v, pool_s, pool_q))
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        nh2, nl2 = counts(caches)
+        torch.cuda.synchronize()
+        e0, e1 = gpu.event(), gpu.event()
+        e0.record(gpu.stream)
+        for i in range(E):
+            cur_k.copy_(hk[i], non_blocking=True)
+            cur_v.copy_(hv[i], non_blocking=True)
+            cur_s.copy_(hs[i], non_blocking=True)
+            cur_q.copy_(hq[i], non_blocking=True)
+            step_graph.replay()
+            hout.copy_(out, non_blocking=True)
+        e1.record(gpu.stream)
+        e1.synchronize()
+        el = max_over_ranks(e0.elapsed_time(e1), gpu.dist, "cuda")
+        nh3, nl3 = counts(caches)
+        nbe = gen_steps_bytes(w, nh2, nl2, nh3, nl3, E)
+        h2d = sum(x[0].numel() * x[0].element_size() for x in (hk, hv, hs, hq))
+        e2e = {"value": gpu.world * nbe["total"] / (el * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hout.numel() * 4, "ms_per_step": el / E,
+               "path": "per step: pinned host -> device copies of the step's generated k, v, scores and queries "
+                       "(all layers), the step's graph, device -> pinned host copy of every layer's attention "
+                       "output"}
+        si[0] += E
+    assert all(c.status() == 0 for c in caches), "device status at the end"
+    del step_graph, dec_graph
+    res = {"total_ms": total_ms, "step_bytes": nb["total"] / K, "bytes": nb, "step_ms": step_ms, "clocks": ck,
+           "prefill": prefill, "decode_ms": dec_ms, "decode_bytes": dec_bytes, "layers": layers, "e2e": e2e,
+           "launches_per_step": layers * DECODE_KERNELS_PER_CALL, "T_end": T + si[0]}
+    caches.clear()
+    del pool_k, pool_v, pool_s, pool_q, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- GPU arm: 32-layer decode
+
+
+def run_decode_layers(gpu, w, K: int, W: int):
+    """A multi-layer cache (one prefill per layer), then K timed steps of one graph holding every
+    layer's semkv_decode_attention."""
+    torch = gpu.torch
+    from mixed_precision_kv_semkv_b200 import SemkvCache, semkv_decode_attention, synth
+
+    layers = gpu.args.layers or w.layers
+    caches, qs, t_sel, t_q = [], [], [], []
+    for layer in range(layers):
+        d = synth.layer_gpu(w, gpu.seed, layer=layer)
+        cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, w.T, w.p)
+        ts, tq = prefill_layer(gpu, w, cache, d, w.T)
+        t_sel.append(ts)
+        t_q.append(tq)
+        caches.append(cache)
+        qs.append(d["q"].clone())
+        del d
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    assert all(c.status() == 0 for c in caches)
+    nh, nl = counts(caches)
+    out = torch.empty((layers, w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    ws = caches[0].workspace()
+    scale = synth.sm_scale(w.D)
+
+    def calls():
+        for layer in range(layers):
+            semkv_decode_attention(caches[layer], qs[layer], scale, out[layer], ws)
+
+    g = gpu.graph(calls)
+    for _ in range(W):
+        g.replay()
+    ms = gpu.time_graph(g, reps=K, flush=False)  # the step reads every layer's cache: far more than L2
+    byts = decode_bytes_now(w, nh, nl)
+    U = w.B * w.H
+    peak, _ = hbm_peak()
+    res = {"ms_per_step": ms, "gbs": byts / (ms * 1e-3) / 1e9, "frac": byts / (ms * 1e-3) / 1e9 / peak,
+           "bytes_per_step": byts, "steps": K, "layers": layers,
+           "prefill_select_gbs": sum(alg_bytes(w, w.T, a // U)["select"] for a in nh) / (sum(t_sel) * 1e-3) / 1e9,
+           "prefill_quantize_gbs": sum(alg_bytes(w, w.T, a // U)["quantize"] for a in nh) / (sum(t_q) * 1e-3) / 1e9,
+           "launches_per_step": layers * DECODE_KERNELS_PER_CALL}
+    assert all(c.status() == 0 for c in caches)
+    del g
+    caches.clear()
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- GPU arm: one-layer step and variants
+
+
+def run_one_layer(gpu, w, K: int, W: int, variants: bool = True):
+    """One layer: select + quantize + append_decode as one graph, timed over K steps with an L2
+    flush between them; the per-call split and (with `variants`) the quantizer variants, each call
+    from a graph of its own."""
+    torch = gpu.torch
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, semkv_append_decode, semkv_append_token,
+                                               semkv_append_token_running, semkv_assign_precision,
+                                               semkv_capacities, semkv_decode_attention, semkv_quantize_pack, synth)
+
+    T = w.T
+    d = synth.layer_gpu(w, seed=gpu.seed)
+    K_, V_, S_, q = d["K"], d["V"], d["scores"], d["q"]
+    gen = synth.gen_steps_gpu(w, K_, seed=gpu.seed, layer=0, steps=1)
+    kn, vn, sn = (gen[x][0].contiguous() for x in ("k", "v", "scores"))
+    # room for the recent-window variant below; the step itself runs the plain selection
+    cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=1, window=WINDOW)
+    cache.struct.window = 0
+    ws = cache.workspace()
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    out_s = torch.empty_like(out)
+    scale = synth.sm_scale(w.D)
+    calls = [lambda: semkv_assign_precision(cache, S_, T, w.p),
+             lambda: semkv_quantize_pack(cache, K_, V_, T),
              lambda: semkv_append_token(cache, kn, vn, sn),
              lambda: semkv_decode_attention(cache, q, scale, out_s, ws)]
     names = ("select", "quantize", "append", "decode_in_step")
-    for c in calls:  # eager once: module loading and kernel attributes happen outside capture
+    for c in calls:
         c()
     torch.cuda.synchronize()
-    # which units' new token went to the L_hi grid (the same every step: same inputs)
-    n_hi0 = n_hi_for(w.p, T)
+    n_hi0 = semkv_capacities(T, w.p)[0]
     new_hi = int((cache.bufs["n_hi"] - n_hi0).sum().item())
     nb = alg_bytes(w, T, n_hi0, new_hi, appended=True)
-    step_bytes = nb["select"] + nb["quantize"] + nb["append"] + nb["decode"]  # the three calls below do this
-    # the step as one CUDA graph (as a serving loop would capture it): the timed `value`; and each
-    # call in a graph of its own: the per-call split (each then also pays its own graph launch)
+    step_bytes = nb["select"] + nb["quantize"] + nb["append"] + nb["decode"]
     fused_call = lambda: semkv_append_decode(cache, kn, vn, sn, q, scale, out, ws)  # noqa: E731
-    step_calls = (calls[0], calls[1], fused_call)
-    calls[0]()  # a fresh prefill first: the cache holds room for one appended token
+    calls[0]()
     calls[1]()
     fused_call()
     torch.cuda.synchronize()
     assert torch.equal(out, out_s), "append+decode in one pass differs from append then decode"
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph, capture_error_mode="relaxed"):
-        for c in step_calls:
-            c()
+        calls[0]()
+        calls[1]()
+        fused_call()
     graphs = []
     for c in calls:
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, capture_error_mode="relaxed"):
             c()
         graphs.append(gr)
-    # the running top-p append (the same token, ranked against every stored score) for the split
-    run_call = lambda: semkv_append_token_running(cache, kn, vn, sn, w.p)  # noqa: E731
-    calls[0]()  # a fresh prefill first: the cache holds room for one appended token
-    calls[1]()
-    run_call()
-    torch.cuda.synchronize()
-    run_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(run_graph, capture_error_mode="relaxed"):
-        run_call()
-    # append + decode in one pass (the step's last call) on its own, likewise after a fresh prefill
-    fused_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(fused_graph, capture_error_mode="relaxed"):
-        fused_call()
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    for _ in range(max(W, 3)):
+        gpu.flush()
         step_graph.replay()
-        if ev is not None:
-            ev[1].record(stream)
-
-    def step_split(ev):
-        for i, gr in enumerate(graphs):
-            ev[i].record(stream)
-            gr.replay()
-        ev[len(graphs)].record(stream)
-
-    steps = 3 if args.profile else args.steps
-    warm = max(args.warmup, 3)
-    for _ in range(warm):
-        flush.zero_()
-        step()
     torch.cuda.synchronize()
-    assert cache.status() == 0, f"device status {cache.status()}"
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
-    clocks = Clocks(local)
-    if not args.profile:
-        clocks.start()
-        time.sleep(0.3)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    for i in range(steps):
-        flush.zero_()  # L2 flush between steps, outside the step's events
-        step(evs[i])
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    ck = clocks.stop() if not args.profile else {}
-    total_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), dist, "cuda")
-    value = weak_scaling_value(world, step_bytes, steps, total_ms)
-
-    # per-call split, outside the timed region
-    split_steps = min(steps, 300)
-    evs_split = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(split_steps)]
-    for i in range(split_steps):
-        flush.zero_()
-        step_split(evs_split[i])
-    torch.cuda.synchronize()
-    t_call = [sum(e[i].elapsed_time(e[i + 1]) for e in evs_split) * steps / split_steps for i in range(len(graphs))]
-    # running append and fused append+decode: each after a fresh prefill (select + quantize
-    # replayed untimed), from a graph of its own
-    def after_prefill(gr):
-        t = 0.0
-        for i in range(split_steps):
-            flush.zero_()
-            graphs[0].replay()
-            graphs[1].replay()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            gr.replay()
-            e1.record(stream)
-            e1.synchronize()
-            t += e0.elapsed_time(e1)
-        return t / split_steps
-
-    t_run = after_prefill(run_graph)
-    t_fused = after_prefill(fused_graph)
-    # the quantizer variants on the same workload, each call in a graph of its own: the selection
-    # with a recent window of WINDOW tokens, the quantization with a clipped range (clip CLIP,
-    # which runs the generic quantize kernel)
-    cache.struct.window = WINDOW
-    win_graph = torch.cuda.CUDAGraph()
-    calls[0]()
-    with torch.cuda.graph(win_graph, capture_error_mode="relaxed"):
-        calls[0]()
-    cache.struct.window = 0
-    calls[0]()
-    cache.struct.clip = CLIP
-    clip_graph = torch.cuda.CUDAGraph()
-    calls[1]()
-    with torch.cuda.graph(clip_graph, capture_error_mode="relaxed"):
-        calls[1]()
-    cache.struct.clip = 0.0
-    torch.cuda.synchronize()
-
-    def timed(gr, before=()):
-        t = 0.0
-        for i in range(split_steps):
-            flush.zero_()
-            for b in before:
-                b.replay()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            gr.replay()
-            e1.record(stream)
-            e1.synchronize()
-            t += e0.elapsed_time(e1)
-        return t / split_steps
-
-    t_win = timed(win_graph)
-    t_clip = timed(clip_graph, before=(graphs[0],))
-    # V level counts of their own: quantize (runtime-L kernel) and decode (tensor cores, own V radix)
-    cache.struct.L_hi_v, cache.struct.L_lo_v = V_LEVELS
-    calls[0]()
-    calls[1]()
-    kvq_graph, kvd_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(kvq_graph, capture_error_mode="relaxed"):
-        calls[1]()
-    out_v = torch.empty_like(out)
-    kv_decode = lambda: semkv_decode_attention(cache, q, scale, out_v, ws)  # noqa: E731
-    kv_decode()
-    with torch.cuda.graph(kvd_graph, capture_error_mode="relaxed"):
-        kv_decode()
-    cache.struct.L_hi_v, cache.struct.L_lo_v = 0, 0
-    torch.cuda.synchronize()
-    t_kvq = timed(kvq_graph, before=(graphs[0],))
-    t_kvd = timed(kvd_graph, before=(graphs[0], kvq_graph))
-    nb_kv = alg_bytes(w, T, n_hi0, v_levels=V_LEVELS)
-    # per-channel K grids: quantize (grid pass over K, then the runtime-L kernel) and decode (CUDA cores)
-    cache.struct.k_per_channel = 1
-    calls[0]()
-    calls[1]()
-    kpq_graph, kpd_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(kpq_graph, capture_error_mode="relaxed"):
-        calls[1]()
-    kv_decode()
-    with torch.cuda.graph(kpd_graph, capture_error_mode="relaxed"):
-        kv_decode()
-    cache.struct.k_per_channel = 0
-    torch.cuda.synchronize()
-    t_kpq = timed(kpq_graph, before=(graphs[0],))
-    t_kpd = timed(kpd_graph, before=(graphs[0], kpq_graph))
-    kpc_range_bytes = w.B * w.H * T * w.D * 2  # the grid pass reads K once more
-    assert cache.status() == 0, f"device status {cache.status()}"
-    assert torch.equal(out, out_s), "append+decode in one pass differs from append then decode"
-    # leave the cache as a timed step leaves it (prefill + the fixed-threshold append)
-    for gr in graphs[:3]:
-        gr.replay()
-    torch.cuda.synchronize()
-
-    # decode alone over an L2-cold cache (decode-attn HBM GB/s of the metric)
-    dec_ms = []
-    for _ in range(min(steps, 200)):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        graphs[3].replay()
-        e1.record(stream)
-        dec_ms.append((e0, e1))
-    torch.cuda.synchronize()
-    dec_cold = sum(a.elapsed_time(b) for a, b in dec_ms) / len(dec_ms)
-
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    except OSError:
-        pass
-    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
-    peak_note = "measured" if "hbm_gbs" in peaks else "fallback"
-    per_kernel = {
-        nm: {"ms": t / steps, "gbs": nb[nm.replace("_in_step", "")] / (t / steps * 1e-3) / 1e9}
-        for nm, t in zip(names, t_call)
-    }
+    step_ms = gpu.time_graph(step_graph, reps=K)
+    t_call = [gpu.time_graph(g, reps=min(K, 300)) for g in graphs]
+    per_kernel = {nm: {"ms": t, "gbs": nb[nm.replace("_in_step", "")] / (t * 1e-3) / 1e9}
+                  for nm, t in zip(names, t_call)}
+    # the fused call and the running append on their own, each after a fresh prefill
+    run_call = lambda: semkv_append_token_running(cache, kn, vn, sn, w.p)  # noqa: E731
+    graphs[0].replay()
+    graphs[1].replay()
+    run_graph = gpu.graph(run_call)
+    graphs[0].replay()
+    graphs[1].replay()
+    fused_graph = gpu.graph(fused_call)
+    t_run = gpu.time_graph(run_graph, reps=min(K, 300), before=graphs[:2])
+    t_fused = gpu.time_graph(fused_graph, reps=min(K, 300), before=graphs[:2])
+    graphs[0].replay()
+    graphs[1].replay()
+    graphs[2].replay()
+    t_dec_cold = gpu.time_graph(graphs[3], reps=min(K, 200))
     per_kernel.update({
-        "decode_l2_cold": {"ms": dec_cold, "gbs": nb["decode"] / (dec_cold * 1e-3) / 1e9},
+        "decode_l2_cold": {"ms": t_dec_cold, "gbs": nb["decode"] / (t_dec_cold * 1e-3) / 1e9},
         "append_running": {"ms": t_run, "gbs": nb["append_running"] / (t_run * 1e-3) / 1e9},
         "append_decode": {"ms": t_fused, "gbs": (nb["append"] + nb["decode"]) / (t_fused * 1e-3) / 1e9},
-        f"select_window{WINDOW}": {"ms": t_win, "gbs": nb["select"] / (t_win * 1e-3) / 1e9},
-        f"quantize_clip{CLIP}": {"ms": t_clip, "gbs": nb["quantize"] / (t_clip * 1e-3) / 1e9},
-        "quantize_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvq, "gbs": nb_kv["quantize"] / (t_kvq * 1e-3) / 1e9},
-        "decode_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvd, "gbs": nb_kv["decode"] / (t_kvd * 1e-3) / 1e9},
-        "quantize_k_per_channel": {"ms": t_kpq, "gbs": (nb["quantize"] + kpc_range_bytes) / (t_kpq * 1e-3) / 1e9},
-        "decode_k_per_channel": {"ms": t_kpd, "gbs": nb["decode"] / (t_kpd * 1e-3) / 1e9},
     })
-    dom = max(("select", "quantize", "append_decode"), key=lambda k: per_kernel[k]["ms"])
-    dom_name = {"select": "semkv_assign_precision (k_select_cluster)",
-                "quantize": "semkv_quantize_pack (k_quantize_fast)",
-                "append_decode": "semkv_append_decode (k_decode_tc x 2 + k_decode_merge)"}[dom]
-    ach = per_kernel[dom]["gbs"]
-    traffic = None  # DRAM bytes per launch from the committed ncu capture, if the kernel is unchanged since
-    try:
-        import hashlib
+    if variants:
+        cache.struct.window = WINDOW
+        win_graph = gpu.graph(calls[0])
+        cache.struct.window = 0
+        calls[0]()
+        cache.struct.clip = CLIP
+        clip_graph = gpu.graph(calls[1])
+        cache.struct.clip = 0.0
+        torch.cuda.synchronize()
+        t_win = gpu.time_graph(win_graph, reps=min(K, 300))
+        t_clip = gpu.time_graph(clip_graph, reps=min(K, 300), before=(graphs[0],))
+        cache.struct.L_hi_v, cache.struct.L_lo_v = V_LEVELS
+        calls[0]()
+        kvq_graph = gpu.graph(calls[1])
+        out_v = torch.empty_like(out)
+        kv_decode = lambda: semkv_decode_attention(cache, q, scale, out_v, ws)  # noqa: E731
+        kvd_graph = gpu.graph(kv_decode)
+        cache.struct.L_hi_v, cache.struct.L_lo_v = 0, 0
+        t_kvq = gpu.time_graph(kvq_graph, reps=min(K, 300), before=(graphs[0],))
+        t_kvd = gpu.time_graph(kvd_graph, reps=min(K, 300), before=(graphs[0], kvq_graph))
+        nb_kv = alg_bytes(w, T, n_hi0, v_levels=V_LEVELS)
+        cache.struct.k_per_channel = 1
+        calls[0]()
+        kpq_graph = gpu.graph(calls[1])
+        kpd_graph = gpu.graph(kv_decode)
+        cache.struct.k_per_channel = 0
+        t_kpq = gpu.time_graph(kpq_graph, reps=min(K, 300), before=(graphs[0],))
+        t_kpd = gpu.time_graph(kpd_graph, reps=min(K, 300), before=(graphs[0], kpq_graph))
+        kpc_range_bytes = w.B * w.H * T * w.D * 2  # the grid pass reads K once more
+        per_kernel.update({
+            f"select_window{WINDOW}": {"ms": t_win, "gbs": nb["select"] / (t_win * 1e-3) / 1e9},
+            f"quantize_clip{CLIP}": {"ms": t_clip, "gbs": nb["quantize"] / (t_clip * 1e-3) / 1e9},
+            "quantize_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvq, "gbs": nb_kv["quantize"] / (t_kvq * 1e-3) / 1e9},
+            "decode_v_levels{}_{}".format(*V_LEVELS): {"ms": t_kvd, "gbs": nb_kv["decode"] / (t_kvd * 1e-3) / 1e9},
+            "quantize_k_per_channel": {"ms": t_kpq,
+                                       "gbs": (nb["quantize"] + kpc_range_bytes) / (t_kpq * 1e-3) / 1e9},
+            "decode_k_per_channel": {"ms": t_kpd, "gbs": nb["decode"] / (t_kpd * 1e-3) / 1e9},
+        })
+    torch.cuda.synchronize()
+    assert cache.status() == 0, f"device status {cache.status()}"
+    peak, _ = hbm_peak()
+    res = {"ms_per_step": step_ms, "gbs": step_bytes / (step_ms * 1e-3) / 1e9, "step_bytes": step_bytes,
+           "per_kernel": per_kernel, "quantize_frac": per_kernel["quantize"]["gbs"] / peak,
+           "decode_frac": per_kernel["decode_l2_cold"]["gbs"] / peak,
+           "timing": "step = one CUDA graph of select, quantize and append_decode, L2 flushed (512 MB write) "
+                     "between steps; per_kernel = each call from a graph of its own, L2 flushed before it"}
+    del graphs, step_graph
+    torch.cuda.empty_cache()
+    return res
 
-        prof = json.load(open(os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")))
-        m = hashlib.sha256()
-        for f in prof["sources"][dom]:
-            m.update(open(os.path.join(ROOT, f), "rb").read())
-        if m.hexdigest() == prof["source_sha256"][dom]:
-            traffic = prof[dom]
-    except (OSError, ValueError, KeyError):
-        pass
 
-    e2e = None
-    if not args.no_e2e and not args.profile:
-        hK, hV, hS, hq, hk, hv, hs = (t.cpu().pin_memory() for t in (K, V, S, q, kn, vn, sn))
-        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-        e2e_steps = min(steps, 20)
-        el = 0.0
-        for i in range(e2e_steps + 2):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            K.copy_(hK, non_blocking=True)
-            V.copy_(hV, non_blocking=True)
-            S.copy_(hS, non_blocking=True)
-            q.copy_(hq, non_blocking=True)
-            kn.copy_(hk, non_blocking=True)
-            vn.copy_(hv, non_blocking=True)
-            sn.copy_(hs, non_blocking=True)
-            step()
-            hout.copy_(out, non_blocking=True)
-            e1.record(stream)
-            e1.synchronize()
-            if i >= 2:
-                el += e0.elapsed_time(e1)
-        el = max_over_ranks(el, dist, "cuda")  # every rank gets here (same flags): the slowest rank's time
-        h2d = sum(t.numel() * t.element_size() for t in (hK, hV, hS, hq, hk, hv, hs))
-        e2e = {"value": world * step_bytes * e2e_steps / (el * 1e-3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * 4,
-               "ms_per_step": el / e2e_steps}
+# ---------------------------------------------------------------- GPU arm: precision sweep
+
+
+def run_sweep(gpu, w, reps: int = 20):
+    """The Mistral-7B-shaped cache (one layer: batch 8, 8 KV heads, T 32768) at every (level pair,
+    p, G) point: prefill, then the decode timed over an L2-cold cache; the storage ratio against
+    fp16 comes from the cache's buffer sizes."""
+    torch = gpu.torch
+    from mixed_precision_kv_semkv_b200 import (SemkvCache, semkv_assign_precision, semkv_decode_attention,
+                                               semkv_quantize_pack, synth)
+
+    d = synth.layer_gpu(w, gpu.seed, layer=0)
+    T = w.T
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    scale = synth.sm_scale(w.D)
+    peak, _ = hbm_peak()
+    fp16_bytes = w.B * w.H * T * w.D * 2 * 2
+    pts = []
+    for (Lh, Ll) in synth.SWEEP_PAIRS:
+        for p in synth.SWEEP_P:
+            for G in synth.SWEEP_G:
+                cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, G, Lh, Ll, T, p)
+                semkv_assign_precision(cache, d["scores"], T, p)
+                semkv_quantize_pack(cache, d["K"], d["V"], T)
+                ws = cache.workspace()
+                g = gpu.graph(lambda: semkv_decode_attention(cache, d["q"], scale, out, ws))  # noqa: B023
+                ms = gpu.time_graph(g, reps=reps)
+                nh = int(cache.bufs["n_hi"].sum().item())
+                nl = int(cache.bufs["n_lo"].sum().item())
+                assert cache.status() == 0
+                wq = type(w)(w.name, w.B, w.H, w.Hq, T, G, Lh, Ll, p)
+                byts = nh * record_bytes(wq, Lh) + nl * record_bytes(wq, Ll) + w.B * w.Hq * w.D * 2
+                gbs = byts / (ms * 1e-3) / 1e9
+                ratio = fp16_bytes / cache.packed_bytes
+                assert abs(ratio - storage_ratio(w.D, G, Lh, Ll, p, T, B=w.B, H=w.H)) < 1e-12
+                pts.append({"L_hi": Lh, "L_lo": Ll, "p": p, "G": G, "ratio_vs_fp16": ratio,
+                            "decode_ms": ms, "decode_gbs": gbs, "decode_frac": gbs / peak})
+                del g, cache, ws
+    del d
+    torch.cuda.empty_cache()
+    return pts
+
+
+# ---------------------------------------------------------------- GPU arm: the JSON line
+
+
+def run_semkv(args):
+    gpu = Gpu(args)
+    torch = gpu.torch
+    from mixed_precision_kv_semkv_b200 import build, synth
+
+    build.build()
+    w = synth.WORKLOADS[args.workload]
+    K = 3 if args.profile else args.steps
+    W = max(args.warmup, 3)
+    want_e2e = not (args.no_e2e or args.profile)
+    peak, peak_kind = hbm_peak()
+    extras, per_kernel, sweep = {}, {}, None
+
+    if w.name == "gen":
+        r = run_gen(gpu, w, K, W, want_e2e)
+        value = weak_scaling_value(gpu.world, r["step_bytes"], K, r["total_ms"])
+        ms_step = r["total_ms"] / K
+        layer_ms = ms_step / r["layers"]
+        layer_bytes = r["step_bytes"] / r["layers"]
+        dom_name = "semkv_append_decode per layer (k_decode_tc hi + lo grids, k_decode_merge)"
+        ach = layer_bytes / (layer_ms * 1e-3) / 1e9
+        per_kernel = {
+            "append_decode_layer": {"ms": layer_ms, "gbs": ach},
+            "decode_32L": {"ms": r["decode_ms"], "gbs": r["decode_bytes"] / (r["decode_ms"] * 1e-3) / 1e9,
+                           "frac": r["decode_bytes"] / (r["decode_ms"] * 1e-3) / 1e9 / peak},
+            "prefill_select": {"ms": r["prefill"]["select_ms"], "gbs": r["prefill"]["select_gbs"]},
+            "prefill_quantize": {"ms": r["prefill"]["quantize_ms"], "gbs": r["prefill"]["quantize_gbs"],
+                                 "frac": r["prefill"]["quantize_gbs"] / peak},
+        }
+        dec_gbs = per_kernel["decode_32L"]["gbs"]
+        launches = r["launches_per_step"] * K
+        clocks, e2e = r["clocks"], r["e2e"]
+        traffic = captured_traffic("gen", "append_decode")
+        cfg_extra = {"l2": "not flushed: a step reads far more than the 126 MB L2",
+                     "generated_tokens": f"T grows from {w.T} (prefill) to {r['T_end']} over the run",
+                     "timing": "per step: CUDA events around one replay of the step graph; the step's generated "
+                               "tokens are staged into the graph's input buffers before the first event"}
+        steps_ms = r["step_ms"]
+    elif w.name == "llama8b_32L":
+        r = run_decode_layers(gpu, w, K, W)
+        value = weak_scaling_value(gpu.world, r["bytes_per_step"], K, max_over_ranks(r["ms_per_step"] * K, gpu.dist,
+                                                                                      "cuda"))
+        ms_step = r["ms_per_step"]
+        dom_name = "semkv_decode_attention per layer (k_decode_tc hi + lo grids, k_decode_merge)"
+        ach = r["gbs"]
+        dec_gbs = r["gbs"]
+        launches = r["launches_per_step"] * K
+        clocks, e2e, traffic, steps_ms = {}, None, captured_traffic("llama8b_32L", "decode"), None
+        cfg_extra = {"l2": "not flushed: a step reads far more than the 126 MB L2"}
+    else:
+        r = run_one_layer(gpu, w, K, W)
+        value = weak_scaling_value(gpu.world, r["step_bytes"], K, max_over_ranks(r["ms_per_step"] * K, gpu.dist,
+                                                                                 "cuda"))
+        ms_step = r["ms_per_step"]
+        per_kernel = r["per_kernel"]
+        dom = max(("select", "quantize", "append_decode"), key=lambda k: per_kernel[k]["ms"])
+        dom_name = {"select": "semkv_assign_precision (k_select_cluster)",
+                    "quantize": "semkv_quantize_pack (k_quantize_fast)",
+                    "append_decode": "semkv_append_decode (k_decode_tc x 2 + k_decode_merge)"}[dom]
+        ach = per_kernel[dom]["gbs"]
+        dec_gbs = per_kernel["decode_l2_cold"]["gbs"]
+        launches = (2 + DECODE_KERNELS_PER_CALL) * K
+        clocks, e2e, traffic, steps_ms = {}, None, captured_traffic(w.name, dom), None
+        cfg_extra = {"l2": "flushed between steps (512 MB write)", "timing": r["timing"]}
+
+    if w.name == "gen" and not (args.no_extras or args.profile):
+        extras["llama8b_32L"] = run_decode_layers(gpu, synth.WORKLOADS["llama8b_32L"], min(K, 50), W)
+        extras["llama8b_1L"] = run_one_layer(gpu, synth.WORKLOADS["llama8b_1L"], min(max(K, 20), 400), W)
+        sweep = run_sweep(gpu, synth.WORKLOADS["mistral_sweep"])
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
-        r = oracle_sample(w)
-        cpu = {"value": r["gbs"], "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": r["sample"]}
+    if gpu.rank == 0 and gpu.world == 1 and not args.no_cpu_baseline and not args.profile:
+        c = oracle_gen_baseline(synth.WORKLOADS["gen"])
+        cpu = {"value": c["gbs"], "unit": "GB/s", "cores": c["threads"], "kind": "oracle", "sample": c["sample"],
+               "value_fp64_attention": c["gbs_fp64"], "prefill_gbs": c["prefill_gbs"]}
 
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warm,
-        "ms_per_step": total_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u32-packed codes, fp32 math", "data": "synthetic",
-        "config": dict(workload_config(w, world), l2="flushed between steps (512 MB write)",
-                       timing="step = one CUDA graph of its three calls; per_kernel = each call (and the separate "
-                              "append_token and decode_attention) replayed from a graph of its own (so each also pays "
-                              "a graph launch)"),
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": gpu.world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "decode: fp16 tensor-core operands (codes, queries, P' = p s_V as two fp16 limbs), fp32 "
+                 "accumulate and softmax; quantize: binary32 IEEE",
+        "data": "synthetic",
+        "config": dict(workload_config(w, gpu.world), **cfg_extra),
         "per_kernel": per_kernel,
-        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": ach / hbm_peak, "peak_kind": peak_note, "traffic": traffic,
-                     "frac_of_8000": ach / 8000.0},
-        "decode_roofline": {"achieved": per_kernel["decode_l2_cold"]["gbs"], "peak": hbm_peak,
-                            "frac": per_kernel["decode_l2_cold"]["gbs"] / hbm_peak,
-                            "frac_of_8000": per_kernel["decode_l2_cold"]["gbs"] / 8000.0},
-        "clocks": ck, "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": LAUNCHES_PER_STEP * steps,
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": ach, "peak": peak, "unit": "GB/s",
+                     "frac": ach / peak, "peak_kind": peak_kind, "traffic": traffic, "frac_of_8000": ach / 8000.0},
+        "decode_roofline": {"achieved": dec_gbs, "peak": peak, "frac": dec_gbs / peak,
+                            "frac_of_8000": dec_gbs / 8000.0},
+        "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches,
     }
-    if rank == 0:
+    if steps_ms:
+        line["step_ms_min_median_max"] = [min(steps_ms), statistics.median(steps_ms), max(steps_ms)]
+    if extras:
+        line["extras"] = extras
+    if sweep is not None:
+        line["sweep"] = sweep
+    if gpu.rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs
-    if dist is not None:
-        dist.destroy_process_group()
+    if gpu.dist is not None:
+        gpu.dist.destroy_process_group()
     return 0
 
 

@@ -143,6 +143,18 @@ enum {
  * (pointers ignored).  Pure host function.  Returns SEMKV_OK or a validation error. */
 SEMKV_API int semkv_cache_bytes(const semkv_cache_t* shape, size_t sizes[SEMKV_NBUF]);
 
+/* Sizing of a cache for a prefill (SemKV page, Abstract: the top fraction p of the tokens goes on
+ * the finer grid).  Pure host function.  For a prefill of T tokens at fraction p with the last
+ * min(window, T) tokens also on the finer grid, and room for `extra` appended tokens per unit:
+ *   *n_sel  = floor(p*T), computed in double from the binary32 p (the count semkv_assign_precision
+ *             puts on the finer grid by score),
+ *   *cap_hi = n_sel + min(window, T) + extra, *cap_lo = T - n_sel + extra (each rounded up to a
+ *             multiple of SEMKV_TILE), *T_cap = T + extra rounded up to a multiple of 32.
+ * Any output pointer may be NULL.  Returns SEMKV_ERR_INVALID_ARG for T < 0, window < 0,
+ * extra < 0, p outside [0, 1], or capacities that overflow int32. */
+SEMKV_API int semkv_capacities(int32_t T, float p, int32_t window, int32_t extra, int32_t* n_sel, int32_t* cap_hi,
+                               int32_t* cap_lo, int32_t* T_cap);
+
 /* Bytes of device workspace semkv_decode_attention needs for this shape on the current device
  * (it depends on the device's SM count, which sets the split-K factor). */
 SEMKV_API int semkv_workspace_bytes(const semkv_cache_t* shape, size_t* bytes);
@@ -226,6 +238,11 @@ SEMKV_API int semkv_append_decode(const semkv_cache_t* cache, const uint16_t* k,
  *   - The first call on a device looks up the array's device address for that device
  *     (cudaGetSymbolAddress, with that device current); make that first call before any stream
  *     capture on the device.
+ *   - Under CUDA's default lazy module loading, that first call is also when the driver loads the
+ *     array into device memory (SEMKV_NOALLOC_SCRATCH_BYTES of it).  A caller whose pool allocator
+ *     later takes all free device memory must therefore make the first call at start-up, before the
+ *     pool is created (or run with CUDA_MODULE_LOADING=EAGER, which loads it with the library);
+ *     otherwise that first call can fail with SEMKV_ERR_CUDA.
  *   - Shapes whose workspace (semkv_workspace_bytes) exceeds SEMKV_NOALLOC_SCRATCH_BYTES are
  *     rejected with SEMKV_ERR_CAPACITY before any launch.
  *   - All calls on a device share the one array and it keeps the last call's contents; nothing in

@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     semkv_append_token_running,
     semkv_assign_precision,
     semkv_cache_bytes,
+    semkv_capacities,
     semkv_decode_attention,
     semkv_decode_attention_noalloc,
     semkv_dequantize,
@@ -21,4 +22,4 @@ from ._lib import (  # noqa: F401
     semkv_workspace_bytes,
     status_string,
 )
-from .cache import SemkvCache, capacities, n_hi_for  # noqa: F401
+from .cache import SemkvCache, capacities  # noqa: F401

@@ -31,7 +31,7 @@ BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
             "semkv_append_token", "semkv_append_token_running", "semkv_append_decode", "semkv_decode_attention",
             "semkv_decode_attention_noalloc", "semkv_dequantize", "semkv_status_string", "semkv_radix_digits",
-            "semkv_p_for_ratio", "semkv_p_for_ratio_kv")
+            "semkv_p_for_ratio", "semkv_p_for_ratio_kv", "semkv_capacities")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.semkv_p_for_ratio.argtypes = [i32, i32, i32, i32, ctypes.c_double, ctypes.POINTER(ctypes.c_double)]
         L.semkv_p_for_ratio_kv.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_double,
                                            ctypes.POINTER(ctypes.c_double)]
+        i32p = ctypes.POINTER(i32)
+        L.semkv_capacities.argtypes = [i32, f32, i32, i32, i32p, i32p, i32p, i32p]
         for n in EXPORTED:
             if n not in ("semkv_status_string", "semkv_radix_digits"):
                 getattr(L, n).restype = ctypes.c_int
@@ -130,6 +132,15 @@ def semkv_p_for_ratio_kv(D: int, G: int, L_hi: int, L_lo: int, L_hi_v: int, L_lo
     _check("semkv_p_for_ratio_kv", lib().semkv_p_for_ratio_kv(int(D), int(G), int(L_hi), int(L_lo), int(L_hi_v),
                                                              int(L_lo_v), float(ratio), ctypes.byref(p)))
     return p.value
+
+
+def semkv_capacities(T: int, p: float, window: int = 0, extra: int = 0) -> tuple[int, int, int, int]:
+    """(n_sel, cap_hi, cap_lo, T_cap) of a cache for a prefill of T tokens at fraction p, with the
+    last `window` tokens also on the finer grid and room for `extra` appended tokens per unit."""
+    out = [ctypes.c_int32() for _ in range(4)]
+    _check("semkv_capacities", lib().semkv_capacities(int(T), float(p), int(window), int(extra),
+                                                      *(ctypes.byref(o) for o in out)))
+    return tuple(int(o.value) for o in out)
 
 
 def semkv_cache_bytes(cache) -> list[int]:

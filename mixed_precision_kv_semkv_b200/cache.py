@@ -5,27 +5,14 @@ semkv_cache_t descriptor that the C entry points take.
 """
 from __future__ import annotations
 
-import math
-
 from . import _lib
-
-
-def n_hi_for(p: float, T: int) -> int:
-    """floor(p*T) with p as a 32-bit float, the count semkv_assign_precision uses."""
-    import numpy as np
-
-    return int(math.floor(float(np.float32(p)) * T))
-
-
-def round_up(x: int, m: int) -> int:
-    return (x + m - 1) // m * m
 
 
 def capacities(T: int, p: float, extra: int = 0, window: int = 0):
     """(cap_hi, cap_lo, T_cap) for a prefill of T tokens at fraction p (plus a recent window of
-    `window` tokens on the finer grid) and `extra` appends."""
-    nh = n_hi_for(p, T)
-    return round_up(nh + min(window, T) + extra, 128), round_up(T - nh + extra, 128), round_up(T + extra, 32)
+    `window` tokens on the finer grid) and `extra` appends (the library's semkv_capacities)."""
+    _, ch, cl, tc = _lib.semkv_capacities(T, p, window, extra)
+    return ch, cl, tc
 
 
 class SemkvCache:

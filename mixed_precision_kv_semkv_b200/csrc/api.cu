@@ -159,6 +159,23 @@ extern "C" {
 
 int32_t semkv_radix_digits(int32_t L) { return level_ok(L) ? radix_k(L) : 0; }
 
+int semkv_capacities(int32_t T, float p, int32_t window, int32_t extra, int32_t* n_sel, int32_t* cap_hi,
+                     int32_t* cap_lo, int32_t* T_cap)
+{
+    if (T < 0 || window < 0 || extra < 0 || !(p >= 0.0f && p <= 1.0f)) return SEMKV_ERR_INVALID_ARG;
+    const long long ns = (long long)std::floor((double)p * (double)T);
+    const long long win = window < T ? window : T;
+    auto up = [](long long x, long long m) { return (x + m - 1) / m * m; };
+    const long long ch = up(ns + win + extra, TILE), cl = up((long long)T - ns + extra, TILE),
+                    tc = up((long long)T + extra, 32);
+    if (ch > INT32_MAX || cl > INT32_MAX || tc > INT32_MAX) return SEMKV_ERR_INVALID_ARG;
+    if (n_sel) *n_sel = (int32_t)ns;
+    if (cap_hi) *cap_hi = (int32_t)ch;
+    if (cap_lo) *cap_lo = (int32_t)cl;
+    if (T_cap) *T_cap = (int32_t)tc;
+    return SEMKV_OK;
+}
+
 int semkv_p_for_ratio(int32_t D, int32_t G, int32_t L_hi, int32_t L_lo, double ratio, double* p)
 {
     return semkv_p_for_ratio_kv(D, G, L_hi, L_lo, L_hi, L_lo, ratio, p);

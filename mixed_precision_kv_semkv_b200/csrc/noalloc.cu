@@ -7,7 +7,9 @@
 // keeps the split-K partials of semkv_decode_attention in a fixed array in device memory that is
 // part of the library image (SEMKV_NOALLOC_SCRATCH_BYTES per GPU that loads the library, held
 // until the process exits), and semkv_decode_attention_noalloc hands that array to the ordinary
-// decode path as its workspace.  Nothing in it allocates.
+// decode path as its workspace.  Nothing in it allocates.  With CUDA's lazy module loading the
+// driver places the array in device memory when the first call looks up its address, so a caller
+// whose pool will take all free device memory makes that first call at start-up.
 #include <mutex>
 
 #include "common.cuh"

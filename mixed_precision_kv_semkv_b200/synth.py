@@ -244,6 +244,20 @@ def layer_gpu(w: Workload, seed: int, layer: int = 0, device: str = "cuda", T: i
     return {"K": K, "V": V, "scores": S, "q": q}
 
 
+def prefill_channel_scales_gpu(w: Workload, seed: int, layer: int = 0, device: str = "cuda"):
+    """The per-channel scales (sigma_K, sigma_V), each [1][H][1][D], that layer_gpu draws first from
+    the layer's generator (None, None for the outlier workload, which has none)."""
+    import torch
+
+    if w.kv_dist not in ("lognormal", "student"):
+        return None, None
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 1000 + layer)
+    sk = torch.empty((1, w.H, 1, w.D), device=device).log_normal_(0.0, w.sigma_c, generator=g)
+    sv = torch.empty((1, w.H, 1, w.D), device=device).log_normal_(0.0, w.sigma_c, generator=g)
+    return sk, sv
+
+
 def gen_steps_gpu(w: Workload, K16, seed: int, layer: int, steps: int, device: str = "cuda"):
     """Generated tokens on the GPU: new k, v fp16 [steps][B][H][D] with the prefill's per-channel
     scales, their scores fp32 [steps][B][H] (softmax mass against 64 scoring queries, normalised by
@@ -251,12 +265,17 @@ def gen_steps_gpu(w: Workload, K16, seed: int, layer: int, steps: int, device: s
     import torch
 
     B, H, T, D = K16.shape
+    sk, sv = prefill_channel_scales_gpu(w, seed, layer, device)
     g = torch.Generator(device=device)
     g.manual_seed(seed * 1000 + layer + 500000)
-    sk = torch.empty((1, 1, H, D), device=device).log_normal_(0.0, w.sigma_c, generator=g)
-    sv = torch.empty((1, 1, H, D), device=device).log_normal_(0.0, w.sigma_c, generator=g)
-    kn = (torch.randn((steps, B, H, D), device=device, generator=g) * sk).to(torch.float16)
-    vn = (torch.randn((steps, B, H, D), device=device, generator=g) * sv).to(torch.float16)
+    if sk is None:
+        kn = torch.randn((steps, B, H, D), device=device, generator=g).to(torch.float16)
+        vn = torch.randn((steps, B, H, D), device=device, generator=g).to(torch.float16)
+    else:
+        sk = sk.reshape(1, 1, H, D)
+        sv = sv.reshape(1, 1, H, D)
+        kn = (torch.randn((steps, B, H, D), device=device, generator=g) * sk).to(torch.float16)
+        vn = (torch.randn((steps, B, H, D), device=device, generator=g) * sv).to(torch.float16)
     qs = torch.randn((steps, B, w.Hq, D), device=device, generator=g).to(torch.float16)
     qsc = torch.randn((B, H, 64, D), device=device, generator=g)
     sc = torch.empty((steps, B, H), device=device, dtype=torch.float32)

@@ -95,6 +95,8 @@ def lib():
         L.oracle_append_unit.restype = _c.c_int
         L.oracle_attention_fp64.argtypes = [_u16p, _c.c_int, _f32p, _f32p, _c.c_int32, _c.c_int, _c.c_float,
                                             _f64p]
+        L.oracle_attention_f32.argtypes = [_u16p, _c.c_int, _f32p, _f32p, _c.c_int32, _c.c_int, _c.c_float,
+                                           _f32p]
         _lib = L
     return _lib
 
@@ -302,6 +304,22 @@ def attention_fp64(q16, Khat, Vhat, sm_scale: float) -> np.ndarray:
         Vh = np.zeros((1, D), np.float32)
     out = np.zeros((g, D), np.float64)
     lib().oracle_attention_fp64(q16.ravel(), g, Kh.ravel(), Vh.ravel(), T, D, float(sm_scale), out.ravel())
+    return out
+
+
+def attention_f32(q16, Khat, Vhat, sm_scale: float) -> np.ndarray:
+    """The same attention with binary32 arithmetic and accumulation (the timed CPU baseline; parity
+    is taken against attention_fp64). q16: [g][D] uint16; Khat, Vhat: [T][D] fp32."""
+    q16 = np.ascontiguousarray(q16, dtype=np.uint16)
+    g, D = q16.shape
+    Kh = np.ascontiguousarray(Khat, dtype=np.float32)
+    Vh = np.ascontiguousarray(Vhat, dtype=np.float32)
+    T = Kh.shape[0]
+    if T == 0:
+        Kh = np.zeros((1, D), np.float32)
+        Vh = np.zeros((1, D), np.float32)
+    out = np.zeros((g, D), np.float32)
+    lib().oracle_attention_f32(q16.ravel(), g, Kh.ravel(), Vh.ravel(), T, D, float(sm_scale), out.ravel())
     return out
 
 

@@ -623,6 +623,40 @@ void oracle_attention_fp64(const uint16_t* q, int g, const float* Khat, const fl
     free(qd);
 }
 
+/*
+ * The same decode attention of one unit with binary32 arithmetic and binary32 accumulation: the
+ * timed CPU baseline of the attention (the fp64 routine above is the one parity is taken
+ * against).  SemKV page, Abstract: attention over the compressed cache, whose dequantized values
+ * Khat, Vhat are exact in binary32.  Plain loops in the order of the fp64 routine: logits
+ * l_t = sm_scale * sum_d q_d Khat[t][d], then out = sum_t exp(l_t - max) Vhat[t] / sum_t exp(l_t - max).
+ */
+void oracle_attention_f32(const uint16_t* q, int g, const float* Khat, const float* Vhat, int32_t T, int D,
+                          float sm_scale, float* out)
+{
+    float* logit = (float*)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1));
+    float* qf = (float*)malloc(sizeof(float) * (size_t)D);
+    for (int h = 0; h < g; h++) {
+        for (int d = 0; d < D; d++) qf[d] = oracle_half_to_float(q[h * D + d]);
+        float mx = -INFINITY;
+        for (int32_t t = 0; t < T; t++) {
+            float acc = 0.0f;
+            for (int d = 0; d < D; d++) acc += qf[d] * Khat[(size_t)t * D + d];
+            logit[t] = sm_scale * acc;
+            if (logit[t] > mx) mx = logit[t];
+        }
+        float l = 0.0f;
+        for (int d = 0; d < D; d++) out[h * D + d] = 0.0f;
+        for (int32_t t = 0; t < T; t++) {
+            float w = expf(logit[t] - mx);
+            l += w;
+            for (int d = 0; d < D; d++) out[h * D + d] += w * Vhat[(size_t)t * D + d];
+        }
+        for (int d = 0; d < D; d++) out[h * D + d] = (l > 0.0f) ? out[h * D + d] / l : 0.0f;
+    }
+    free(logit);
+    free(qf);
+}
+
 /* ------------------------------------------------------------------ array helpers for the tests */
 
 void oracle_half_to_float_array(const uint16_t* h, float* f, int64_t n)

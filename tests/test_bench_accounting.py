@@ -58,4 +58,55 @@ def test_reference_arm_prints_its_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert d["config"]["workload"] == bench.workload_config(synth.WORKLOADS["llama8b_1L"], 1)["workload"]
+    assert d["config"]["workload"] == bench.workload_config(synth.WORKLOADS["gen"], 1)["workload"]
+    assert d["cpu_baseline"]["cores"] >= 1
+
+
+def test_generation_step_bytes_by_hand():
+    """Two layers of the generation workload's shape (16 x 8 = 128 units), 4 steps: layer 0 puts 3
+    of its 512 new tokens on the fine grid, layer 1 none.  Per step j the decode reads every record
+    of T0 + j tokens per unit plus the queries; the append reads k, v rows and the score and writes
+    one record per unit."""
+    w = synth.WORKLOADS["gen"]
+    U, steps = 128, 4
+    rec_hi, rec_lo = 120, 96  # L 8 and L 5 at G64 (see test_decode_and_quantize_bytes_by_hand)
+    nh0, nl0 = [U * 8192, U * 8192], [U * 24576, U * 24576]
+    nh1, nl1 = [nh0[0] + 3, nh0[1]], [nl0[0] + U * steps - 3, nl0[1] + U * steps]
+    nb = bench.gen_steps_bytes(w, nh0, nl0, nh1, nl1, steps)
+    q = 16 * 32 * 128 * 2
+    dec = 0.0
+    for j in range(1, steps + 1):
+        for layer, dh in ((0, 3), (1, 0)):
+            dec += (nh0[layer] + j * dh / steps) * rec_hi + (nl0[layer] + j * (U * steps - dh) / steps) * rec_lo + q
+    assert nb["decode"] == dec
+    app = 2 * steps * U * (128 * 2 * 2 + 4) + 3 * rec_hi + (2 * U * steps - 3) * rec_lo
+    assert nb["append"] == app and nb["total"] == dec + app
+
+
+# storage reduction against fp16 of the precision sweep's 45 points, from the closed form of the
+# physical bits per value worked out by hand:
+#   bits(p) = p B(L_hi) + (1 - p) B(L_lo) + 32/G + 1/256,  B(L) = 32 ceil(128/k(L)) / 128
+# with k(5, 6, 8, 16) = 13, 12, 10, 8 codes per word (10, 11, 13, 16 words: B = 2.5, 2.75, 3.25, 4),
+# ratio = 16 / bits(p), rounded to 3 decimals (one row per level pair, G = 32 / 64 / 128 per p).
+SWEEP_RATIOS = {
+    (6, 5): {0.0: (4.566, 5.326, 5.810), 0.25: (4.486, 5.218, 5.681), 0.5: (4.409, 5.114, 5.558),
+             0.75: (4.334, 5.013, 5.440), 1.0: (4.262, 4.917, 5.326)},
+    (8, 6): {0.0: (4.262, 4.917, 5.326), 0.25: (4.125, 4.735, 5.114), 0.5: (3.996, 4.566, 4.917),
+             0.75: (3.875, 4.409, 4.735), 1.0: (3.761, 4.262, 4.566)},
+    (16, 8): {0.0: (3.761, 4.262, 4.566), 0.25: (3.602, 4.059, 4.334), 0.5: (3.457, 3.875, 4.125),
+              0.75: (3.322, 3.707, 3.935), 1.0: (3.198, 3.552, 3.761)},
+}
+
+
+def test_sweep_storage_ratios_equal_the_closed_form(semkv):
+    """The ratio the bench prints per sweep point (from the library's buffer sizes for the sweep's
+    cache: batch 8, 8 KV heads, T 32768) equals the closed form at all 45 points."""
+    w = synth.WORKLOADS["mistral_sweep"]
+    n = 0
+    for (Lh, Ll), rows in SWEEP_RATIOS.items():
+        for p, per_g in rows.items():
+            for G, want in zip((32, 64, 128), per_g):
+                got = bench.storage_ratio(128, G, Lh, Ll, p, w.T, B=w.B, H=w.H)
+                assert round(got, 3) == want, (Lh, Ll, p, G, got, want)
+                n += 1
+    assert n == 45 == len(synth.SWEEP_PAIRS) * len(synth.SWEEP_P) * len(synth.SWEEP_G)

@@ -143,3 +143,30 @@ def test_workspace_bytes_cover_the_split_partials(semkv):
     units, g, D = 16, 4, 128
     per_split = units * g * (D + 2) * 4
     assert n % per_split == 0 and 2 <= n // per_split <= 2 + 8  # at least one split per segment
+
+
+def test_capacities_by_hand(semkv):
+    """semkv_capacities: floor(p T) in double from the binary32 p, each segment rounded up to whole
+    128-slot tiles, T_cap to whole 32-token bitmap words."""
+    assert semkv.semkv_capacities(32768, 0.25) == (8192, 8192, 24576, 32768)
+    assert semkv.semkv_capacities(32768, 0.25, extra=300) == (8192, 8576, 24960, 33088)
+    assert semkv.semkv_capacities(1000, 0.3, window=16, extra=1) == (300, 384, 768, 1024)
+    # 0.1 as binary32 is 0.100000001490116..., so floor(p * 10) = 1 (and not 0.99999...)
+    assert semkv.semkv_capacities(10, 0.1)[0] == 1
+    assert semkv.semkv_capacities(0, 0.5) == (0, 0, 0, 0)
+    assert semkv.semkv_capacities(7, 1.0, window=100) == (7, 128, 0, 32)
+    for bad in ((-1, 0.5, 0, 0), (10, 1.5, 0, 0), (10, -0.1, 0, 0), (10, 0.5, -1, 0), (10, 0.5, 0, -1),
+                (2 ** 31 - 1, 0.5, 0, 2 ** 30)):
+        with pytest.raises(semkv.SemkvError) as e:
+            semkv.semkv_capacities(*bad)
+        assert e.value.code == semkv._lib.SEMKV_ERR_INVALID_ARG, bad
+
+
+def test_capacities_match_the_oracle_count(semkv, orc):
+    import numpy as np
+
+    r = np.random.default_rng(0)
+    for _ in range(200):
+        T = int(r.integers(0, 200000))
+        p = float(np.float32(r.random()))
+        assert semkv.semkv_capacities(T, p)[0] == orc.n_hi(p, T)

@@ -437,6 +437,41 @@ def test_attention_one_hot_and_uniform_logits(orc):
     assert not o.any()
 
 
+@pytest.mark.parametrize("T,g", [(1, 4), (100, 4), (513, 8), (4096, 4)])
+def test_attention_f32_matches_torch_sdpa_in_fp32(orc, T, g):
+    """The fp32-accumulate attention (the timed CPU variant) against torch's fp32 SDPA, within the
+    rounding of binary32 sums over T terms."""
+    import torch
+
+    r = np.random.default_rng(T + 1)
+    D = 128
+    q = r.standard_normal((g, D)).astype(np.float16)
+    Kh = (r.standard_normal((T, D)) * 2).astype(np.float32)
+    Vh = r.standard_normal((T, D)).astype(np.float32)
+    got = orc.attention_f32(q.view(np.uint16), Kh, Vh, float(np.float32(1 / math.sqrt(D))))
+    assert got.dtype == np.float32
+    qt = torch.from_numpy(q.astype(np.float32))[None, :, None, :]
+    kt = torch.from_numpy(Kh)[None, None].expand(1, g, -1, -1)
+    vt = torch.from_numpy(Vh)[None, None].expand(1, g, -1, -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=float(np.float32(1 / math.sqrt(D))))
+    assert np.allclose(got, ref[0, :, 0].numpy(), rtol=1e-4, atol=2e-5)
+
+
+def test_attention_f32_one_hot_uniform_and_empty(orc):
+    D, T = 128, 50
+    r = np.random.default_rng(2)
+    Vh = r.standard_normal((T, D)).astype(np.float32)
+    q = np.zeros((1, D), np.float16)
+    q[0, 0] = 1.0
+    Kh = np.zeros((T, D), np.float32)
+    Kh[17, 0] = 1e4
+    assert np.array_equal(orc.attention_f32(q.view(np.uint16), Kh, Vh, 1.0)[0], Vh[17])
+    o = orc.attention_f32(q.view(np.uint16), np.zeros((T, D), np.float32), Vh, 1.0)
+    assert np.allclose(o[0], Vh.astype(np.float64).mean(0), atol=1e-6)
+    o = orc.attention_f32(q.view(np.uint16), np.zeros((0, D), np.float32), np.zeros((0, D), np.float32), 1.0)
+    assert not o.any()
+
+
 def test_layout_as_documented(orc):
     """Read the oracle's buffers with plain indexing per the documented layout and check each
     digit against a one-group quantization of that token's row (K: row words; V: column words)."""

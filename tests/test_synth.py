@@ -38,3 +38,28 @@ def test_p_for_ratio_kv_rejects_bad_arguments(semkv):
         with pytest.raises(semkv.SemkvError) as e:
             semkv.semkv_p_for_ratio_kv(*args)
         assert e.value.code == code, args
+
+
+def test_generated_tokens_share_the_prefill_channel_scales():
+    """The GPU-path generator (run here on the CPU device) draws generated k, v with the prefill's
+    per-channel scales: divided by those scales, both the prefill rows and the generated rows have
+    unit spread in every channel, while the raw channels do not."""
+    import torch
+
+    w = synth.WORKLOADS["llama8b_1L"]
+    d = synth.layer_gpu(w, 5, layer=2, device="cpu", T=4096)
+    sk, sv = synth.prefill_channel_scales_gpu(w, 5, layer=2, device="cpu")
+    gen = synth.gen_steps_gpu(w, d["K"], 5, 2, steps=4096, device="cpu")
+    assert gen["k"].shape == (4096, 1, 8, 128) and gen["k"].dtype == torch.float16
+    for x, s in ((d["K"].float(), sk), (d["V"].float(), sv)):
+        r = (x / s).std(dim=2)  # [B][H][D] over the prefill tokens
+        assert torch.allclose(r, torch.ones_like(r), atol=0.08)
+    for x, s in ((gen["k"].float(), sk.reshape(1, 1, 8, 128)), (gen["v"].float(), sv.reshape(1, 1, 8, 128))):
+        r = (x / s).std(dim=0)  # over the generated tokens
+        assert torch.allclose(r, torch.ones_like(r), atol=0.08)
+        raw = x.std(dim=0)
+        assert raw.max() / raw.min() > 2.0  # the channel scales are really there
+
+
+def test_outlier_workload_has_no_channel_scales():
+    assert synth.prefill_channel_scales_gpu(synth.WORKLOADS["tiny"], 0, device="cpu") == (None, None)
