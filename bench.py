@@ -889,7 +889,7 @@ def run_semkv(args):
         ms_step = r["total_ms"] / K
         layer_ms = ms_step / r["layers"]
         layer_bytes = r["step_bytes"] / r["layers"]
-        dom_name = "semkv_append_decode per layer (k_decode_tc hi + lo grids, k_decode_merge)"
+        dom_name = "semkv_append_decode per layer (k_decode_i8 hi + lo grids, k_decode_merge)"
         ach = layer_bytes / (layer_ms * 1e-3) / 1e9
         per_kernel = {
             "append_decode_layer": {"ms": layer_ms, "gbs": ach},
@@ -913,7 +913,7 @@ def run_semkv(args):
         value = weak_scaling_value(gpu.world, r["bytes_per_step"], K, max_over_ranks(r["ms_per_step"] * K, gpu.dist,
                                                                                       "cuda"))
         ms_step = r["ms_per_step"]
-        dom_name = "semkv_decode_attention per layer (k_decode_tc hi + lo grids, k_decode_merge)"
+        dom_name = "semkv_decode_attention per layer (k_decode_i8 hi + lo grids, k_decode_merge)"
         ach = r["gbs"]
         dec_gbs = r["gbs"]
         launches = r["launches_per_step"] * K
@@ -928,7 +928,7 @@ def run_semkv(args):
         dom = max(("select", "quantize", "append_decode"), key=lambda k: per_kernel[k]["ms"])
         dom_name = {"select": "semkv_assign_precision (k_select_cluster)",
                     "quantize": "semkv_quantize_pack (k_quantize_fast)",
-                    "append_decode": "semkv_append_decode (k_decode_tc x 2 + k_decode_merge)"}[dom]
+                    "append_decode": "semkv_append_decode (k_decode_i8 x 2 + k_decode_merge)"}[dom]
         ach = per_kernel[dom]["gbs"]
         dec_gbs = per_kernel["decode_l2_cold"]["gbs"]
         launches = (2 + DECODE_KERNELS_PER_CALL) * K
@@ -949,8 +949,9 @@ def run_semkv(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": gpu.world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "decode: fp16 tensor-core operands (codes, queries, P' = p s_V as two fp16 limbs), fp32 "
-                 "accumulate and softmax; quantize: binary32 IEEE",
+        "dtype": "decode: u8 codes x s8/u8 fixed-point limbs on the integer tensor cores (queries as three s8 "
+                 "limbs of a 20-bit image, P' = p s_V as three u8 limbs of a 22-bit image per tile), s32 "
+                 "accumulate, f32 softmax; quantize: binary32 IEEE",
         "data": "synthetic",
         "config": dict(workload_config(w, gpu.world), **cfg_extra),
         "per_kernel": per_kernel,

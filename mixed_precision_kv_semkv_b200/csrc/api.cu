@@ -86,6 +86,53 @@ void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
     *ns_lo = pick(tl);
 }
 
+// How a decode of this shape runs on the current device.  The integer tensor-core decode (when it
+// covers both segments): one CTA per SM, the SMs shared by the segments in proportion to their
+// work (capacity tiles x a per-tile cost that grows with the words per row: the decode issues
+// instructions faster than HBM delivers bytes), at least 8 tiles per CTA, and
+// 4 * ctas / units + 2 partial slots per unit and segment (the most workers that can touch one
+// unit).  Otherwise the split-K factors of the other decode kernels.
+struct DecodePlan {
+    bool i8;
+    int ctas_hi, ctas_lo, slots_hi, slots_lo;  // i8
+    int ns_hi, ns_lo;                          // otherwise
+    int slots() const { return i8 ? slots_hi + slots_lo : ns_hi + ns_lo; }
+};
+
+DecodePlan decode_plan(const semkv_cache_t* c)
+{
+    DecodePlan p = {};
+    const int g = c->Hq / c->H, units = c->B * c->H;
+    const bool kpc = c->k_per_channel != 0;
+    const int th = c->cap_hi / TILE, tl = c->cap_lo / TILE;
+    const bool hi_ok = th == 0 || decode_i8_supported(c->L_hi, level_v(*c, true), c->G, g, kpc);
+    const bool lo_ok = tl == 0 || decode_i8_supported(c->L_lo, level_v(*c, false), c->G, g, kpc);
+    if (hi_ok && lo_ok && th + tl > 0) {
+        p.i8 = true;
+        const int sms = sm_count();
+        const double bh = (double)th * (400 + 40 * words_row(c->L_hi)), bl = (double)tl * (400 + 40 * words_row(c->L_lo));
+        int ch = 0, cl = 0;
+        if (th && tl) {
+            ch = (int)std::lround(sms * bh / (bh + bl));
+            ch = ch < 1 ? 1 : (ch > sms - 1 ? sms - 1 : ch);
+            cl = sms - ch;
+        } else {
+            ch = th ? sms : 0;
+            cl = tl ? sms : 0;
+        }
+        const long long mh = ((long long)units * th + 7) / 8, ml = ((long long)units * tl + 7) / 8;
+        if (ch > mh) ch = (int)mh;
+        if (cl > ml) cl = (int)ml;
+        p.ctas_hi = ch;
+        p.ctas_lo = cl;
+        p.slots_hi = ch ? 4 * ch / units + 2 : 0;
+        p.slots_lo = cl ? 4 * cl / units + 2 : 0;
+    } else {
+        decode_splits(c, &p.ns_hi, &p.ns_lo);
+    }
+    return p;
+}
+
 SegView seg_view(const semkv_cache_t* c, bool hi)
 {
     SegView s;
@@ -131,11 +178,20 @@ static int decode_impl(const semkv_cache_t* c, const uint16_t* q, float softmax_
 {
     const int r = decode_args(c, q, softmax_scale, out, workspace, workspace_bytes);
     if (r != SEMKV_OK) return r;
-    int nh, nl;
-    decode_splits(c, &nh, &nl);
+    const DecodePlan plan = decode_plan(c);
     const int units = c->B * c->H, g = c->Hq / c->H;
     const float scale_log2 = softmax_scale * 1.4426950408889634f;
     float* ws = static_cast<float*>(workspace);
+    if (plan.i8) {
+        const SegView hs = seg_view(c, true), ls = seg_view(c, false);
+        launch_decode_i8(hs, q, units, c->H, g, c->G, scale_log2, plan.ctas_hi, plan.slots_hi, 0, plan.slots(), ws,
+                         c->status, false, app, st);
+        launch_decode_i8(ls, q, units, c->H, g, c->G, scale_log2, plan.ctas_lo, plan.slots_lo, plan.slots_hi,
+                         plan.slots(), ws, c->status, plan.ctas_hi > 0, app, st);
+        launch_decode_merge(ws, units, c->H, g, c->D, plan.slots(), out, app, st);
+        return launch_status();
+    }
+    const int nh = plan.ns_hi, nl = plan.ns_lo;
     bool dependent = false;
     for (int hi = 1; hi >= 0; --hi) {
         const SegView sv = seg_view(c, hi != 0);
@@ -235,9 +291,7 @@ int semkv_workspace_bytes(const semkv_cache_t* c, size_t* bytes)
     int r = validate_shape(c);
     if (r != SEMKV_OK) return r;
     if (!bytes) return SEMKV_ERR_INVALID_ARG;
-    int nh, nl;
-    decode_splits(c, &nh, &nl);
-    *bytes = (size_t)c->B * c->H * (size_t)(nh + nl) * (c->Hq / c->H) * (c->D + 2) * sizeof(float);
+    *bytes = (size_t)c->B * c->H * (size_t)decode_plan(c).slots() * (c->Hq / c->H) * (c->D + 2) * sizeof(float);
     return SEMKV_OK;
 }
 
@@ -307,8 +361,8 @@ int semkv_append_decode(const semkv_cache_t* c, const uint16_t* k, const uint16_
     if (r != SEMKV_OK) return r;
     if (!k || !v || !score) return SEMKV_ERR_INVALID_ARG;
     const int g = c->Hq / c->H;
-    if (!decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g, c->k_per_channel != 0) ||
-        !decode_tc_supported(c->L_lo, level_v(*c, false), c->G, g, c->k_per_channel != 0)) {
+    if (!decode_plan(c).i8 && (!decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g, c->k_per_channel != 0) ||
+                               !decode_tc_supported(c->L_lo, level_v(*c, false), c->G, g, c->k_per_channel != 0))) {
         // shapes the fused path does not cover: the two calls, in order
         launch_append(*c, k, v, score, -1.0f, (cudaStream_t)stream);
         r = launch_status();

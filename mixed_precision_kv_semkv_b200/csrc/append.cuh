@@ -15,16 +15,19 @@
 
 namespace semkv {
 
-// Row of the new token of unit u (grid hi; nh, nl: the unit's counts before it; kx, vx: this
-// thread's channel of the new K and V rows).  Every thread of the CTA calls it; returns true on
-// every thread if a K or V value of the row is not finite.
-__device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool hi, int nh, int nl, float kx, float vx)
+// Row of the new token of unit u (grid hi; nh, nl: the unit's counts before it; kx, vx: channel d
+// of the new K and V rows), written by 128 threads (d = 0..127) that synchronize with sync() and
+// OR a flag over themselves with sync_or(flag).  kc: 160 ints of shared scratch; gmn, gmx: per-warp
+// partial extrema of groups wider than a warp.  Returns true on every thread if a K or V value of
+// the row is not finite.
+template <class Sync, class SyncOr>
+__device__ __forceinline__ bool append_row_impl(const semkv_cache_t& c, int u, bool hi, int nh, int nl, float kx,
+                                                float vx, int d, int* kc, float (*gmn)[4], float (*gmx)[4], Sync sync,
+                                                SyncOr sync_or)
 {
     constexpr int D = 128;
-    const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+    const int lane = d & 31, warp = d >> 5;
     const int G = c.G, NG = D / G;
-    __shared__ int kc[D + 32];
-    __shared__ float gmn[2][4], gmx[2][4];  // per-warp partial extrema of groups wider than a warp
     const int slot = hi ? nh : nl;
     const int L = hi ? c.L_hi : c.L_lo, Lv = level_v(c, hi);
     const int k = radix_k(L), kv = radix_k(Lv);
@@ -54,7 +57,7 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
             gmn[1][warp] = vmn;
             gmx[1][warp] = vmx;
         }
-        __syncthreads();
+        sync();
         const int w0 = (d / G) * (G / 32);
         for (int i = 0; i < G / 32; ++i) {
             kmn = fminf(kmn, gmn[0][w0 + i]);
@@ -81,7 +84,7 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
     }
     const uint32_t cv = (uint32_t)quant_code(vx, h2f(vz16), h2f(vs16), Lv);
     const bool bad = !isfinite(kx) || !isfinite(vx);
-    __syncthreads();
+    sync();
 
     if (d < WK) {  // K word d: Horner over its k digits, top digit first
         uint32_t w = 0u;
@@ -101,7 +104,17 @@ __device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool h
             atomicAdd(p, cv * pw);
         }
     }
-    return __syncthreads_or(bad) != 0;
+    return sync_or(bad);
+}
+
+// append_row_impl by every thread of a 128-thread CTA (thread d = channel d)
+__device__ __forceinline__ bool append_row(const semkv_cache_t& c, int u, bool hi, int nh, int nl, float kx, float vx)
+{
+    __shared__ int kc[128 + 32];
+    __shared__ float gmn[2][4], gmx[2][4];
+    return append_row_impl(
+        c, u, hi, nh, nl, kx, vx, (int)threadIdx.x, kc, gmn, gmx, [] { __syncthreads(); },
+        [](bool b) { return __syncthreads_or(b) != 0; });
 }
 
 // The unit's bookkeeping after its new token went in (one thread): bitmap bit, rank directory,

@@ -73,6 +73,15 @@ void launch_decode_tc(const SegView& seg, const uint16_t* q, int units, int H, i
                       int nsplit, int split_off, int nsplit_total, float* ws, int32_t* status, bool dependent,
                       const AppendIn& app, cudaStream_t st);
 
+// integer tensor-core decode (decode_i8.cu): one CTA of 4 warpgroups per SM; `ctas` CTAs share the
+// segment's units x tiles_cap tiles in contiguous ranges; unit u's partial states go to slots
+// [slot_off, slot_off + slots) of its slots_total.  Covers equal K/V level counts in {4, 5, 6, 8,
+// 16}, per-token K grids, and (g, groups) in {(2,1), (2,2), (4,1), (4,2), (8,1)}.
+bool decode_i8_supported(int Lk, int Lv, int G, int g, bool kpc);
+void launch_decode_i8(const SegView& seg, const uint16_t* q, int units, int H, int g, int G, float scale_log2,
+                      int ctas, int slots, int slot_off, int slots_total, float* ws, int32_t* status, bool dependent,
+                      const AppendIn& app, cudaStream_t st);
+
 void launch_dequantize(const semkv_cache_t& c, int T, float* K, float* V, cudaStream_t st);
 
 }  // namespace semkv

@@ -62,6 +62,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase)
     return false;
 }
 
+// One non-blocking test of the phase parity.
+__device__ __forceinline__ bool mbar_test_now(uint64_t* bar, uint32_t phase)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the barrier's phase parity by polling (a few tests back to back, then short sleeps);
+// false after about 2^25 tests (well over a second).
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t phase)
+{
+    for (uint32_t i = 0; i < (1u << 25); ++i) {
+        if (mbar_test_now(bar, phase)) return true;
+        if (i >= 8) __nanosleep(32);
+    }
+    return false;
+}
+
 // 32-bit loads from a shared-memory address (as returned by smem_u32).  lds_u32_after_wait is
 // ordered after earlier volatile asm (an mbarrier wait that made the data visible); lds_u32 may be
 // scheduled freely and is for data written before the CTA's set-up barrier (tables).
@@ -220,6 +245,106 @@ __device__ __forceinline__ float ex2_approx(float x)
 {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+}  // namespace semkv
+
+namespace semkv {
+
+// ------------------------------------------------------------------ integer tensor cores, wide TMEM moves
+
+// D[tmem] (+)= A[tmem] x B[smem desc], kind::i8 (8-bit integer operands, s32 accumulators), issued
+// by one thread.
+__device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// Instruction descriptor, kind::i8: D s32, A u8 (K-major), B u8 or s8, B K-major or MN-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_i8_s32(int M, int N, bool b_signed, bool b_mn_major)
+{
+    return (2u << 4)                               // D format: s32
+           | (0u << 7)                             // A: unsigned 8-bit
+           | ((b_signed ? 1u : 0u) << 10)          // B: signed or unsigned 8-bit
+           | (0u << 15)                            // A K-major
+           | ((b_mn_major ? 1u : 0u) << 16)        // B major
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane <- r[0..31]
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// r[0..31] <- 32 consecutive 32-bit columns of this thread's TMEM lane (complete after tc_wait_ld)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// N (8, 16 or 32) consecutive columns of this thread's TMEM lane into r[0..N)
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[32])
+{
+    if constexpr (N == 32) {
+        tmem_ld32(taddr, r);
+    } else if constexpr (N == 16) {
+        tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+    } else {
+        static_assert(N == 8, "8, 16 or 32 columns");
+        tmem_ld8(taddr, *reinterpret_cast<uint32_t(*)[8]>(&r[0]));
+    }
+}
+
+// 16 bytes to shared memory
+__device__ __forceinline__ void sts128(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// named barrier `id` over `count` threads that also ORs a predicate over them
+__device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.or.pred q, %1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(count), "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
+
+// maximum of an unsigned value over the 32 lanes of a warp
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v)
+{
+    uint32_t r;
+    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
     return r;
 }
 
