@@ -203,6 +203,18 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
         }
         const int tiles_n = min(ceil_div(n, TILE), T);
         const int e = min(b, tiles_n);  // tiles [a, e) hold tokens
+        const int nt = e > a ? e - a : 0;
+        // the first two tiles' copies overlap the query set-up, unless the appended token is written
+        // into one of them first
+        const bool fetch_early = !(APP && app_tile >= a && app_tile < a + 2);
+        auto fetch_first = [&] {
+            if (t == 0 && nt > 0) {
+                fence_async_smem();
+                fetch(u, a, fetched);
+                if (nt > 1) fetch(u, a + 1, fetched + 1);
+            }
+        };
+        if (fetch_early) fetch_first();
 
         // ---------------- the unit's queries: B_Q limbs, group sums, fixed-point scale
         if (u != cur_unit) {
@@ -299,7 +311,7 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
             for (int g2 = 0; g2 < NG; ++g2) zacc[g2][h] = 0.f;
         }
         float psa = 0.f;  // 2^-a of channel t's group for the tile whose p.V is in flight
-        const int nt = e > a ? e - a : 0;
+        if (!fetch_early) fetch_first();
 
         // D_V of the finished p.V -> O (after waiting for it)
         auto take_pv = [&] {
@@ -334,11 +346,6 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
         };
 
         if (nt > 0) {
-            if (t == 0) {
-                fence_async_smem();
-                fetch(u, a, fetched);
-                if (nt > 1) fetch(u, a + 1, fetched + 1);
-            }
             wait_stage(fetched);
             unpack_to_tmem(smem_u32(wsm + (fetched & 1u) * C::STAGE + C::ST_K), lane_base + C::COL_AK);
             issue_qk();
@@ -433,13 +440,11 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
                 for (int nb = 0; nb < NV / 16; ++nb)
                     sts128(bp_addr + (uint32_t)((vpos >> 3) * C::LBO_P + nb * C::SBO_P + (vpos & 7) * 16),
                            wd[4 * nb], wd[4 * nb + 1], wd[4 * nb + 2], wd[4 * nb + 3]);
-                // ---- p.V
+                // ---- p.V (q.k is issued by warp 0, p.V and the copies by warp 2)
                 tc_wait_st();
                 fence_async_smem();
                 tc_fence_before();
                 wg_sync();
-                // the single-thread duties go to different warps: q.k to warp 0, p.V to warp 2,
-                // the copies to warp 1
                 if (t == 64) {
                     tc_fence_after();
 #pragma unroll
@@ -447,12 +452,9 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
                         mma_ts_i8(tmem + C::COL_DV, tmem + C::COL_AV + 8 * s,
                                   smem_desc(bp_addr + s * 4 * C::LBO_P, C::LBO_P, C::SBO_P), C::IDESC_PV, s > 0);
                     mma_commit(&bar[3]);
-                }
-                // every thread has read this stage (K codes last iteration, V codes and scales
-                // above): refill it two tiles ahead
-                if (t == 32 && i + 2 < nt) {
-                    fence_async_smem();
-                    fetch(u, tile + 2, nf + 2);
+                    // every thread has read this stage (K codes last iteration, V codes and scales
+                    // above): refill it two tiles ahead
+                    if (i + 2 < nt) fetch(u, tile + 2, nf + 2);
                 }
                 // ---- next tile's K codes and q.k, overlapping this p.V
                 if (i + 1 < nt) {
