@@ -414,10 +414,14 @@ class Gpu:
             self.dist = dist
         self.stream = torch.cuda.current_stream()
         self.flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+        self.flush_sink = torch.empty((), dtype=torch.int64, device="cuda")
         self.seed = rank_seed(self.rank)
 
     def flush(self):
+        """Evict the L2: write 512 MB, then read back the first half of it, so that the next kernel
+        finds a cold L2 holding no dirty lines (it does not pay for writing back the flush)."""
         self.flush_buf.zero_()
+        self.torch.sum(self.flush_buf[: L2_FLUSH_BYTES // 8], dim=0, out=self.flush_sink)
 
     def event(self):
         return self.torch.cuda.Event(enable_timing=True)
@@ -480,11 +484,15 @@ def counts(caches):
     return nh, nl
 
 
-def prefill_layer(gpu, w, cache, d, T):
+def prefill_layer(gpu, w, cache, d, T, warm: bool = False):
     """semkv_assign_precision then semkv_quantize_pack of one layer, each timed after an L2 flush;
-    returns (select ms, quantize ms)."""
+    returns (select ms, quantize ms).  With `warm`, both calls run once untimed first (they write
+    the same cache again): the first launch of a kernel loads its module, which must not be timed."""
     from mixed_precision_kv_semkv_b200 import semkv_assign_precision, semkv_quantize_pack
 
+    if warm:
+        semkv_assign_precision(cache, d["scores"], T, w.p)
+        semkv_quantize_pack(cache, d["K"], d["V"], T)
     gpu.flush()
     e = [gpu.event() for _ in range(3)]
     e[0].record(gpu.stream)
@@ -522,7 +530,7 @@ def run_gen(gpu, w, K: int, W: int, want_e2e: bool):
     for layer in range(layers):
         d = synth.layer_gpu(w, gpu.seed, layer=layer)
         cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, T, w.p, extra=S)
-        ts, tq = prefill_layer(gpu, w, cache, d, T)
+        ts, tq = prefill_layer(gpu, w, cache, d, T, warm=layer == 0)
         t_sel.append(ts)
         t_q.append(tq)
         gen = synth.gen_steps_gpu(w, d["K"], gpu.seed, layer, S)
@@ -656,7 +664,7 @@ def run_decode_layers(gpu, w, K: int, W: int):
     for layer in range(layers):
         d = synth.layer_gpu(w, gpu.seed, layer=layer)
         cache = SemkvCache.for_prefill(w.B, w.H, w.Hq, w.G, w.L_hi, w.L_lo, w.T, w.p)
-        ts, tq = prefill_layer(gpu, w, cache, d, w.T)
+        ts, tq = prefill_layer(gpu, w, cache, d, w.T, warm=layer == 0)
         t_sel.append(ts)
         t_q.append(tq)
         caches.append(cache)
@@ -817,7 +825,7 @@ def run_one_layer(gpu, w, K: int, W: int, variants: bool = True):
     res = {"ms_per_step": step_ms, "gbs": step_bytes / (step_ms * 1e-3) / 1e9, "step_bytes": step_bytes,
            "per_kernel": per_kernel, "quantize_frac": per_kernel["quantize"]["gbs"] / peak,
            "decode_frac": per_kernel["decode_l2_cold"]["gbs"] / peak,
-           "timing": "step = one CUDA graph of select, quantize and append_decode, L2 flushed (512 MB write) "
+           "timing": "step = one CUDA graph of select, quantize and append_decode, L2 flushed (512 MB written, 256 MB of it read back) "
                      "between steps; per_kernel = each call from a graph of its own, L2 flushed before it"}
     del graphs, step_graph
     torch.cuda.empty_cache()
@@ -933,7 +941,7 @@ def run_semkv(args):
         dec_gbs = per_kernel["decode_l2_cold"]["gbs"]
         launches = (2 + DECODE_KERNELS_PER_CALL) * K
         clocks, e2e, traffic, steps_ms = {}, None, captured_traffic(w.name, dom), None
-        cfg_extra = {"l2": "flushed between steps (512 MB write)", "timing": r["timing"]}
+        cfg_extra = {"l2": "flushed between steps (512 MB written, then 256 MB of it read back: a cold L2 with no dirty lines)", "timing": r["timing"]}
 
     if w.name == "gen" and not (args.no_extras or args.profile):
         extras["llama8b_32L"] = run_decode_layers(gpu, synth.WORKLOADS["llama8b_32L"], min(K, 50), W)

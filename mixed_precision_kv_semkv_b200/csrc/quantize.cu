@@ -294,17 +294,23 @@ struct GroupGrid {
     bool finite;
 };
 
-// CLIP: the clipped-range grid (clip < 1); otherwise the plain min/max grid
-template <int L, int G, bool CLIP>
-__device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2], float clip)
+// running minimum and maximum (as binary16 pairs) over N pairs of values
+template <int N>
+__device__ __forceinline__ void minmax_pairs(const uint32_t (&h)[N], __half2& mn2, __half2& mx2, bool first)
 {
-    __half2 mn2 = *reinterpret_cast<const __half2*>(&h[0]), mx2 = mn2;
+    if (first) mn2 = mx2 = *reinterpret_cast<const __half2*>(&h[0]);
 #pragma unroll
-    for (int i = 1; i < G / 2; ++i) {
+    for (int i = first ? 1 : 0; i < N; ++i) {
         const __half2 v = *reinterpret_cast<const __half2*>(&h[i]);
         mn2 = __hmin2_nan(mn2, v);
         mx2 = __hmax2_nan(mx2, v);
     }
+}
+
+// CLIP: the clipped-range grid (clip < 1); otherwise the plain min/max grid
+template <int L, bool CLIP>
+__device__ __forceinline__ GroupGrid group_grid(__half2 mn2, __half2 mx2, float clip)
+{
     const float mn = __half2float(__hmin_nan(__low2half(mn2), __high2half(mn2)));
     const float mx = __half2float(__hmax_nan(__low2half(mx2), __high2half(mx2)));
     GroupGrid g;
@@ -327,16 +333,16 @@ __device__ __forceinline__ GroupGrid group_grid(const uint32_t (&h)[G / 2], floa
     return g;
 }
 
-// codes (as magic-offset fp32 bits) of one group's G values, two at a time, handed to `sink(i, bits)`.
-// CLIP: values below the zero are raised to it first (exact: the zero is a binary16) and the
-// quotient is clamped to L - 1 before the rounding add, so codes are clamp(rint(q), 0, L - 1) and
-// the add stays in its exact range.
-template <int L, int G, bool CLIP, typename Sink>
-__device__ __forceinline__ void group_codes(const uint32_t (&h)[G / 2], const GroupGrid& g, Sink&& sink)
+// codes (as magic-offset fp32 bits) of N values (N / 2 pairs), two at a time, handed to
+// `sink(i, bits)`.  CLIP: values below the zero are raised to it first (exact: the zero is a
+// binary16) and the quotient is clamped to L - 1 before the rounding add, so codes are
+// clamp(rint(q), 0, L - 1) and the add stays in its exact range.
+template <int L, int N, bool CLIP, typename Sink>
+__device__ __forceinline__ void group_codes(const uint32_t (&h)[N / 2], const GroupGrid& g, Sink&& sink)
 {
     const uint64_t m2 = f2_pack(12582912.0f, 12582912.0f);
 #pragma unroll
-    for (int i = 0; i < G / 2; ++i) {
+    for (int i = 0; i < N / 2; ++i) {
         __half2 hv = *reinterpret_cast<const __half2*>(&h[i]);
         if constexpr (CLIP) hv = __hmax2(hv, *reinterpret_cast<const __half2*>(&g.zh2));
         const float2 xf = __half22float2(hv);
@@ -363,6 +369,41 @@ __device__ __forceinline__ void group_codes(const uint32_t (&h)[G / 2], const Gr
     }
 }
 
+// One group of G values of a row in shared memory: its grid, and its codes handed to
+// `sink(i, bits)` (i = the value's index in the group).  Groups of more than 64 values are read
+// twice in chunks of 64 (range, then codes), so that a chunk, not the group, is held in registers;
+// the last chunk's codes come first.
+template <int L, int G, bool CLIP, typename Sink>
+__device__ __forceinline__ GroupGrid quantize_group(const uint16_t* src, float clip, Sink&& sink)
+{
+    constexpr int CH = G > 64 ? 64 : G, NCH = G / CH;
+    uint32_t h[CH / 2];
+    auto load = [&](int c) {
+#pragma unroll
+        for (int i = 0; i < CH / 8; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + c * CH + 8 * i);
+            h[4 * i] = v.x;
+            h[4 * i + 1] = v.y;
+            h[4 * i + 2] = v.z;
+            h[4 * i + 3] = v.w;
+        }
+    };
+    __half2 mn2, mx2;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        load(c);
+        minmax_pairs<CH / 2>(h, mn2, mx2, c == 0);
+    }
+    const GroupGrid g = group_grid<L, CLIP>(mn2, mx2, clip);
+    group_codes<L, CH, CLIP>(h, g, [&](int i, uint32_t bits) { sink((NCH - 1) * CH + i, bits); });
+#pragma unroll
+    for (int c = 0; c + 1 < NCH; ++c) {
+        load(c);
+        group_codes<L, CH, CLIP>(h, g, [&](int i, uint32_t bits) { sink(c * CH + i, bits); });
+    }
+    return g;
+}
+
 // K rows of a tile: thread `tid` quantizes row tid and packs it along the channels
 template <int L, int G, bool CLIP>
 __device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw, uint32_t* kz, int tid, bool& bad,
@@ -376,22 +417,12 @@ __device__ __forceinline__ void quantize_k_rows(const uint16_t* Ks, uint32_t* kw
         const uint16_t* row = Ks + tid * QROW;
 #pragma unroll
         for (int grp = 0; grp < NG; ++grp) {
-            uint32_t h[G / 2];
-#pragma unroll
-            for (int i = 0; i < G / 8; ++i) {
-                const uint4 v = *reinterpret_cast<const uint4*>(row + grp * G + 8 * i);
-                h[4 * i] = v.x;
-                h[4 * i + 1] = v.y;
-                h[4 * i + 2] = v.z;
-                h[4 * i + 3] = v.w;
-            }
-            const GroupGrid g = group_grid<L, G, CLIP>(h, clip);
-            bad |= !g.finite;
-            kz[grp * TILE + tid] = g.packed;
-            group_codes<L, G, CLIP>(h, g, [&](int i, uint32_t bits) {
+            const GroupGrid g = quantize_group<L, G, CLIP>(row + grp * G, clip, [&](int i, uint32_t bits) {
                 const int d = grp * G + i;
                 w[d / k] += bits * upow(L, d % k);
             });
+            bad |= !g.finite;
+            kz[grp * TILE + tid] = g.packed;
         }
 #pragma unroll
         for (int j = 0; j < WK; ++j) {
@@ -468,24 +499,15 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
         uint32_t bytes[D / 4];
 #pragma unroll
         for (int grp = 0; grp < NG; ++grp) {
-            uint32_t h[G / 2];
-#pragma unroll
-            for (int i = 0; i < G / 8; ++i) {
-                const uint4 v = *reinterpret_cast<const uint4*>(row + grp * G + 8 * i);
-                h[4 * i] = v.x;
-                h[4 * i + 1] = v.y;
-                h[4 * i + 2] = v.z;
-                h[4 * i + 3] = v.w;
-            }
-            const GroupGrid g = group_grid<L, G, CLIP>(h, clip);
-            bad |= !g.finite;
-            packed[grp] = g.packed;
-            // the low byte of each magic sum is the code: byte i%4 of word i/4
-            group_codes<L, G, CLIP>(h, g, [&](int i, uint32_t b) {
+            // the low byte of each magic sum is the code: byte i%4 of word i/4 (a chunk of the
+            // group covers whole words)
+            const GroupGrid g = quantize_group<L, G, CLIP>(row + grp * G, clip, [&](int i, uint32_t b) {
                 const int c = grp * G + i;
                 constexpr uint32_t sel[4] = {0x3214u, 0x3240u, 0x3410u, 0x4210u};
                 bytes[c / 4] = (c % 4 == 0) ? (b & 0xffu) : __byte_perm(bytes[c / 4], b, sel[c % 4]);
             });
+            bad |= !g.finite;
+            packed[grp] = g.packed;
         }
 #pragma unroll
         for (int grp = 0; grp < NG; ++grp) vz[grp * TILE + tid] = packed[grp];
@@ -510,11 +532,10 @@ __device__ __forceinline__ void quantize_v_rows(uint16_t* Vs, uint32_t* vw, uint
 
 // LH, LL: level counts of the K codes of the two segments; LHV, LLV: of the V codes; CLIP: the
 // clipped-range grid with ratio `clip`; KPC: K on the per-channel grids of seg.kc
-template <int LH, int LL, int LHV, int LLV, int G, bool CLIP, bool KPC = false>
-__global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
-                                                        const uint16_t* __restrict__ V,
-                                                        int T, float clip,
-                                                        int32_t* __restrict__ status)
+template <int LH, int LL, int LHV, int LLV, int G, bool CLIP, bool KPC>
+__device__ __forceinline__ void quantize_fast_body(const QuantSeg& hi, const QuantSeg& lo,
+                                                   const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
+                                                   int T, float clip, int32_t* __restrict__ status)
 {
     constexpr int D = 128, NG = D / G;
     // order: the L_lo segment's K rows, its V rows, then the L_hi segment's K rows and V rows
@@ -580,6 +601,32 @@ __global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo,
     if (bad && tid < n - s0) atomicOr(status, SEMKV_STATUS_NONFINITE_KV);
 }
 
+template <int LH, int LL, int LHV, int LLV, int G, bool CLIP, bool KPC>
+__global__ void __launch_bounds__(128) k_quantize_fast(QuantSeg hi, QuantSeg lo, const uint16_t* __restrict__ K,
+                                                        const uint16_t* __restrict__ V, int T, float clip,
+                                                        int32_t* __restrict__ status)
+{
+    quantize_fast_body<LH, LL, LHV, LLV, G, CLIP, KPC>(hi, lo, K, V, T, clip, status);
+}
+
+// groups of 128: registers capped for 6 CTAs per SM (the compiler would otherwise take ~100,
+// leaving 4 CTAs and fewer rows in flight; the cap costs a few spilled bytes)
+template <int LH, int LL, int LHV, int LLV, int G, bool CLIP, bool KPC>
+__global__ void __launch_bounds__(128, 6) k_quantize_fast_wide(QuantSeg hi, QuantSeg lo,
+                                                                const uint16_t* __restrict__ K,
+                                                                const uint16_t* __restrict__ V, int T, float clip,
+                                                                int32_t* __restrict__ status)
+{
+    quantize_fast_body<LH, LL, LHV, LLV, G, CLIP, KPC>(hi, lo, K, V, T, clip, status);
+}
+
+template <int LH, int LL, int LHV, int LLV, int G, bool CLIP, bool KPC = false>
+static auto quantize_fast_kernel()
+{
+    if constexpr (G > 64) return k_quantize_fast_wide<LH, LL, LHV, LLV, G, CLIP, KPC>;
+    else return k_quantize_fast<LH, LL, LHV, LLV, G, CLIP, KPC>;
+}
+
 static size_t quantize_smem(int G)
 {
     return (size_t)2 * TILE * QROW * 2 + (size_t)TILE * (128 / G) * 16 + 128 * 16;
@@ -620,7 +667,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
 #define SEMKV_QK(LH, LL, GG)                                                                                  \
     if (kc && !clipped && shi.L == LH && slo.L == LL && shi.Lv == LH && slo.Lv == LL && G == GG) {            \
         const size_t sm = (size_t)TILE * QROW * 2 + 64 * sizeof(KpcPair);                                     \
-        const auto kern = k_quantize_fast<LH, LL, LH, LL, GG, false, true>;                                   \
+        const auto kern = quantize_fast_kernel<LH, LL, LH, LL, GG, false, true>();                            \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);                    \
         kern<<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, clip, status);                                       \
         return;                                                                                               \
@@ -631,7 +678,7 @@ void launch_quantize(const SegView& shi, const SegView& slo, const uint16_t* K, 
 #define SEMKV_QF(LH, LL, LHV, LLV, GG, CL)                                                                    \
     if (clipped == CL && shi.L == LH && slo.L == LL && shi.Lv == LHV && slo.Lv == LLV && G == GG) {           \
         const size_t sm = (size_t)TILE * QROW * 2;                                                            \
-        const auto kern = k_quantize_fast<LH, LL, LHV, LLV, GG, CL>;                                          \
+        const auto kern = quantize_fast_kernel<LH, LL, LHV, LLV, GG, CL>();                                   \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);                    \
         kern<<<2 * grid, 128, sm, st>>>(qh, ql, K, V, T, clip, status);                                       \
         return;                                                                                               \
