@@ -256,6 +256,18 @@ SEMKV_API int semkv_decode_attention_noalloc(const semkv_cache_t* cache, const u
  * SEMKV_STATUS_LENGTH_MISMATCH and the unit's rows are left as they were). */
 SEMKV_API int semkv_dequantize(const semkv_cache_t* cache, float* K, float* V, int32_t T, void* stream);
 
+/* Self-test of the bounded waits (test hook; the SemKV page has no counterpart).  Every wait in
+ * the library's kernels gives up after a bounded number of tests and then sets
+ * SEMKV_STATUS_TIMEOUT, frees the tensor memory it holds and returns; those waits cannot be made to
+ * fail without breaking a copy or a product, so this call launches one small kernel (one warp)
+ * whose wait nothing completes: one thread arrives on an mbarrier that expects two arrivals and
+ * waits for the phase with at most `tests` tests (1 <= tests <= 65536; each sleeps at most
+ * ~20 us).  use_tmem = 1: the warp allocates 32 tensor-memory columns before the wait and frees
+ * them after it, as the decode kernels do.  On return of the kernel, *status (device int32) has
+ * SEMKV_STATUS_TIMEOUT set.  Returns SEMKV_ERR_INVALID_ARG (null status, tests or use_tmem out of
+ * range) or SEMKV_ERR_CUDA (launch failure). */
+SEMKV_API int semkv_selftest_wait_timeout(int32_t* status, int32_t tests, int32_t use_tmem, void* stream);
+
 /* Name of a host return code (SEMKV_OK ... SEMKV_ERR_CUDA). */
 SEMKV_API const char* semkv_status_string(int code);
 

@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     semkv_p_for_ratio,
     semkv_p_for_ratio_kv,
     semkv_radix_digits,
+    semkv_selftest_wait_timeout,
     semkv_workspace_bytes,
     status_string,
 )

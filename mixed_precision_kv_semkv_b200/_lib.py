@@ -31,7 +31,7 @@ BUF_NAMES = ("k_hi", "v_hi", "kz_hi", "vz_hi", "k_lo", "v_lo", "kz_lo", "vz_lo",
 EXPORTED = ("semkv_cache_bytes", "semkv_workspace_bytes", "semkv_assign_precision", "semkv_quantize_pack",
             "semkv_append_token", "semkv_append_token_running", "semkv_append_decode", "semkv_decode_attention",
             "semkv_decode_attention_noalloc", "semkv_dequantize", "semkv_status_string", "semkv_radix_digits",
-            "semkv_p_for_ratio", "semkv_p_for_ratio_kv", "semkv_capacities")
+            "semkv_p_for_ratio", "semkv_p_for_ratio_kv", "semkv_capacities", "semkv_selftest_wait_timeout")
 NOALLOC_SCRATCH_BYTES = 4 << 20  # SEMKV_NOALLOC_SCRATCH_BYTES
 
 
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
                                            ctypes.POINTER(ctypes.c_double)]
         i32p = ctypes.POINTER(i32)
         L.semkv_capacities.argtypes = [i32, f32, i32, i32, i32p, i32p, i32p, i32p]
+        L.semkv_selftest_wait_timeout.argtypes = [vp, i32, i32, vp]
         for n in EXPORTED:
             if n not in ("semkv_status_string", "semkv_radix_digits"):
                 getattr(L, n).restype = ctypes.c_int
@@ -208,3 +209,10 @@ def semkv_decode_attention_noalloc(cache, q, softmax_scale: float, out, stream=N
 def semkv_dequantize(cache, K, V, T: int, stream=None) -> int:
     return _check("semkv_dequantize",
                   lib().semkv_dequantize(ctypes.byref(_struct(cache)), _ptr(K), _ptr(V), int(T), _stream(stream)))
+
+
+def semkv_selftest_wait_timeout(status, tests: int = 16, use_tmem: bool = True, stream=None) -> None:
+    """Launch the bounded-wait self-test: a kernel whose wait nothing completes gives up after
+    `tests` tests and ORs SEMKV_STATUS_TIMEOUT into `status` (a device int32 tensor of one element)."""
+    _check("semkv_selftest_wait_timeout",
+           lib().semkv_selftest_wait_timeout(_ptr(status), int(tests), 1 if use_tmem else 0, _stream(stream)))

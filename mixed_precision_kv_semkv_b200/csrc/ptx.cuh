@@ -53,11 +53,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase, uint32_
     return ok != 0;
 }
 
-// Wait for the barrier's phase parity; false after 2^16 tests (each sleeps at most ~20 us, so
-// the wait is bounded by about a second).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase)
+// Wait for the barrier's phase parity; false after `tests` tests (by default 2^16; each sleeps at
+// most ~20 us, so the wait is bounded by about a second).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, uint32_t tests = 1u << 16)
 {
-    for (uint32_t i = 0; i < (1u << 16); ++i)
+    for (uint32_t i = 0; i < tests; ++i)
         if (mbar_test(bar, phase, 20000u)) return true;
     return false;
 }

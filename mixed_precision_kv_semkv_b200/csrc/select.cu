@@ -215,9 +215,39 @@ __global__ void __launch_bounds__(1024) k_select(const float* __restrict__ score
 //     each CTA sums all SEL_CS histograms through distributed shared memory and finds the same bin,
 //     so nothing is broadcast;
 //   * the bitmap pass takes the tie and one counts of the earlier CTAs from distributed shared
-//     memory for its prefix sums.
+//     memory for its prefix sums; the four per-CTA counts share one 64-bit block scan.
 
 constexpr int SEL_CS = 8, SEL_THREADS = 512, SEL_WARPS = SEL_THREADS / 32;
+
+// Exclusive scan of 64-bit values over the block (blockDim.x = SEL_THREADS); `tmp` holds 33 words.
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* tmp, uint64_t* total)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint64_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) tmp[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        const uint64_t t = lane < SEL_WARPS ? tmp[lane] : 0ull;
+        uint64_t ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint64_t n = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += n;
+        }
+        tmp[lane] = ti - t;
+        if (lane == 31) tmp[32] = ti;
+    }
+    __syncthreads();
+    const uint64_t r = tmp[wid] + inc - v;
+    *total = tmp[32];
+    __syncthreads();
+    return r;
+}
 
 template <int KPT>
 __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
@@ -241,6 +271,7 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
     __shared__ uint32_t hist[2][256], merged[256];
     __shared__ uint32_t gtm[KPT * SEL_WARPS], eqm[KPT * SEL_WARPS];
     __shared__ uint32_t scan_tmp[33];
+    __shared__ uint64_t scan_tmp64[33];
     __shared__ uint32_t andor[2];   // this CTA's AND and OR of its keys
     __shared__ __align__(16) uint32_t totals[4];  // ties, strictly-greater, window-and-not-greater, window ties
     __shared__ uint32_t sh_prefix, sh_remaining, red_and[SEL_WARPS], red_or[SEL_WARPS];
@@ -372,18 +403,18 @@ __global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
         my_eq = eqm[tid];
     }
     const uint32_t my_win = tid < nw ? window_bits(w0 + tid, T, T - window) : 0u;
-    uint32_t tot_ties, tot_gt, tot_wng = 0u, tot_wt = 0u;
-    uint32_t ties_before = block_excl_scan((uint32_t)__popc(my_eq), scan_tmp, &tot_ties);
-    block_excl_scan((uint32_t)__popc(my_gt), scan_tmp, &tot_gt);
-    if (window > 0) {  // uniform over the cluster
-        block_excl_scan((uint32_t)__popc(my_win & ~my_gt), scan_tmp, &tot_wng);
-        block_excl_scan((uint32_t)__popc(my_win & my_eq), scan_tmp, &tot_wt);
-    }
+    // the four counts of my word as 16-bit fields of one scan (a CTA holds at most
+    // KPT * SEL_THREADS <= 16384 tokens)
+    const uint64_t packed = (uint64_t)__popc(my_eq) | ((uint64_t)__popc(my_gt) << 16) |
+                            ((uint64_t)__popc(my_win & ~my_gt) << 32) | ((uint64_t)__popc(my_win & my_eq) << 48);
+    uint64_t tot4;
+    const uint64_t before4 = block_excl_scan64(packed, scan_tmp64, &tot4);
+    uint32_t ties_before = (uint32_t)(before4 & 0xffffu);
     if (tid == 0) {
-        totals[0] = tot_ties;
-        totals[1] = tot_gt;
-        totals[2] = tot_wng;
-        totals[3] = tot_wt;
+        totals[0] = (uint32_t)(tot4 & 0xffffu);
+        totals[1] = (uint32_t)((tot4 >> 16) & 0xffffu);
+        totals[2] = (uint32_t)((tot4 >> 32) & 0xffffu);
+        totals[3] = (uint32_t)(tot4 >> 48);
     }
     cluster.sync();
     // ones (L_hi tokens) of the earlier CTAs, and of all: CTA r holds gt_r greater keys and takes

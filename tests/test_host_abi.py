@@ -117,6 +117,11 @@ def test_calls_fail_before_any_launch(semkv):
     assert L.semkv_append_decode(ref, one, one, one, nul, sc, one, one, 1 << 30, nul) == 1
     s.L_hi_v = 0
     assert semkv.status_string(3) == "SEMKV_ERR_CAPACITY"
+    # the bounded-wait self-test: null status, test bound or use_tmem out of range
+    assert L.semkv_selftest_wait_timeout(nul, 16, 1, nul) == 1
+    assert L.semkv_selftest_wait_timeout(one, 0, 1, nul) == 1
+    assert L.semkv_selftest_wait_timeout(one, (1 << 16) + 1, 1, nul) == 1
+    assert L.semkv_selftest_wait_timeout(one, 16, 2, nul) == 1
 
 
 @pytest.mark.parametrize("L_hi,L_lo,L_hi_v,L_lo_v", [(8, 5, 3, 2), (16, 8, 5, 4), (6, 4, 256, 17)])
