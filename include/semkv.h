@@ -208,7 +208,13 @@ SEMKV_API int semkv_append_token_running(const semkv_cache_t* cache, const uint1
  * tiles, then a log-sum-exp merge.  q must be 16-byte aligned (its rows are read 16 bytes at a
  * time).  workspace: device buffer of at least semkv_workspace_bytes() bytes (partial softmax
  * states), contents need not be initialized.
- * A unit with no tokens gives zeros. */
+ * A unit with no tokens gives zeros.
+ * Kernels: the integer tensor-core decode (codes as bytes, queries and p s_V as fixed-point limbs)
+ * for level counts 4, 5, 6, 8, 16 with equal K and V counts and at least 8 tiles per warpgroup;
+ * otherwise the fp16 tensor-core decode or, for shapes neither serves, the CUDA-core decode.  The
+ * environment variable SEMKV_DECODE (read at every call, and by semkv_workspace_bytes) overrides
+ * the tile-count rule: "i8" takes the integer decode wherever it serves the shape, "tc" never
+ * takes it.  Size the workspace under the same setting as the call. */
 SEMKV_API int semkv_decode_attention(const semkv_cache_t* cache, const uint16_t* q, float softmax_scale, float* out,
                            void* workspace, size_t workspace_bytes, void* stream);
 

@@ -1,6 +1,8 @@
 // C ABI of libsemkv: argument validation, buffer sizes, split-K choice and kernel launches.
 // Every entry point is documented in include/semkv.h.
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -92,6 +94,19 @@ void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
 // instructions faster than HBM delivers bytes), at least 8 tiles per CTA, and
 // 4 * ctas / units + 2 partial slots per unit and segment (the most workers that can touch one
 // unit).  Otherwise the split-K factors of the other decode kernels.
+constexpr int I8_MIN_TILES = 8;
+
+// SEMKV_DECODE=i8: the integer-MMA decode wherever it serves the shape; =tc: never it (the fp16-MMA
+// or CUDA-core decode); unset or anything else: chosen by the tile count.  Read at every call.
+int decode_path_override()
+{
+    const char* e = std::getenv("SEMKV_DECODE");
+    if (!e) return 0;
+    if (std::strcmp(e, "i8") == 0) return 1;
+    if (std::strcmp(e, "tc") == 0) return 2;
+    return 0;
+}
+
 struct DecodePlan {
     bool i8;
     int ctas_hi, ctas_lo, slots_hi, slots_lo;  // i8
@@ -107,7 +122,16 @@ DecodePlan decode_plan(const semkv_cache_t* c)
     const int th = c->cap_hi / TILE, tl = c->cap_lo / TILE;
     const bool hi_ok = th == 0 || decode_i8_supported(c->L_hi, level_v(*c, true), c->G, g, kpc);
     const bool lo_ok = tl == 0 || decode_i8_supported(c->L_lo, level_v(*c, false), c->G, g, kpc);
-    if (hi_ok && lo_ok && th + tl > 0) {
+    // Fewer than I8_MIN_TILES tiles per warpgroup of the integer-MMA decode: its fixed cost per
+    // warpgroup (query operand, pipeline fill, partial record) outweighs its faster tiles, and the
+    // fp16-MMA decode (one warpgroup per CTA, four CTAs per SM) is faster when it serves the shape
+    // (measured on B200: 2048 and 4096 tiles favour it, 8192 and more the integer decode).
+    const bool tc_ok = (th == 0 || decode_tc_supported(c->L_hi, level_v(*c, true), c->G, g, kpc)) &&
+                       (tl == 0 || decode_tc_supported(c->L_lo, level_v(*c, false), c->G, g, kpc));
+    const bool few = (long long)units * (th + tl) < (long long)I8_MIN_TILES * 4 * sm_count();
+    const int force = decode_path_override();
+    const bool use_i8 = force == 1 ? true : (force == 2 ? false : !(few && tc_ok));
+    if (hi_ok && lo_ok && th + tl > 0 && use_i8) {
         p.i8 = true;
         const int sms = sm_count();
         const double bh = (double)th * (400 + 40 * words_row(c->L_hi)), bl = (double)tl * (400 + 40 * words_row(c->L_lo));

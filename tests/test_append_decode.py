@@ -8,6 +8,14 @@ import pytest
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True, params=["i8", "tc"])
+def decode_path(request, monkeypatch):
+    """Every case through both tensor-core decodes: the integer one ("i8") wherever it serves the
+    shape, and the fp16 one ("tc"); by default the library picks one by the tile count."""
+    monkeypatch.setenv("SEMKV_DECODE", request.param)
+    return request.param
+
+
 def _run(B, H, Hq, T0, steps, G, L_hi, L_lo, p, extra, seed):
     import torch
 

@@ -23,6 +23,14 @@ def _rand_case(B, H, Hq, T, seed, dist="normal"):
     return K.astype(np.float16), V.astype(np.float16), S, q
 
 
+@pytest.fixture(autouse=True, params=["i8", "tc"])
+def decode_path(request, monkeypatch):
+    """Every case through both tensor-core decodes: the integer one ("i8") wherever it serves the
+    shape, and the fp16 one ("tc"); by default the library picks one by the tile count."""
+    monkeypatch.setenv("SEMKV_DECODE", request.param)
+    return request.param
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _built():
     import torch
