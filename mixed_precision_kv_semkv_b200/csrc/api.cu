@@ -96,6 +96,21 @@ void decode_splits(const semkv_cache_t* c, int* ns_hi, int* ns_lo)
 // unit).  Otherwise the split-K factors of the other decode kernels.
 constexpr int I8_MIN_TILES = 8;
 
+// Relative time of one tile of the integer-MMA decode per level count (B200, tiles per SM-second
+// measured with all tokens on one grid, 64 units x 32768 tokens, G64): the code table's digits
+// per lookup and the words per row set it.  The SMs are split between the two segments' grids in
+// proportion to tiles x this cost, so that both grids end together.
+double i8_tile_cost(int L)
+{
+    switch (L) {
+    case 4: return 0.70;
+    case 6: return 1.10;
+    case 8: return 1.02;
+    case 16: return 0.70;
+    default: return 1.0;
+    }
+}
+
 // SEMKV_DECODE=i8: the integer-MMA decode wherever it serves the shape; =tc: never it (the fp16-MMA
 // or CUDA-core decode); unset or anything else: chosen by the tile count.  Read at every call.
 int decode_path_override()
@@ -134,7 +149,7 @@ DecodePlan decode_plan(const semkv_cache_t* c)
     if (hi_ok && lo_ok && th + tl > 0 && use_i8) {
         p.i8 = true;
         const int sms = sm_count();
-        const double bh = (double)th * (400 + 40 * words_row(c->L_hi)), bl = (double)tl * (400 + 40 * words_row(c->L_lo));
+        const double bh = (double)th * i8_tile_cost(c->L_hi), bl = (double)tl * i8_tile_cost(c->L_lo);
         int ch = 0, cl = 0;
         if (th && tl) {
             ch = (int)std::lround(sms * bh / (bh + bl));
