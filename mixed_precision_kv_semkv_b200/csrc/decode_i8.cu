@@ -97,7 +97,11 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     extern __shared__ __align__(1024) unsigned char smem[];
-    const int tid = threadIdx.x, wg = tid >> 7, t = tid & 127, lane = tid & 31, wl = (tid >> 5) & 3;
+    // the warpgroup index through a shuffle from lane 0: the compiler then knows it is the same in
+    // every lane and keeps the shared-memory and TMEM addresses derived from it (the MMA operands)
+    // in uniform registers
+    const int tid = threadIdx.x, wg = __shfl_sync(0xffffffffu, tid >> 7, 0), t = tid & 127, lane = tid & 31,
+              wl = (tid >> 5) & 3;
     const uint32_t bar_id = 1 + (uint32_t)wg;
     auto wg_sync = [&] { named_sync(bar_id, 128); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::LUT_SPAN + 4 * C::WG_SPAN);
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot + (uint32_t)(wg * 128);
+    const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0) + (uint32_t)(wg * 128);
     const uint32_t lane_base = tmem + ((uint32_t)(wl * 32) << 16);
 
     // operand orders: K position t holds channel kch; slot t's V code sits at K position vpos
