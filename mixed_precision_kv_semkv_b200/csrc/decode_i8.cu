@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
     // every lane and keeps the shared-memory and TMEM addresses derived from it (the MMA operands)
     // in uniform registers
     const int tid = threadIdx.x, wg = __shfl_sync(0xffffffffu, tid >> 7, 0), t = tid & 127, lane = tid & 31,
-              wl = (tid >> 5) & 3;
+              wl = __shfl_sync(0xffffffffu, (tid >> 5) & 3, 0);
     const uint32_t bar_id = 1 + (uint32_t)wg;
     auto wg_sync = [&] { named_sync(bar_id, 128); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::LUT_SPAN + 4 * C::WG_SPAN);
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
 
     // operand orders: K position t holds channel kch; slot t's V code sits at K position vpos
     const int kch = row_index<L>(t), vpos = row_pos<L>(t);
-    const int grp_d = t / G;  // group of channel t (uniform over a warp: G >= 32)
+    const int grp_d = wl * 32 / G;  // group of channel t (the same in every lane of the warp: G >= 32)
 
     const int T = pr.seg.tiles_cap, U = pr.units, NW = pr.workers;
     const long long line = (long long)U * T;
@@ -152,11 +152,15 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
     uint32_t ph_qk = 0, ph_pv = 0;
     bool timeout = false;
     int cur_unit = -1;
-    float cK = 0.f, zq[NG][GQ];
+    // per-head values are kept as pairs of heads (h, h + 1) for the packed FP32 instructions
+    constexpr int GP = GQ / 2;
+    static_assert(GQ % 2 == 0, "heads per kv head come in pairs");
+    float cK = 0.f;
+    uint64_t zq[NG][GP];
 #pragma unroll
     for (int g2 = 0; g2 < NG; ++g2)
 #pragma unroll
-        for (int h = 0; h < GQ; ++h) zq[g2][h] = 0.f;
+        for (int h = 0; h < GP; ++h) zq[g2][h] = 0ull;
 
     auto fetch = [&](int unit, int tile, uint32_t n) {  // one thread
         const uint32_t stg = n & 1u;
@@ -285,7 +289,8 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
 #pragma unroll
             for (int g2 = 0; g2 < NG; ++g2)
 #pragma unroll
-                for (int h = 0; h < GQ; ++h) zq[g2][h] = qsm[g2][h] * pr.scale_log2;
+                for (int h = 0; h < GP; ++h)
+                    zq[g2][h] = f2(qsm[g2][2 * h] * pr.scale_log2, qsm[g2][2 * h + 1] * pr.scale_log2);
             wg_sync();  // B_Q complete; red[] free again
         }
 
@@ -306,13 +311,14 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
         // ---------------- the chunk's tiles
         // running maximum of head h in lane h; every thread keeps the sums of its slot and the
         // output of its channel
-        float m_l = NEG_INF, lsum[GQ], O[GQ], zacc[NG][GQ], pa[GQ], pb[GQ];
+        float m_l = NEG_INF;
+        uint64_t lsum[GP], O[GP], zacc[NG][GP], pa[GP], pb[GP];
 #pragma unroll
-        for (int h = 0; h < GQ; ++h) {
-            lsum[h] = O[h] = 0.f;
-            pa[h] = pb[h] = 0.f;
+        for (int h = 0; h < GP; ++h) {
+            lsum[h] = O[h] = 0ull;
+            pa[h] = pb[h] = 0ull;
 #pragma unroll
-            for (int g2 = 0; g2 < NG; ++g2) zacc[g2][h] = 0.f;
+            for (int g2 = 0; g2 < NG; ++g2) zacc[g2][h] = 0ull;
         }
         float psa = 0.f;  // 2^-a of channel t's group for the tile whose p.V is in flight
         if (!fetch_early) fetch_first();
@@ -325,11 +331,14 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
             uint32_t dv[32];
             tmem_ld_n<4 * GQ>(lane_base + C::COL_DV + (uint32_t)(grp_d * 4 * GQ), dv);
             tc_wait_ld();
+            const uint64_t psa2 = f2(psa, psa), c16 = f2(65536.f, 65536.f);
 #pragma unroll
-            for (int h = 0; h < GQ; ++h) {
-                const int a01 = (int)dv[4 * h] + ((int)dv[4 * h + 1] << 8);
-                const float v = fmaf((float)(int)dv[4 * h + 2], 65536.f, (float)a01);
-                O[h] = fmaf(v * psa, pb[h], O[h] * pa[h]);
+            for (int h = 0; h < GP; ++h) {
+                const int a0 = (int)dv[8 * h] + ((int)dv[8 * h + 1] << 8);
+                const int a1 = (int)dv[8 * h + 4] + ((int)dv[8 * h + 5] << 8);
+                const uint64_t v = fma2(f2((float)(int)dv[8 * h + 2], (float)(int)dv[8 * h + 6]), c16,
+                                        f2((float)a0, (float)a1));
+                O[h] = fma2(mul2(v, psa2), pb[h], mul2(O[h], pa[h]));
             }
         };
         auto wait_stage = [&](uint32_t nfetch) {
@@ -379,15 +388,18 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
                 tc_wait_ld();
                 float lg[GQ];
 #pragma unroll
-                for (int h = 0; h < GQ; ++h) {
-                    float acc = 0.f;
+                for (int h = 0; h < GP; ++h) {
+                    uint64_t acc = 0ull;
 #pragma unroll
                     for (int g2 = 0; g2 < NG; ++g2) {
-                        const int n0 = g2 * 3 * GQ + h;
-                        const int qc = (int)dk[n0] + ((int)dk[n0 + GQ] << 8) + ((int)dk[n0 + 2 * GQ] << 16);
-                        acc = fmaf(sK[g2], (float)qc, fmaf(zK[g2], zq[g2][h], acc));
+                        const int n0 = g2 * 3 * GQ + 2 * h;
+                        const int q0 = (int)dk[n0] + ((int)dk[n0 + GQ] << 8) + ((int)dk[n0 + 2 * GQ] << 16);
+                        const int q1 = (int)dk[n0 + 1] + ((int)dk[n0 + 1 + GQ] << 8) + ((int)dk[n0 + 1 + 2 * GQ] << 16);
+                        acc = fma2(f2(sK[g2], sK[g2]), f2((float)q0, (float)q1),
+                                   fma2(f2(zK[g2], zK[g2]), zq[g2][h], acc));
                     }
-                    lg[h] = valid ? acc : NEG_INF;
+                    lg[2 * h] = valid ? f2lo(acc) : NEG_INF;
+                    lg[2 * h + 1] = valid ? f2hi(acc) : NEG_INF;
                 }
                 // ---- tile maxima: logits per head, V scales per group
 #pragma unroll
@@ -425,19 +437,26 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
                 uint32_t wd[NV / 4];
 #pragma unroll
                 for (int i2 = 0; i2 < NV / 4; ++i2) wd[i2] = 0u;
+                const uint64_t magic = f2(8388608.f, 8388608.f);
 #pragma unroll
-                for (int h = 0; h < GQ; ++h) {
-                    const float mh = __shfl_sync(0xffffffffu, x0, h), alh = __shfl_sync(0xffffffffu, x1, h);
-                    const float p = valid ? ex2_approx(lg[h] - mh) : 0.f;
-                    lsum[h] = fmaf(lsum[h], alh, p);
+                for (int h = 0; h < GP; ++h) {
+                    const uint64_t mh = f2(__shfl_sync(0xffffffffu, x0, 2 * h), __shfl_sync(0xffffffffu, x0, 2 * h + 1));
+                    const uint64_t alh = f2(__shfl_sync(0xffffffffu, x1, 2 * h), __shfl_sync(0xffffffffu, x1, 2 * h + 1));
+                    const uint64_t d = sub2(f2(lg[2 * h], lg[2 * h + 1]), mh);
+                    const uint64_t p = f2(valid ? ex2_approx(f2lo(d)) : 0.f, valid ? ex2_approx(f2hi(d)) : 0.f);
+                    lsum[h] = fma2(lsum[h], alh, p);
 #pragma unroll
-                    for (int g2 = 0; g2 < NG; ++g2) zacc[g2][h] = fmaf(p, zV[g2], zacc[g2][h] * alh);
-                    const float p2 = p * __shfl_sync(0xffffffffu, x2, h);
+                    for (int g2 = 0; g2 < NG; ++g2) zacc[g2][h] = fma2(p, f2(zV[g2], zV[g2]), mul2(zacc[g2][h], alh));
+                    const uint64_t p2 =
+                        mul2(p, f2(__shfl_sync(0xffffffffu, x2, 2 * h), __shfl_sync(0xffffffffu, x2, 2 * h + 1)));
 #pragma unroll
-                    for (int g2 = 0; g2 < NG; ++g2)
-                        wd[g2 * GQ + h] = __float_as_uint(fmaf(p2, sVa[g2], 8388608.f)) & 0x7FFFFFu;
+                    for (int g2 = 0; g2 < NG; ++g2) {
+                        const uint64_t y = fma2(p2, f2(sVa[g2], sVa[g2]), magic);
+                        wd[g2 * GQ + 2 * h] = (uint32_t)y & 0x7FFFFFu;
+                        wd[g2 * GQ + 2 * h + 1] = (uint32_t)(y >> 32) & 0x7FFFFFu;
+                    }
                     pa[h] = alh;
-                    pb[h] = __shfl_sync(0xffffffffu, x3, h);
+                    pb[h] = f2(__shfl_sync(0xffffffffu, x3, 2 * h), __shfl_sync(0xffffffffu, x3, 2 * h + 1));
                 }
                 // my slot's row of B_P (K position vpos), 16 bytes per MN core-matrix row
 #pragma unroll
@@ -474,11 +493,11 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
         // ---------------- the chunk's partial state -> its workspace slot
         float vals[GQ + NG * GQ];
 #pragma unroll
-        for (int h = 0; h < GQ; ++h) vals[h] = lsum[h];
+        for (int h = 0; h < GQ; ++h) vals[h] = h & 1 ? f2hi(lsum[h >> 1]) : f2lo(lsum[h >> 1]);
 #pragma unroll
         for (int g2 = 0; g2 < NG; ++g2)
 #pragma unroll
-            for (int h = 0; h < GQ; ++h) vals[GQ + g2 * GQ + h] = zacc[g2][h];
+            for (int h = 0; h < GQ; ++h) vals[GQ + g2 * GQ + h] = h & 1 ? f2hi(zacc[g2][h >> 1]) : f2lo(zacc[g2][h >> 1]);
         tc_fence_before();
         wg_sync();  // every thread is past its reads of red[]
 #pragma unroll
@@ -497,7 +516,7 @@ __global__ void __launch_bounds__(512, 1) k_decode_i8(const I8Params pr)
         for (int h = 0; h < GQ; ++h) {
             const int zi = GQ + grp_d * GQ + h;
             const float zs = red[zi] + red[16 + zi] + red[32 + zi] + red[48 + zi];
-            rec[h * (D + 2) + t] = O[h] + zs;
+            rec[h * (D + 2) + t] = (h & 1 ? f2hi(O[h >> 1]) : f2lo(O[h >> 1])) + zs;
             const float mh = __shfl_sync(0xffffffffu, m_l, h);
             if (t == 0) {
                 rec[h * (D + 2) + D] = mh;

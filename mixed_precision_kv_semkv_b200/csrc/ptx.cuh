@@ -252,6 +252,34 @@ __device__ __forceinline__ float ex2_approx(float x)
 
 namespace semkv {
 
+// ------------------------------------------------------------------ packed FP32 (two lanes per instruction)
+
+// (lo, hi) as one 64-bit register pair; each packed operation rounds each lane as its scalar form
+__device__ __forceinline__ uint64_t f2(float lo, float hi)
+{
+    return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // ------------------------------------------------------------------ integer tensor cores, wide TMEM moves
 
 // D[tmem] (+)= A[tmem] x B[smem desc], kind::i8 (8-bit integer operands, s32 accumulators), issued
