@@ -156,7 +156,9 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int split = blockIdx.x, u = blockIdx.y, b = u / H, hk = u % H, Hq = H * GQ;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // the warp index through a shuffle from lane 0: the compiler then keeps the addresses derived
+    // from it (TMEM lanes, MMA operands) in uniform registers
+    const int tid = threadIdx.x, lane = tid & 31, warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
 
     extern __shared__ __align__(1024) unsigned char smem[];
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::LUT_K);
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(128, 4) k_decode_tc(SegView seg, const uint16_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = tmem_base_s;
+    const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_base_s, 0);
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     constexpr uint32_t idesc_k = idesc_f16_f32(128, NK), idesc_v = idesc_f16_f32(128, NV);
     const uint32_t bq_addr = smem_u32(bq), bp_addr = smem_u32(bp);
